@@ -1,0 +1,228 @@
+// abi.cu -- the C ABI of libentmax_attn.so (declared and documented in
+// include/entmax_attn.h): argument checks, workspace layout, TMA descriptors, launches.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/entmax_attn.h"
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace entmax;
+
+namespace {
+
+constexpr int kDefaultSweeps = 12;
+constexpr int kMaxSweeps = 64;
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct Layout {
+  int BH, Tr, Tc, Wc, Wr;
+  size_t off_status, off_M, off_MT, off_sumg, off_Ot, off_delta, off_sweeps, total;
+  size_t bytes_M, bytes_MT, bytes_sweeps;
+};
+
+bool layout_of(const entmax_attn_desc* d, Layout* l) {
+  l->BH = d->B * d->H;
+  l->Tr = (d->L + kTile - 1) / kTile;
+  l->Tc = l->Tr;
+  l->Wc = (l->Tc + 31) / 32;
+  l->Wr = (l->Tr + 31) / 32;
+  const size_t rows = (size_t)l->BH * d->L;
+  size_t off = 0;
+  l->off_status = off;
+  off += 256;
+  l->off_M = off;
+  l->bytes_M = (size_t)l->BH * l->Tr * l->Wc * 4;
+  off += align256(l->bytes_M);
+  l->off_MT = off;
+  l->bytes_MT = (size_t)l->BH * l->Tc * l->Wr * 4;
+  off += align256(l->bytes_MT);
+  l->off_sumg = off;
+  off += align256(rows * 4);
+  l->off_Ot = off;
+  off += align256(rows * kD * 4);
+  l->off_delta = off;
+  off += align256(rows * 4);
+  l->off_sweeps = off;
+  l->bytes_sweeps = (size_t)l->BH * l->Tr * 4;
+  off += align256(l->bytes_sweeps);
+  l->total = off;
+  return true;
+}
+
+entmax_status check_desc(const entmax_attn_desc* d) {
+  if (!d) return ENTMAX_EINVAL;
+  if (d->B < 1 || d->H < 1 || d->L < 1 || d->d < 1) return ENTMAX_EINVAL;
+  if ((long long)d->B * d->H * d->L > (1ll << 31)) return ENTMAX_EINVAL;
+  if (!(d->scale > 0.f) || !std::isfinite(d->scale)) return ENTMAX_EINVAL;
+  if (d->causal != 0 && d->causal != 1) return ENTMAX_EINVAL;
+  if (d->max_sweeps < 0 || d->max_sweeps > kMaxSweeps) return ENTMAX_EINVAL;
+  if (d->dtype != ENTMAX_BF16 && d->dtype != ENTMAX_FP32) return ENTMAX_EINVAL;
+  if (d->d != kD) return ENTMAX_EUNSUPPORTED;
+  if (d->L > ENTMAX_MAX_L) return ENTMAX_EUNSUPPORTED;
+  if (d->alpha != 1.5f && d->alpha != 2.0f) return ENTMAX_EUNSUPPORTED;
+  if (d->dtype == ENTMAX_FP32) return ENTMAX_EUNSUPPORTED;
+  return ENTMAX_OK;
+}
+
+bool aligned(const void* p, size_t a) { return p && (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// bf16 [BH][L][64] viewed as a 3-D tensor; box = one 128 x 64 tile, 128-byte swizzle.
+// Rows past L read as zeros.
+bool make_map(CUtensorMap* m, const void* base, int L, int BH) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)L, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)L * kD * 2};
+  cuuint32_t box[3] = {(cuuint32_t)kD, (cuuint32_t)kTile, 1}, es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+extern "C" size_t entmax_attn_workspace_bytes(const entmax_attn_desc* d) {
+  if (check_desc(d) != ENTMAX_OK) return 0;
+  Layout l;
+  layout_of(d, &l);
+  return l.total;
+}
+
+extern "C" entmax_status entmax_attn_fwd(const entmax_attn_desc* d, const void* Q, const void* K, const void* V,
+                                         float* O, float* tau, void* ws, void* stream) {
+  entmax_status st = check_desc(d);
+  if (st != ENTMAX_OK) return st;
+  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(O, 16) || !aligned(tau, 4) ||
+      !aligned(ws, 256))
+    return ENTMAX_EINVAL;
+  Layout l;
+  layout_of(d, &l);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  FwdParams p;
+  std::memset(&p, 0, sizeof(p));
+  if (!make_map(&p.tQ, Q, d->L, l.BH) || !make_map(&p.tK, K, d->L, l.BH) || !make_map(&p.tV, V, d->L, l.BH))
+    return ENTMAX_ECUDA;
+  p.O = O;
+  p.tau = tau;
+  p.sumg = reinterpret_cast<float*>(w + l.off_sumg);
+  p.Ot = reinterpret_cast<float*>(w + l.off_Ot);
+  p.M = reinterpret_cast<uint32_t*>(w + l.off_M);
+  p.MT = reinterpret_cast<uint32_t*>(w + l.off_MT);
+  p.sweeps = reinterpret_cast<int*>(w + l.off_sweeps);
+  p.status = reinterpret_cast<int*>(w + l.off_status);
+  p.kv_len = d->kv_len;
+  p.H = d->H;
+  p.L = d->L;
+  p.Tr = l.Tr;
+  p.Tc = l.Tc;
+  p.Wc = l.Wc;
+  p.Wr = l.Wr;
+  p.BH = l.BH;
+  p.cz = (d->alpha - 1.0f) * d->scale;
+  p.causal = d->causal || d->window >= 0;
+  p.window = d->window < 0 ? -1 : d->window;
+  p.max_sweeps = d->max_sweeps == 0 ? kDefaultSweeps : d->max_sweeps;
+  if (cudaMemsetAsync(w + l.off_status, 0, 256, s) != cudaSuccess) return ENTMAX_ECUDA;
+  if (cudaMemsetAsync(p.MT, 0, l.bytes_MT, s) != cudaSuccess) return ENTMAX_ECUDA;
+  return launch_fwd(d->alpha == 1.5f, p, l.BH * l.Tr, s) == cudaSuccess ? ENTMAX_OK : ENTMAX_ECUDA;
+}
+
+extern "C" entmax_status entmax_attn_bwd(const entmax_attn_desc* d, const void* Q, const void* K, const void* V,
+                                         const void* dO, const float* tau, void* ws, float* dQ, float* dK,
+                                         float* dV, void* stream) {
+  entmax_status st = check_desc(d);
+  if (st != ENTMAX_OK) return st;
+  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(dO, 16) || !aligned(tau, 4) ||
+      !aligned(ws, 256) || !aligned(dQ, 16) || !aligned(dK, 16) || !aligned(dV, 16))
+    return ENTMAX_EINVAL;
+  Layout l;
+  layout_of(d, &l);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  BwdParams p;
+  std::memset(&p, 0, sizeof(p));
+  if (!make_map(&p.tQ, Q, d->L, l.BH) || !make_map(&p.tK, K, d->L, l.BH) || !make_map(&p.tV, V, d->L, l.BH) ||
+      !make_map(&p.tdO, dO, d->L, l.BH))
+    return ENTMAX_ECUDA;
+  float* delta = reinterpret_cast<float*>(w + l.off_delta);
+  p.tau = tau;
+  p.delta = delta;
+  p.MT = reinterpret_cast<const uint32_t*>(w + l.off_MT);
+  p.dQ = dQ;
+  p.dK = dK;
+  p.dV = dV;
+  p.status = reinterpret_cast<int*>(w + l.off_status);
+  p.kv_len = d->kv_len;
+  p.H = d->H;
+  p.L = d->L;
+  p.Tr = l.Tr;
+  p.Tc = l.Tc;
+  p.Wr = l.Wr;
+  p.BH = l.BH;
+  p.cz = (d->alpha - 1.0f) * d->scale;
+  p.scale = d->scale;
+  p.causal = d->causal || d->window >= 0;
+  p.window = d->window < 0 ? -1 : d->window;
+  const long rows = (long)l.BH * d->L;
+  if (cudaMemsetAsync(dQ, 0, (size_t)rows * kD * 4, s) != cudaSuccess) return ENTMAX_ECUDA;
+  if (launch_delta(static_cast<const uint16_t*>(dO), reinterpret_cast<const float*>(w + l.off_Ot),
+                   reinterpret_cast<const float*>(w + l.off_sumg), delta, rows, s) != cudaSuccess)
+    return ENTMAX_ECUDA;
+  return launch_bwd(d->alpha == 1.5f, p, l.BH * l.Tc, s) == cudaSuccess ? ENTMAX_OK : ENTMAX_ECUDA;
+}
+
+extern "C" entmax_status entmax_rows(const float* S, int rows, int n, int ld, float alpha, float* P, float* tau,
+                                     void* stream) {
+  if (rows < 0 || n < 1 || ld < n || (ld % 4) != 0) return ENTMAX_EINVAL;
+  if (alpha != 1.5f && alpha != 2.0f) return ENTMAX_EUNSUPPORTED;
+  if (rows == 0) return ENTMAX_OK;
+  if (!aligned(S, 16) || !aligned(P, 16) || !aligned(tau, 4)) return ENTMAX_EINVAL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return launch_rows(alpha == 1.5f, S, rows, n, ld, P, tau, s) == cudaSuccess ? ENTMAX_OK : ENTMAX_ECUDA;
+}
+
+extern "C" entmax_status entmax_last_device_status(const entmax_attn_desc* d, const void* ws, int* status_out,
+                                                   void* stream) {
+  if (check_desc(d) != ENTMAX_OK || !aligned(ws, 256) || !status_out) return ENTMAX_EINVAL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return ENTMAX_ECUDA;
+  int word = 0;
+  if (cudaMemcpy(&word, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return ENTMAX_ECUDA;
+  *status_out = word;
+  if (word & kStatusTimeout) return ENTMAX_ETIMEOUT;
+  if (word & kStatusNoConverge) return ENTMAX_ENOCONVERGE;
+  return ENTMAX_OK;
+}
+
+extern "C" entmax_status entmax_attn_block_mask(const entmax_attn_desc* d, const void* ws, uint32_t* M,
+                                                int* sweeps, void* stream) {
+  if (check_desc(d) != ENTMAX_OK || !aligned(ws, 256)) return ENTMAX_EINVAL;
+  Layout l;
+  layout_of(d, &l);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const uint8_t* w = static_cast<const uint8_t*>(ws);
+  if (M && cudaMemcpyAsync(M, w + l.off_M, l.bytes_M, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    return ENTMAX_ECUDA;
+  if (sweeps && cudaMemcpyAsync(sweeps, w + l.off_sweeps, l.bytes_sweeps, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    return ENTMAX_ECUDA;
+  return ENTMAX_OK;
+}

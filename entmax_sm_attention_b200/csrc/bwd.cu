@@ -1,0 +1,335 @@
+// bwd.cu -- fused alpha-entmax attention backward for sm_100a.
+//
+// "AdaSplash-2: Faster Differentiable Sparse Attention", §3.3 "Backward pass" and
+// Appendix C.6: gradients are nonzero only on the entmax support, so the backward
+// visits only the (query tile, key tile) blocks the forward flagged, through the
+// transposed block mask. The Jacobian is not printed on the pages. From Eq. 3,
+// implicit differentiation of sum_j p_j = 1 gives dp_j/ds_k = g_j delta_jk - g_j g_k /
+// sum g, with g = p^{2-alpha}. Per element that yields
+//   dS_ij = g_ij (dA_ij - delta_i),  dA_ij = dO_i . V_j,  delta_i = dO_i . Ot_i / sum_j g_ij
+// and dQ = scale dS K, dK = scale dS^T Q, dV = A^T dO.
+//
+// One CTA per (batch*head, 128-key tile). K_j and V_j stay in shared memory; the
+// flagged query tiles stream through a 2-stage ring of (Q_i, dO_i). Per query tile the
+// tensor cores compute S = Q_i K_j^T and dA = dO_i V_j^T into TMEM (M = queries).
+// Warps 0-3 (one query row per thread) form A and dS as two-term bf16 splits
+// (hi + lo, about fp32 accuracy in the products) into swizzled shared-memory buffers.
+// Those buffers then feed dV += A^T dO_i and dK += dS^T Q_i as MN-major operands
+// (M = keys, accumulated in TMEM), and dQ_i = dS K_j as a K-major operand
+// (double-buffered in TMEM). The row owners add dQ_i to global memory with
+// vector reductions. TMEM: [0,128) S, [128,256) dA, [256,320) dV, [320,384) dK,
+// [384,512) dQ x2.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace entmax {
+
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kStages = 2;
+constexpr int kPairBytes = 2 * kTileBytes;   // Q_i and dO_i
+
+struct Shared {
+  uint64_t full[kStages], empty[kStages];
+  uint64_t bar_kv, s_full, p_ready, mma2_done;
+  uint32_t tmem_base;
+  int abort_flag;
+  uint32_t qlist[kMaskWords];
+};
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+
+}  // namespace
+
+int bwd_smem_bytes() { return 1024 + 2 * kTileBytes + kStages * kPairBytes + 8 * kTileBytes; }
+
+template <int AK>
+__global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant__ BwdParams p) {
+  extern __shared__ uint8_t dsm_raw[];
+  __shared__ Shared sh;
+  uint8_t* dsm = align1024(dsm_raw);
+  uint8_t* sK = dsm;
+  uint8_t* sV = dsm + kTileBytes;
+  uint8_t* ring = dsm + 2 * kTileBytes;                       // stage s: Q at +0, dO at +16 KB
+  // [128 q][128 k] bf16 matrices, each as 2 swizzled panels of 64 keys: A hi, A lo, dS hi, dS lo
+  uint8_t* sA = ring + kStages * kPairBytes;
+  uint8_t* sAl = sA + 2 * kTileBytes;
+  uint8_t* sdS = sAl + 2 * kTileBytes;
+  uint8_t* sdSl = sdS + 2 * kTileBytes;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int bh = blockIdx.x % p.BH;
+  const int kt = blockIdx.x / p.BH;          // key tile (low key tiles have the most query tiles)
+  const int b = bh / p.H;
+  const Pattern pat{p.L, p.kv_len ? min(max(p.kv_len[b], 1), p.L) : p.L, p.causal, p.window};
+  const int j0 = kt * kTile;
+  int* status = p.status;
+  volatile int* abrt = &sh.abort_flag;
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sh.full[s], 1);
+      mbar_init(&sh.empty[s], 1);
+    }
+    mbar_init(&sh.bar_kv, 1);
+    mbar_init(&sh.s_full, 1);
+    mbar_init(&sh.p_ready, 4);
+    mbar_init(&sh.mma2_done, 1);
+    sh.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (tid < kMaskWords) sh.qlist[tid] = (tid < p.Wr) ? p.MT[((size_t)bh * p.Tc + kt) * p.Wr + tid] : 0u;
+  if (warp == 5) {
+    tmem_alloc(&sh.tmem_base, 512);
+    tmem_relinquish();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t T = sh.tmem_base;
+  uint32_t qlist[kMaskWords];
+#pragma unroll
+  for (int w = 0; w < kMaskWords; ++w) qlist[w] = sh.qlist[w];
+  int nq = 0;
+#pragma unroll
+  for (int w = 0; w < kMaskWords; ++w) nq += __popc(qlist[w]);
+
+  if (warp == 4) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0 && nq > 0) {
+      tma_prefetch_desc(&p.tQ);
+      tma_prefetch_desc(&p.tdO);
+      mbar_expect_tx(&sh.bar_kv, 2 * kTileBytes);
+      tma_load_3d(sK, &p.tK, &sh.bar_kv, 0, j0, bh);
+      tma_load_3d(sV, &p.tV, &sh.bar_kv, 0, j0, bh);
+      uint32_t seq = 0;
+      for_each_bit(qlist, kMaskWords, [&](int it) {
+        const int st = seq % kStages;
+        mbar_wait(&sh.empty[st], ((seq / kStages) & 1) ^ 1, status, abrt);
+        mbar_expect_tx(&sh.full[st], kPairBytes);
+        tma_load_3d(ring + st * kPairBytes, &p.tQ, &sh.full[st], 0, it * kTile, bh);
+        tma_load_3d(ring + st * kPairBytes + kTileBytes, &p.tdO, &sh.full[st], 0, it * kTile, bh);
+        ++seq;
+      });
+      volatile int no_abort = 0;
+      for (uint32_t k = (seq > kStages ? seq - kStages : 0); k < seq; ++k)
+        mbar_wait(&sh.full[k % kStages], (k / kStages) & 1, status, &no_abort);
+    }
+    __syncwarp();
+  } else if (warp == 5) {
+    // ------------------------------------------------------------------- MMA issuer
+    if (lane == 0 && nq > 0) {
+      const uint32_t id128 = idesc_bf16(128, 128, 0, 0);
+      const uint32_t idMN = idesc_bf16(128, 64, 1, 1);   // A MN-major (from sA/sdS), B MN-major
+      const uint32_t idQ = idesc_bf16(128, 64, 0, 1);    // A K-major (sdS), B MN-major (K_j)
+      const uint32_t kA = smem_u32(sK), vA = smem_u32(sV);
+      const uint32_t aH = smem_u32(sA), aL = smem_u32(sAl), dH = smem_u32(sdS), dL = smem_u32(sdSl);
+      mbar_wait(&sh.bar_kv, 0, status, abrt);
+      uint32_t seq = 0;
+      for_each_bit(qlist, kMaskWords, [&](int) {
+        const int st = seq % kStages;
+        const uint32_t qA = smem_u32(ring + st * kPairBytes), oA = qA + kTileBytes;
+        // S and dA of the previous step were consumed before its p_ready, waited below.
+        mbar_wait(&sh.full[st], (seq / kStages) & 1, status, abrt);
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          mma_ss(T, sdesc_sw128(qA + k * 32, 16, 1024), sdesc_sw128(kA + k * 32, 16, 1024), id128, k > 0);
+          mma_ss(T + 128, sdesc_sw128(oA + k * 32, 16, 1024), sdesc_sw128(vA + k * 32, 16, 1024), id128, k > 0);
+        }
+        mma_commit(&sh.s_full);
+        mbar_wait(&sh.p_ready, seq & 1, status, abrt);   // A and dS in shared memory
+        tc_fence_after();
+        const uint32_t dq = T + 384 + (seq & 1) * 64;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          // dV += A^T dO_i and dK += dS^T Q_i: K = queries (16 per step), M = keys.
+          const uint32_t acc = (seq > 0 || t > 0) ? 1u : 0u;
+          const uint64_t bO = sdesc_sw128(oA + t * 2048, 8192, 1024), bQ = sdesc_sw128(qA + t * 2048, 8192, 1024);
+          mma_ss(T + 256, sdesc_sw128(aH + t * 2048, 16384, 1024), bO, idMN, acc);
+          mma_ss(T + 256, sdesc_sw128(aL + t * 2048, 16384, 1024), bO, idMN, 1u);
+          mma_ss(T + 320, sdesc_sw128(dH + t * 2048, 16384, 1024), bQ, idMN, acc);
+          mma_ss(T + 320, sdesc_sw128(dL + t * 2048, 16384, 1024), bQ, idMN, 1u);
+          // dQ_i = dS K_j: K = keys (16 per step; panel t/4), M = queries.
+          const uint32_t koff = (t >> 2) * kTileBytes + (t & 3) * 32;
+          const uint64_t bK = sdesc_sw128(kA + t * 2048, 8192, 1024);
+          mma_ss(dq, sdesc_sw128(dH + koff, 16, 1024), bK, idQ, t > 0 ? 1u : 0u);
+          mma_ss(dq, sdesc_sw128(dL + koff, 16, 1024), bK, idQ, 1u);
+        }
+        mma_commit(&sh.empty[st]);
+        mma_commit(&sh.mma2_done);
+        ++seq;
+      });
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- row owners
+    const int row = tid;
+    const uint32_t tl = T + ((uint32_t)(warp * 32) << 16);
+    const float cz = p.cz;
+    uint32_t seq = 0;
+    int prev_i = -1;
+    // Adds dQ of the query tile handled at step `s` (TMEM buffer s & 1) to global memory.
+    // Each mma2_done phase is waited on exactly once: inside the loop the wait before
+    // the shared-memory writes of step s+1 already covers step s.
+    auto flush_dq = [&](uint32_t s, int irow, bool wait) {
+      if (wait) warp_wait(&sh.mma2_done, s & 1, status, abrt);
+      tc_fence_after();
+      const uint32_t dq = tl + 384 + (s & 1) * 64;
+      uint32_t a[32], c[32];
+      tmem_ld32(dq, a);
+      tmem_ld32(dq + 32, c);
+      tmem_wait_ld();
+      if (irow < p.L) {
+        float* dst = p.dQ + ((size_t)bh * p.L + irow) * kD;
+        const float sc = p.scale;
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          red_add_v4(dst + 4 * k, sc * __uint_as_float(a[4 * k]), sc * __uint_as_float(a[4 * k + 1]),
+                     sc * __uint_as_float(a[4 * k + 2]), sc * __uint_as_float(a[4 * k + 3]));
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          red_add_v4(dst + 32 + 4 * k, sc * __uint_as_float(c[4 * k]), sc * __uint_as_float(c[4 * k + 1]),
+                     sc * __uint_as_float(c[4 * k + 2]), sc * __uint_as_float(c[4 * k + 3]));
+      }
+      __syncwarp();
+    };
+    for_each_bit(qlist, kMaskWords, [&](int it) {
+      const int i = it * kTile + row;
+      const bool valid = i < p.L;
+      const float tau = valid ? p.tau[(size_t)bh * p.L + i] : INFINITY;
+      const float dl = valid ? p.delta[(size_t)bh * p.L + i] : 0.f;
+      const bool full = pat.block_full(it * kTile, min(p.L, it * kTile + kTile), j0, j0 + kTile);
+      warp_wait(&sh.s_full, seq & 1, status, abrt);
+      // The previous tile's dV/dK/dQ MMAs must be done reading sA / sdS.
+      if (seq > 0) warp_wait(&sh.mma2_done, (seq - 1) & 1, status, abrt);
+      tc_fence_after();
+#pragma unroll 1
+      for (int q = 0; q < 4; ++q) {
+        uint32_t sr[32], ar[32];
+        tmem_ld32(tl + q * 32, sr);
+        tmem_ld32(tl + 128 + q * 32, ar);
+        tmem_wait_ld();
+        uint32_t ah[16], al[16], dh[16], dl2[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          float s0 = __uint_as_float(sr[2 * c]), s1 = __uint_as_float(sr[2 * c + 1]);
+          if (!full) {
+            const int jj = j0 + q * 32 + 2 * c;
+            if (!pat.active(i, jj)) s0 = -INFINITY;
+            if (!pat.active(i, jj + 1)) s1 = -INFINITY;
+          }
+          const float u0 = fmaf(s0, cz, -tau), u1 = fmaf(s1, cz, -tau);
+          const float v0 = fmaxf(u0, 0.f), v1 = fmaxf(u1, 0.f);
+          const float d0 = __uint_as_float(ar[2 * c]) - dl, d1 = __uint_as_float(ar[2 * c + 1]) - dl;
+          if (AK == kAlpha15) {
+            split_bf16x2(v0 * v0, v1 * v1, ah[c], al[c]);
+            split_bf16x2(v0 * d0, v1 * d1, dh[c], dl2[c]);
+          } else {
+            split_bf16x2(v0, v1, ah[c], al[c]);
+            split_bf16x2(u0 > 0.f ? d0 : 0.f, u1 > 0.f ? d1 : 0.f, dh[c], dl2[c]);
+          }
+        }
+        // Keys q*32 .. q*32+31 -> panel q/2, 16-byte chunks (q%2)*4 .. +3 of row `row`.
+        const int pan = (q >> 1) * kTileBytes;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t off = pan + sw128_offset(row, (q & 1) * 32 + k * 8);
+          *reinterpret_cast<uint4*>(sA + off) = make_uint4(ah[4 * k], ah[4 * k + 1], ah[4 * k + 2], ah[4 * k + 3]);
+          *reinterpret_cast<uint4*>(sAl + off) = make_uint4(al[4 * k], al[4 * k + 1], al[4 * k + 2], al[4 * k + 3]);
+          *reinterpret_cast<uint4*>(sdS + off) = make_uint4(dh[4 * k], dh[4 * k + 1], dh[4 * k + 2], dh[4 * k + 3]);
+          *reinterpret_cast<uint4*>(sdSl + off) =
+              make_uint4(dl2[4 * k], dl2[4 * k + 1], dl2[4 * k + 2], dl2[4 * k + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      warp_arrive(&sh.p_ready);
+      if (seq > 0) flush_dq(seq - 1, prev_i, false);
+      prev_i = i;
+      ++seq;
+    });
+    if (seq > 0) flush_dq(seq - 1, prev_i, true);
+    // dK and dV of this key tile (TMEM lane = key). Every lane executes the TMEM loads
+    // (.sync.aligned); only the global stores depend on the key being inside L.
+    const int j = j0 + row;
+    const bool jvalid = j < p.L;
+    float* dk = p.dK + ((size_t)bh * p.L + (jvalid ? j : 0)) * kD;
+    float* dv = p.dV + ((size_t)bh * p.L + (jvalid ? j : 0)) * kD;
+    const float sc = p.scale;
+    for (int h = 0; h < 2; ++h) {
+      uint32_t a[32], c[32];
+      if (seq > 0) {
+        tmem_ld32(tl + 256 + h * 32, a);
+        tmem_ld32(tl + 320 + h * 32, c);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int k = 0; k < 32; ++k) a[k] = c[k] = 0u;
+      }
+      if (jvalid) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          reinterpret_cast<float4*>(dv + h * 32)[k] =
+              make_float4(__uint_as_float(a[4 * k]), __uint_as_float(a[4 * k + 1]), __uint_as_float(a[4 * k + 2]),
+                          __uint_as_float(a[4 * k + 3]));
+          reinterpret_cast<float4*>(dk + h * 32)[k] =
+              make_float4(sc * __uint_as_float(c[4 * k]), sc * __uint_as_float(c[4 * k + 1]),
+                          sc * __uint_as_float(c[4 * k + 2]), sc * __uint_as_float(c[4 * k + 3]));
+        }
+      }
+      __syncwarp();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) tmem_dealloc(T, 512);
+}
+
+cudaError_t launch_bwd(bool alpha15, const BwdParams& p, int grid, cudaStream_t s) {
+  const int smem = bwd_smem_bytes();
+  auto kern = alpha15 ? bwd_kernel<kAlpha15> : bwd_kernel<kAlpha2>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kThreads, smem, s>>>(p);
+  return cudaGetLastError();
+}
+
+// delta_i = dO_i . Ot_i / sum_j g_ij for every row (the backward's per-row scalar).
+__global__ void bwd_delta_kernel(const uint16_t* __restrict__ dO, const float* __restrict__ Ot,
+                                 const float* __restrict__ sumg, float* __restrict__ delta, long rows) {
+  const long r = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (r >= rows) return;
+  const uint4* d = reinterpret_cast<const uint4*>(dO + r * kD);
+  const float4* o = reinterpret_cast<const float4*>(Ot + r * kD);
+  float acc = 0.f;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const uint4 w = d[k];
+    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float lo = __uint_as_float(ww[e] << 16), hi = __uint_as_float(ww[e] & 0xffff0000u);
+      const float4 ov = o[2 * k + (e >> 1)];
+      acc = fmaf(lo, (e & 1) ? ov.z : ov.x, acc);
+      acc = fmaf(hi, (e & 1) ? ov.w : ov.y, acc);
+    }
+  }
+  delta[r] = acc / sumg[r];
+}
+
+cudaError_t launch_delta(const uint16_t* dO, const float* Ot, const float* sumg, float* delta, long rows,
+                         cudaStream_t s) {
+  bwd_delta_kernel<<<(unsigned)((rows + 255) / 256), 256, 0, s>>>(dO, Ot, sumg, delta, rows);
+  return cudaGetLastError();
+}
+
+}  // namespace entmax

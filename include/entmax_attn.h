@@ -1,0 +1,134 @@
+/*
+ * entmax_attn.h -- C ABI of the fused alpha-entmax attention library for NVIDIA B200
+ * (sm_100a). The library is libentmax_attn.so.
+ *
+ * Operation (definitions from "AdaSplash-2: Faster Differentiable Sparse Attention"):
+ *   - §2.2: scores s_ij = scale * q_i . k_j and output O = pi(S) V.
+ *   - §2.3 Eq. 3: pi = alpha-entmax, p_ij = [(alpha-1) s_ij - tau_i]_+^{1/(alpha-1)}.
+ *   - §2.4 Eq. 4: tau_i is the root of
+ *     f(tau) = -1 + sum_j [(alpha-1) s_ij - tau]_+^{1/(alpha-1)}, inside the bracket
+ *     m - 1 <= tau <= m - n^{1-alpha}, with m = (alpha-1) max_j s_ij.
+ *   - §3.3 Phases 1-4: the forward takes a max pass, threshold refinement, a bit-packed
+ *     block mask, and an output pass over the flagged blocks only. The same section's
+ *     "Backward pass" reuses that mask.
+ *   - Appendix C.4: mask packing, 32 key tiles per uint32.
+ *   - "gpt2-adasplash-attention" model card, "Causal Splash Masking with Sink
+ *     Preservation": window mask {0} U [max(1, i-W), i].
+ * At alpha = 1.5 this equals the model cards' score-unit form
+ * A_ij = max(0, (s_ij - tau'_i)/2)^2 with tau' = tau / (alpha-1).
+ *
+ * Backward: the Jacobian of Eq. 3 is dp_j/ds_k = g_j delta_jk - g_j g_k / sum_l g_l, with
+ * g = p^{2-alpha}. The pages state only that gradients live on the support (§3.3); this
+ * formula comes from implicit differentiation of sum_j p_j = 1. Hence
+ *   dS_ij = g_ij (dO_i . V_j - delta_i),   delta_i = dO_i . Ot_i / sum_j g_ij,
+ *   Ot_i  = sum_j g_ij V_j                (written by the forward into the workspace),
+ *   dQ = scale dS K,  dK = scale dS^T Q,  dV = P^T dO.
+ *
+ * Conventions for every entry point:
+ *   - Layout: Q, K, V, dO, O, dQ, dK, dV are contiguous row-major [B, H, L, d] (one
+ *     64-element row per token); tau is [B, H, L]. All are device pointers.
+ *   - Ownership: the caller allocates and frees all memory, the workspace included.
+ *     The library never allocates, frees or keeps device memory, and holds no global
+ *     state beyond cached kernel attributes.
+ *   - Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream). All device work is enqueued on it. No call synchronises except
+ *     entmax_last_device_status.
+ *   - Errors: argument errors are found on the host before anything is launched, and
+ *     are returned as ENTMAX_EINVAL or ENTMAX_EUNSUPPORTED. A failed launch returns
+ *     ENTMAX_ECUDA. Conditions found on the device (solver cap reached, a bounded wait
+ *     that expired) are recorded in the workspace status word and read back with
+ *     entmax_last_device_status. Nothing throws across the ABI.
+ *   - Non-finite inputs give undefined results.
+ */
+#ifndef ENTMAX_ATTN_H
+#define ENTMAX_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    ENTMAX_OK = 0,
+    ENTMAX_EINVAL = 1,        /* bad pointer, size, stride or option                     */
+    ENTMAX_EUNSUPPORTED = 2,  /* valid request that this build does not implement         */
+    ENTMAX_ECUDA = 3,         /* a CUDA call or kernel launch failed                      */
+    ENTMAX_ENOCONVERGE = 4,   /* device: a row hit the refinement cap (tau kept bracketed) */
+    ENTMAX_ETIMEOUT = 5       /* device: a bounded wait inside a kernel expired            */
+} entmax_status;
+
+typedef enum { ENTMAX_BF16 = 0, ENTMAX_FP32 = 1 } entmax_dtype;
+
+typedef struct {
+    int B, H, L, d;       /* batch, heads, sequence length, head dim. d must be 64;
+                             1 <= L <= ENTMAX_MAX_L.                                     */
+    float alpha;          /* 1.5 or 2.0; any other value -> ENTMAX_EUNSUPPORTED           */
+    float scale;          /* score scale, usually 1/sqrt(d); must be > 0                 */
+    int causal;           /* 0: every key j < kv_len is active; 1: only keys j <= i      */
+    int window;           /* < 0: no window. >= 0: active = {0} U [max(1, i-window), i];
+                             this implies causal                                          */
+    const int *kv_len;    /* device int32[B]: valid keys per sequence (1 <= kv_len <= L),
+                             or NULL for all L. Every query row is computed, including
+                             rows at or past kv_len.                                      */
+    entmax_dtype dtype;   /* dtype of Q, K, V (and dO). ENTMAX_FP32 is forward-only.      */
+    int max_sweeps;       /* cap on threshold-refinement passes; 0 = library default (12) */
+} entmax_attn_desc;
+
+#define ENTMAX_MAX_L 16384   /* longest supported sequence (the per-row tile maxima live
+                                in shared memory, 4 bytes per key tile per row)           */
+#define ENTMAX_TILE 128      /* query and key tile edge; the block mask uses this size    */
+
+/* Bytes of device workspace needed by entmax_attn_fwd / entmax_attn_bwd for *desc.
+ * The workspace holds the status word, the block mask M and its transpose M^T, the
+ * per-row sum_j g_ij and Ot_i = sum_j g_ij V_j, delta_i, per-tile refinement counts
+ * and, for fp32 inputs, split copies of Q, K and V. Returns 0 for an invalid
+ * descriptor. The base address must be 256-byte aligned; the fwd -> bwd pair must use
+ * the same workspace, and the caller keeps it alive in between. */
+size_t entmax_attn_workspace_bytes(const entmax_attn_desc *desc);
+
+/* Forward (AdaSplash-2 §3.3 Phases 1-4).
+ * In:  Q, K, V [B,H,L,d] in desc->dtype.
+ * Out: O [B,H,L,d] fp32; tau [B,H,L] fp32 in Eq. 3 units; the workspace (block mask,
+ *      its transpose, sum g, Ot, refinement counts, status).
+ * The status word is cleared at the start of each forward. */
+entmax_status entmax_attn_fwd(const entmax_attn_desc *desc, const void *Q, const void *K,
+                              const void *V, float *O, float *tau, void *workspace, void *stream);
+
+/* Backward over the blocks the forward flagged (§3.3 "Backward pass").
+ * In:  Q, K, V, dO [B,H,L,d] (bf16); tau from the forward; the forward's workspace.
+ * Out: dQ, dK, dV [B,H,L,d] fp32. The call overwrites them; dQ is zeroed on the stream
+ *      and then accumulated.
+ * The forward output O is not an input: delta needs Ot = sum g V, not O (see above). */
+entmax_status entmax_attn_bwd(const entmax_attn_desc *desc, const void *Q, const void *K,
+                              const void *V, const void *dO, const float *tau,
+                              void *workspace, float *dQ, float *dK, float *dV, void *stream);
+
+/* Row-wise alpha-entmax of explicit fp32 scores (AdaSplash-2 §2.3-2.4; the §4.1 solver
+ * study works on such score vectors). Row r holds S[r*ld + j], j < n. Scores of -inf
+ * are inactive; every row needs at least one finite score.
+ * Out: P[r*ld + j] = [(alpha-1) S - tau_r]_+^{1/(alpha-1)} and tau[r] (Eq. 3 units).
+ * Constraints: rows >= 0, 1 <= n <= ld, 16-byte-aligned S and P, ld % 4 == 0,
+ * alpha in {1.5, 2}. rows == 0 is a no-op. */
+entmax_status entmax_rows(const float *S, int rows, int n, int ld, float alpha, float *P,
+                          float *tau, void *stream);
+
+/* Synchronises `stream`, then reads the workspace status word left by the last
+ * fwd/bwd: ENTMAX_OK, ENTMAX_ENOCONVERGE or ENTMAX_ETIMEOUT. *status_out receives the
+ * raw word: bit 0 = no convergence, bit 1 = wait timeout. */
+entmax_status entmax_last_device_status(const entmax_attn_desc *desc, const void *workspace,
+                                        int *status_out, void *stream);
+
+/* Copies the forward's packed block mask out of the workspace, device to device, on
+ * `stream`. M is uint32 [B, H, Tr, ceil(Tc/32)] with Tr = Tc = ceil(L/128); bit
+ * (jt % 32) of word jt/32 is set when some row of query tile it has a nonzero weight
+ * in key tile jt (Appendix C.4). sweeps receives int32 [B, H, Tr]: the refinement
+ * passes each query tile used. Either output may be NULL. */
+entmax_status entmax_attn_block_mask(const entmax_attn_desc *desc, const void *workspace,
+                                     uint32_t *M, int *sweeps, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ENTMAX_ATTN_H */

@@ -1,0 +1,96 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry point the
+header declares, and rejects bad arguments on the host before any launch."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from entmax_sm_attention_b200 import binding as eb
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "entmax_attn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from entmax_sm_attention_b200 import build
+
+    build.build()
+    return eb.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(entmax_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_names():
+    assert declared_functions() == sorted(eb.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", eb.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r"\sT\s+(\w+)", out))
+    for name in declared_functions():
+        assert name in exported, name
+        assert getattr(lib, name) is not None
+
+
+def _desc(**kw):
+    base = dict(B=1, H=2, L=300, d=64, alpha=1.5, scale=0.125, causal=0, window=-1, kv_len=None,
+                dtype=eb.ENTMAX_BF16, max_sweeps=0)
+    base.update(kw)
+    return eb.AttnDesc(base["B"], base["H"], base["L"], base["d"], base["alpha"], base["scale"], base["causal"],
+                       base["window"], base["kv_len"], base["dtype"], base["max_sweeps"])
+
+
+def test_workspace_bytes_valid_and_invalid(lib):
+    n = lib.entmax_attn_workspace_bytes(ctypes.byref(_desc()))
+    assert n > 0 and n % 256 == 0
+    # grows with L
+    assert lib.entmax_attn_workspace_bytes(ctypes.byref(_desc(L=4096))) > n
+    for bad in (dict(B=0), dict(L=0), dict(d=32), dict(alpha=1.25), dict(scale=0.0), dict(causal=2),
+                dict(max_sweeps=-1), dict(max_sweeps=65), dict(L=eb.ENTMAX_MAX_L + 1), dict(dtype=7)):
+        assert lib.entmax_attn_workspace_bytes(ctypes.byref(_desc(**bad))) == 0, bad
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(d=128), eb.ENTMAX_EUNSUPPORTED),
+    (dict(alpha=3.0), eb.ENTMAX_EUNSUPPORTED),
+    (dict(L=eb.ENTMAX_MAX_L + 128), eb.ENTMAX_EUNSUPPORTED),
+    (dict(B=-1), eb.ENTMAX_EINVAL),
+    (dict(scale=float("nan")), eb.ENTMAX_EINVAL),
+    (dict(max_sweeps=100), eb.ENTMAX_EINVAL),
+])
+def test_forward_rejects_on_host(lib, bad, code):
+    d = _desc(**bad)
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced: validation fails before any launch
+    rc = lib.entmax_attn_fwd(ctypes.byref(d), fake, fake, fake, fake, fake, fake, None)
+    assert rc == code
+
+
+def test_null_and_misaligned_pointers_rejected(lib):
+    d = _desc()
+    good = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    assert lib.entmax_attn_fwd(ctypes.byref(d), None, good, good, good, good, good, None) == eb.ENTMAX_EINVAL
+    assert lib.entmax_attn_fwd(ctypes.byref(d), odd, good, good, good, good, good, None) == eb.ENTMAX_EINVAL
+    ws_odd = ctypes.c_void_p((1 << 20) + 128)   # workspace must be 256-byte aligned
+    assert lib.entmax_attn_fwd(ctypes.byref(d), good, good, good, good, good, ws_odd, None) == eb.ENTMAX_EINVAL
+    assert lib.entmax_attn_bwd(ctypes.byref(d), good, good, good, odd, good, good, good, good, good,
+                               None) == eb.ENTMAX_EINVAL
+    assert lib.entmax_attn_fwd(None, good, good, good, good, good, good, None) == eb.ENTMAX_EINVAL
+
+
+def test_rows_rejects_on_host(lib):
+    p = ctypes.c_void_p(1 << 20)
+    assert lib.entmax_rows(p, 4, 0, 4, ctypes.c_float(1.5), p, p, None) == eb.ENTMAX_EINVAL   # n = 0
+    assert lib.entmax_rows(p, 4, 8, 6, ctypes.c_float(1.5), p, p, None) == eb.ENTMAX_EINVAL   # ld % 4
+    assert lib.entmax_rows(p, 4, 8, 4, ctypes.c_float(1.5), p, p, None) == eb.ENTMAX_EINVAL   # ld < n
+    assert lib.entmax_rows(p, 4, 8, 8, ctypes.c_float(1.2), p, p, None) == eb.ENTMAX_EUNSUPPORTED
+    assert lib.entmax_rows(p, -1, 8, 8, ctypes.c_float(1.5), p, p, None) == eb.ENTMAX_EINVAL
+    assert lib.entmax_rows(p, 0, 8, 8, ctypes.c_float(1.5), p, p, None) == eb.ENTMAX_OK      # empty: no-op

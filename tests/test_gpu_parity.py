@@ -1,0 +1,81 @@
+"""GPU (B200) vs fp64 oracle, element by element, through the C ABI.
+
+Sizes are small enough for the oracle to finish in seconds, yet span several 128-wide
+tiles with a ragged tail. The edge cases are L = 1, single-tile and tile-boundary
+lengths, key padding, window + sink, peaked rows, and the refinement cap.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from entmax_sm_attention_b200 import binding as eb
+from entmax_sm_attention_b200.workloads import make_score_rows, small_case
+
+from parity import TOL_TAU, compare
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    small_case("full_L300", L=300),
+    small_case("causal_L300", L=300, causal=True),
+    small_case("window_L300", L=300, causal=True, window=32),
+    small_case("padded_L300", B=2, L=300, kv_len=200),
+    small_case("peaked_causal_L520", L=520, causal=True, sigma_q=3.0),
+    small_case("single_row", L=1),
+    small_case("one_tile_L128", L=128, causal=True),
+    small_case("tile_plus_one_L129", L=129),
+    small_case("padded_short_kv", B=1, L=260, kv_len=5),
+    small_case("window0_L200", L=200, causal=True, window=0),
+    small_case("wide_sigma8_L384", L=384, causal=True, sigma_q=8.0),
+]
+
+
+@pytest.mark.parametrize("alpha", [1.5, 2.0])
+@pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
+def test_fwd_bwd_small(w, alpha):
+    rep = {}
+    compare(w, alpha, backward=True, report=rep)
+    print(w.name, alpha, {k: (float(v) if not isinstance(v, int) else v) for k, v in rep.items()})
+
+
+@pytest.mark.parametrize("alpha", [1.5, 2.0])
+def test_entmax_rows(alpha):
+    # The 128 x 128 score rows of the single-head workload, plus long rows with inactive entries.
+    for rows, n, sigma in ((128, 128, 1.0), (64, 1000, 2.0), (16, 4096, 0.5)):
+        S = make_score_rows(rows, n, seed=n, sigma=sigma)
+        if n == 1000:
+            S[3, 10:] = -float("inf")
+            S[4, :999] = -float("inf")
+        P, tau = eb.rows(S.cuda(), alpha)
+        P, tau = P.cpu().double().numpy(), tau.cpu().double().numpy()
+        Pr, taur = oracle.entmax_rows(S, alpha)
+        assert np.abs(tau - taur).max() <= 1e-5
+        assert np.abs(P - Pr).max() <= 1e-5
+        z = (alpha - 1) * S.double().numpy()
+        decided = np.abs(z - taur[:, None]) > 1e-3
+        assert np.array_equal((P > 0)[decided], (Pr > 0)[decided])
+
+
+def test_refinement_cap_reports_no_convergence():
+    """Refinement capped at one sweep on rows that need several: the status word says
+    so. Per §2.4 tau stays inside the bracket, so O stays finite."""
+    w = small_case("capped", L=256, causal=False, sigma_q=1.0)
+    from parity import gpu_run
+    from entmax_sm_attention_b200.workloads import make_inputs
+    g = gpu_run(make_inputs(w), w, 1.5, backward=False, max_sweeps=1)
+    assert g["status"][0] == eb.ENTMAX_ENOCONVERGE
+    assert np.isfinite(g["O"]).all() and np.isfinite(g["tau"]).all()
+
+
+def test_repeatable():
+    """Two forward+backward calls give bit-identical O, tau and dK/dV. dQ uses float
+    atomics and is only compared to tolerance."""
+    w = small_case("rep", L=384, causal=True)
+    from parity import gpu_run
+    from entmax_sm_attention_b200.workloads import make_inputs
+    inp = make_inputs(w)
+    a, b = gpu_run(inp, w, 1.5), gpu_run(inp, w, 1.5)
+    for k in ("O", "tau", "dK", "dV", "M"):
+        assert np.array_equal(a[k], b[k]), k
+    assert np.abs(a["dQ"] - b["dQ"]).max() < 1e-5
