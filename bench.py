@@ -1,0 +1,355 @@
+#!/usr/bin/env python
+"""Throughput of fused alpha-entmax attention (forward + backward) on B200.
+
+One step is one forward + backward pass over one batch of the long-context causal
+workload: B=1, H=12, L=8192, d=64, bf16, alpha=1.5, with Q ~ N(0, 3^2) (the query
+variance knob of AdaSplash-2 §4.2). Prints one JSON line.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--alpha A]
+
+With N > 1 (under torchrun) every rank runs its own batch with no data-path
+collective (weak scaling). Only the timing uses a barrier and a max-reduce.
+--impl reference times the fp64 CPU oracle on the host cores, on a bounded sample
+of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fwd+bwd tokens/s & TFLOP/s at L=8192 vs tensor-core roofline, 1×B200"
+UNIT = "tokens/s"
+TILE = 128
+UNIT_FLOP = 2 * TILE * TILE * 64      # one 128x128x64 (or 128x64x128) bf16 tile product
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="long_causal_L8192")
+    ap.add_argument("--alpha", type=float, default=1.5)
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU-oracle sample time")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ------------------------------------------------------------------ clock sampling
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines: list[str] = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------ CPU oracle
+def cpu_oracle_sample(w, alpha: float, seed: int, target_s: float):
+    """Times the fp64 oracle (as it stands) on whole heads of the workload: forward and
+    backward of head 0, 1, ... until target_s has passed. Returns tokens/s scaled to the
+    full batch (heads done / H of B*L tokens), the thread count and a description."""
+    import oracle
+    from entmax_sm_attention_b200.workloads import make_inputs
+
+    inp = make_inputs(w.with_(B=1, H=1), seed)
+    heads, t_total = 0, 0.0
+    g = __import__("torch").Generator().manual_seed(seed)
+    while heads < w.B * w.H and (heads == 0 or t_total < target_s):
+        if heads > 0:   # a fresh head of the same distribution per iteration
+            inp = make_inputs(w.with_(B=1, H=1), seed + heads)
+        pr = oracle.Problem(inp["Q"], inp["K"], inp["V"], inp["dO"], alpha=alpha, scale=w.scale,
+                            causal=w.causal, window=w.window,
+                            kv_len=None if w.kv_len is None else [w.kv_len])
+        t0 = time.perf_counter()
+        r = pr.rows(backward=True)
+        pr.cols(r["tau"], r["delta"])
+        t_total += time.perf_counter() - t0
+        heads += 1
+    del g
+    tokens = w.B * w.L * heads / (w.B * w.H)
+    return tokens / t_total, oracle.max_threads(), (
+        f"{heads} of {w.B * w.H} heads (b,h) of {w.name}, full fwd+bwd per head in fp64; "
+        f"tokens/s = heads/(B*H) * B*L / seconds")
+
+
+def run_reference(args):
+    """--impl reference: the oracle on the host cores, one head per step."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from entmax_sm_attention_b200.workloads import WORKLOADS
+
+    w = WORKLOADS[args.workload]
+    import oracle
+
+    times = []
+    for k in range(args.warmup + args.steps):
+        v, cores, _ = cpu_oracle_sample(w, args.alpha, args.seed + 100 * k, 0.0)   # one head per step
+        if k >= args.warmup:
+            times.append(v)
+    value = statistics.mean(times)
+    sample = (f"each step = full fwd+bwd of one (b,h) head of {w.name} (of {w.B * w.H}); "
+              f"tokens/s scaled by heads/(B*H)")
+    ms = w.B * w.L / value * 1e3
+    out = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+           "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "d": w.d, "alpha": args.alpha,
+                      "causal": w.causal, "sigma_q": w.sigma_q},
+           "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+           "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+# ------------------------------------------------------------------------ GPU arm
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from entmax_sm_attention_b200 import binding as eb
+    from entmax_sm_attention_b200.workloads import WORKLOADS, make_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = WORKLOADS[args.workload]
+    alpha = args.alpha
+
+    host = make_inputs(w, seed=args.seed + rank)
+    pinned = {k: v.pin_memory() for k, v in host.items()}
+    d = {k: v.to(dev) for k, v in host.items()}
+    kv = None if w.kv_len is None else torch.tensor(w.kv_len_list(), dtype=torch.int32, device=dev)
+    desc = eb.make_desc(w.B, w.H, w.L, w.d, alpha=alpha, scale=w.scale, causal=w.causal, window=w.window,
+                        kv_len=kv, dtype=eb.ENTMAX_BF16)
+    ws = eb.alloc_workspace(desc, dev)
+    shp = (w.B, w.H, w.L, w.d)
+    O = torch.empty(shp, dtype=torch.float32, device=dev)
+    tau = torch.empty(shp[:3], dtype=torch.float32, device=dev)
+    dQ, dK, dV = (torch.empty(shp, dtype=torch.float32, device=dev) for _ in range(3))
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(src):
+        eb.entmax_attn_fwd(desc, src["Q"], src["K"], src["V"], O, tau, ws, stream)
+        eb.entmax_attn_bwd(desc, src["Q"], src["K"], src["V"], src["dO"], tau, ws, dQ, dK, dV, stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step(d)
+    torch.cuda.synchronize(dev)
+    code, word = eb.entmax_last_device_status(desc, ws, stream)
+    if code != eb.ENTMAX_OK:
+        raise SystemExit(f"device status {eb.STATUS_NAMES[code]} (word {word}) after warm-up")
+
+    # ---- device-timed region: inputs resident in HBM, L2 flushed before every step
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize(dev)
+    for k in range(args.steps):
+        flush.zero_()
+        ev[k][0].record(stream)
+        eb.entmax_attn_fwd(desc, d["Q"], d["K"], d["V"], O, tau, ws, stream)
+        ev[k][1].record(stream)
+        eb.entmax_attn_bwd(desc, d["Q"], d["K"], d["V"], d["dO"], tau, ws, dQ, dK, dV, stream)
+        ev[k][2].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clk = clocks.stop()
+    fwd_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    bwd_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    total_ms = sum(fwd_ms) + sum(bwd_ms)
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    tokens_per_step = w.B * w.L
+    value = world * tokens_per_step * args.steps / (total_ms / 1e3)
+
+    # ---- end to end through the public API: pinned host -> device, fwd+bwd, device -> host
+    out_host = {k: torch.empty(shp, dtype=torch.float32).pin_memory() for k in ("O", "dQ", "dK", "dV")}
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+    d2h = sum(v.numel() * v.element_size() for v in out_host.values())
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(args.steps):
+        for k in ("Q", "K", "V", "dO"):
+            d[k].copy_(pinned[k], non_blocking=True)
+        step(d)
+        for k, src in (("O", O), ("dQ", dQ), ("dK", dK), ("dV", dV)):
+            out_host[k].copy_(src, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    e2e_value = world * tokens_per_step * args.steps / (float(e2e_ms.item()) / 1e3)
+
+    # ---- work actually done (per-tile counters written by the forward)
+    M, st = eb.block_mask((desc, ws))
+    st = st.cpu().long()
+    n_sweeps, n_s, n_out, n_act = (st[..., c] for c in range(4))
+    s_tiles, out_tiles, act_tiles = int(n_s.sum()), int(n_out.sum()), int(n_act.sum())
+    # Algorithmic tensor work (SURVEY-style count, tile granularity): forward = every
+    # S tile computed (max pass + refinement passes + output pass) + O and Ot products
+    # on flagged tiles; backward = S, dA, dV, dK, dQ on every flagged tile pair.
+    fwd_flops = UNIT_FLOP * (s_tiles + 2 * out_tiles)
+    bwd_flops = UNIT_FLOP * 5 * out_tiles
+    # Issued tensor work, counting the two-term (hi + lo) splits.
+    fwd_issued = UNIT_FLOP * (s_tiles + (4 if alpha == 1.5 else 3) * out_tiles)
+    bwd_issued = UNIT_FLOP * 8 * out_tiles
+    fwd_avg, bwd_avg = statistics.mean(fwd_ms), statistics.mean(bwd_ms)
+    peaks = load_peaks()
+    peak = peaks["bf16_tflops_sustained"]
+    dom = "bwd" if bwd_avg >= fwd_avg else "fwd"
+    dom_ms = bwd_avg if dom == "bwd" else fwd_avg
+    dom_flops = bwd_flops if dom == "bwd" else fwd_flops
+    achieved = dom_flops / (dom_ms * 1e-3) / 1e12
+    total_tflops = (fwd_flops + bwd_flops) / (ms_per_step * 1e-3) / 1e12
+    # Softmax-equivalent work over structurally active pairs (4d fwd, 10d bwd per pair).
+    pairs = act_pairs(w)
+    sm_eq = (4 + 10) * w.d * pairs / (ms_per_step * 1e-3) / 1e12
+
+    result = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "d": w.d, "alpha": alpha,
+                   "causal": w.causal, "window": w.window, "kv_len": w.kv_len, "sigma_q": w.sigma_q,
+                   "seed": args.seed, "l2": "flushed (256 MB write) before every timed step",
+                   "parallelism": f"replica x{world} (independent batches)"},
+        "roofline": {"bound": "tensor", "kernel": f"entmax {dom} (algorithmic bf16 tile products)",
+                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "peak_source": f"{peaks['source']} bf16 sustained (cuBLAS loop under the power cap)",
+                     "traffic": None},
+        "clocks": clk,
+        "gpu_launches": 3 * args.steps,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "detail": {
+            "fwd_ms": fwd_avg, "bwd_ms": bwd_avg,
+            "tflops_total_algorithmic": total_tflops,
+            "tflops_fwd_algorithmic": fwd_flops / (fwd_avg * 1e-3) / 1e12,
+            "tflops_bwd_algorithmic": bwd_flops / (bwd_avg * 1e-3) / 1e12,
+            "tflops_fwd_issued": fwd_issued / (fwd_avg * 1e-3) / 1e12,
+            "tflops_bwd_issued": bwd_issued / (bwd_avg * 1e-3) / 1e12,
+            "softmax_equiv_tflops": sm_eq,
+            "block_sparsity_128": 1.0 - out_tiles / max(1, act_tiles),
+            "refine_sweeps_mean": float(n_sweeps.float().mean()), "refine_sweeps_max": int(n_sweeps.max()),
+            "s_tiles": s_tiles, "flagged_tiles": out_tiles, "active_tiles": act_tiles,
+            "memsets_per_step": 3,
+        },
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, cores, sample = cpu_oracle_sample(w, alpha, args.seed, args.cpu_seconds)
+        result["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def act_pairs(w) -> int:
+    """Structurally active (query, key) pairs of the workload."""
+    L = w.L
+    kv = L if w.kv_len is None else w.kv_len
+    if w.window >= 0:
+        per = sum(1 + max(0, min(i, kv - 1) - max(1, i - w.window) + 1) for i in range(L))
+    elif w.causal:
+        per = sum(min(i + 1, kv) for i in range(L))
+    else:
+        per = L * kv
+    return w.B * w.H * per
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

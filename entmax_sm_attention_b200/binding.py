@@ -144,9 +144,9 @@ def entmax_last_device_status(desc: AttnDesc, workspace, stream=None) -> tuple[i
     return code, word.value
 
 
-def entmax_attn_block_mask(desc: AttnDesc, workspace, M=None, sweeps=None, stream=None) -> int:
+def entmax_attn_block_mask(desc: AttnDesc, workspace, M=None, stats=None, stream=None) -> int:
     return _check("entmax_attn_block_mask", load_library().entmax_attn_block_mask(
-        ctypes.byref(desc), _ptr(workspace), _ptr(M), _ptr(sweeps), _stream(stream)))
+        ctypes.byref(desc), _ptr(workspace), _ptr(M), _ptr(stats), _stream(stream)))
 
 
 # ---------------------------------------------------------------- tensor conveniences
@@ -185,12 +185,13 @@ def backward(ctx, Q, K, V, dO, tau):
 
 
 def block_mask(ctx):
-    """(M uint32 [B, H, Tr, ceil(Tc/32)], refinement sweeps int32 [B, H, Tr]) of a forward."""
+    """(M as int32 bit patterns [B, H, Tr, ceil(Tc/32)], stats int32 [B, H, Tr, 4]) of a
+    forward; stats = (refinement passes, S tiles computed, flagged tiles, active tiles)."""
     desc, ws = ctx
     Mv = torch.empty(mask_shape(desc), dtype=torch.int32, device=ws.device)
-    sw = torch.empty(mask_shape(desc)[:3], dtype=torch.int32, device=ws.device)
-    entmax_attn_block_mask(desc, ws, Mv, sw)
-    return Mv, sw
+    st = torch.empty(mask_shape(desc)[:3] + (4,), dtype=torch.int32, device=ws.device)
+    entmax_attn_block_mask(desc, ws, Mv, st)
+    return Mv, st
 
 
 def rows(S: torch.Tensor, alpha: float = 1.5):

@@ -22,8 +22,8 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct Layout {
   int BH, Tr, Tc, Wc, Wr;
-  size_t off_status, off_M, off_MT, off_sumg, off_Ot, off_delta, off_sweeps, total;
-  size_t bytes_M, bytes_MT, bytes_sweeps;
+  size_t off_status, off_M, off_MT, off_sumg, off_Ot, off_delta, off_stats, total;
+  size_t bytes_M, bytes_MT, bytes_stats;
 };
 
 bool layout_of(const entmax_attn_desc* d, Layout* l) {
@@ -48,9 +48,9 @@ bool layout_of(const entmax_attn_desc* d, Layout* l) {
   off += align256(rows * kD * 4);
   l->off_delta = off;
   off += align256(rows * 4);
-  l->off_sweeps = off;
-  l->bytes_sweeps = (size_t)l->BH * l->Tr * 4;
-  off += align256(l->bytes_sweeps);
+  l->off_stats = off;
+  l->bytes_stats = (size_t)l->BH * l->Tr * 16;
+  off += align256(l->bytes_stats);
   l->total = off;
   return true;
 }
@@ -127,7 +127,7 @@ extern "C" entmax_status entmax_attn_fwd(const entmax_attn_desc* d, const void* 
   p.Ot = reinterpret_cast<float*>(w + l.off_Ot);
   p.M = reinterpret_cast<uint32_t*>(w + l.off_M);
   p.MT = reinterpret_cast<uint32_t*>(w + l.off_MT);
-  p.sweeps = reinterpret_cast<int*>(w + l.off_sweeps);
+  p.stats = reinterpret_cast<int*>(w + l.off_stats);
   p.status = reinterpret_cast<int*>(w + l.off_status);
   p.kv_len = d->kv_len;
   p.H = d->H;
@@ -214,7 +214,7 @@ extern "C" entmax_status entmax_last_device_status(const entmax_attn_desc* d, co
 }
 
 extern "C" entmax_status entmax_attn_block_mask(const entmax_attn_desc* d, const void* ws, uint32_t* M,
-                                                int* sweeps, void* stream) {
+                                                int* stats, void* stream) {
   if (check_desc(d) != ENTMAX_OK || !aligned(ws, 256)) return ENTMAX_EINVAL;
   Layout l;
   layout_of(d, &l);
@@ -222,7 +222,7 @@ extern "C" entmax_status entmax_attn_block_mask(const entmax_attn_desc* d, const
   const uint8_t* w = static_cast<const uint8_t*>(ws);
   if (M && cudaMemcpyAsync(M, w + l.off_M, l.bytes_M, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
     return ENTMAX_ECUDA;
-  if (sweeps && cudaMemcpyAsync(sweeps, w + l.off_sweeps, l.bytes_sweeps, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+  if (stats && cudaMemcpyAsync(stats, w + l.off_stats, l.bytes_stats, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
     return ENTMAX_ECUDA;
   return ENTMAX_OK;
 }

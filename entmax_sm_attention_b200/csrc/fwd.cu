@@ -418,7 +418,12 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           p.tau[(size_t)bh * p.L + i] = tau;
           p.sumg[(size_t)bh * p.L + i] = sg;
         }
-        if (tid == 0) p.sweeps[(size_t)bh * p.Tr + qt] = sweeps;
+        if (tid == 0) {
+          int n_act = 0;
+          for (int w = 0; w < kMaskWords; ++w) n_act += __popc(act[w]);
+          int4* st = reinterpret_cast<int4*>(p.stats) + (size_t)bh * p.Tr + qt;
+          *st = make_int4(sweeps, (int)n_s, n_out, n_act);
+        }
         break;
       }
 

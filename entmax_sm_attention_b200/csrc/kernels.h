@@ -14,7 +14,7 @@ struct FwdParams {
   float* Ot;                // [B*H][L][64]  sum_j g_ij V_j
   uint32_t* M;              // [B*H][Tr][Wc]
   uint32_t* MT;             // [B*H][Tc][Wr] (zeroed before the launch)
-  int* sweeps;              // [B*H][Tr]
+  int* stats;               // [B*H][Tr][4]: sweeps, S tiles computed, flagged tiles, active tiles
   int* status;
   const int* kv_len;        // [B] or nullptr
   int H, L, Tr, Tc, Wc, Wr, BH;

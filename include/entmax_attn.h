@@ -82,7 +82,7 @@ typedef struct {
 
 /* Bytes of device workspace needed by entmax_attn_fwd / entmax_attn_bwd for *desc.
  * The workspace holds the status word, the block mask M and its transpose M^T, the
- * per-row sum_j g_ij and Ot_i = sum_j g_ij V_j, delta_i, per-tile refinement counts
+ * per-row sum_j g_ij and Ot_i = sum_j g_ij V_j, delta_i, per-tile counters
  * and, for fp32 inputs, split copies of Q, K and V. Returns 0 for an invalid
  * descriptor. The base address must be 256-byte aligned; the fwd -> bwd pair must use
  * the same workspace, and the caller keeps it alive in between. */
@@ -120,13 +120,17 @@ entmax_status entmax_rows(const float *S, int rows, int n, int ld, float alpha, 
 entmax_status entmax_last_device_status(const entmax_attn_desc *desc, const void *workspace,
                                         int *status_out, void *stream);
 
-/* Copies the forward's packed block mask out of the workspace, device to device, on
- * `stream`. M is uint32 [B, H, Tr, ceil(Tc/32)] with Tr = Tc = ceil(L/128); bit
- * (jt % 32) of word jt/32 is set when some row of query tile it has a nonzero weight
- * in key tile jt (Appendix C.4). sweeps receives int32 [B, H, Tr]: the refinement
- * passes each query tile used. Either output may be NULL. */
+/* Copies the forward's packed block mask and per-tile counters out of the workspace,
+ * device to device, on `stream`.
+ *   - M is uint32 [B, H, Tr, ceil(Tc/32)], with Tr = Tc = ceil(L/128). Bit (jt % 32)
+ *     of word jt/32 is set when some row of query tile it has a nonzero weight in key
+ *     tile jt (Appendix C.4).
+ *   - stats is int32 [B, H, Tr, 4]. Per query tile it holds: the refinement passes
+ *     used, the S = Q K^T tiles computed (all passes), the flagged key tiles (the
+ *     output pass), and the structurally active key tiles.
+ * Either output may be NULL. */
 entmax_status entmax_attn_block_mask(const entmax_attn_desc *desc, const void *workspace,
-                                     uint32_t *M, int *sweeps, void *stream);
+                                     uint32_t *M, int *stats, void *stream);
 
 #ifdef __cplusplus
 }

@@ -34,12 +34,12 @@ def gpu_run(inp: dict, w: Workload, alpha: float, backward: bool = True, max_swe
     out = {"O": O, "tau": tau}
     if backward:
         out["dQ"], out["dK"], out["dV"] = eb.backward(ctx, dev["Q"], dev["K"], dev["V"], dev["dO"], tau)
-    M, sweeps = eb.block_mask(ctx)
+    M, stats = eb.block_mask(ctx)
     code, word = eb.entmax_last_device_status(ctx[0], ctx[1])
     torch.cuda.synchronize()
     res = {k: v.cpu().double().numpy() for k, v in out.items()}
     res["M"] = M.cpu().numpy().view(np.uint32)
-    res["sweeps"] = sweeps.cpu().numpy()
+    res["stats"] = stats.cpu().numpy()
     res["status"] = (code, word)
     return res
 
