@@ -22,7 +22,8 @@ ENTMAX_BF16, ENTMAX_FP32 = 0, 1
 ENTMAX_MAX_L = 16384
 ENTMAX_TILE = 128
 EXPORTS = ("entmax_attn_workspace_bytes", "entmax_attn_fwd", "entmax_attn_bwd", "entmax_rows",
-           "entmax_last_device_status", "entmax_attn_block_mask")
+           "entmax_last_device_status", "entmax_attn_block_mask", "entmax_attn_fwd_noalloc")
+ENTMAX_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 class EntmaxError(RuntimeError):
@@ -66,6 +67,8 @@ def load_library(path: str = LIB_PATH):
     lib.entmax_last_device_status.restype = i
     lib.entmax_attn_block_mask.argtypes = [dp, vp, vp, vp, vp]
     lib.entmax_attn_block_mask.restype = i
+    lib.entmax_attn_fwd_noalloc.argtypes = [dp, vp, vp, vp, vp, vp, vp]
+    lib.entmax_attn_fwd_noalloc.restype = i
     _lib = lib
     return lib
 
@@ -147,6 +150,14 @@ def entmax_last_device_status(desc: AttnDesc, workspace, stream=None) -> tuple[i
 def entmax_attn_block_mask(desc: AttnDesc, workspace, M=None, stats=None, stream=None) -> int:
     return _check("entmax_attn_block_mask", load_library().entmax_attn_block_mask(
         ctypes.byref(desc), _ptr(workspace), _ptr(M), _ptr(stats), _stream(stream)))
+
+
+def entmax_attn_fwd_noalloc(desc: AttnDesc, Q, K, V, O, tau, stream=None) -> int:
+    """Forward for callers that cannot allocate: the library's fixed per-GPU scratch
+    replaces the workspace (see include/entmax_attn.h for the size limit and the rule
+    that overlapping calls race)."""
+    return _check("entmax_attn_fwd_noalloc", load_library().entmax_attn_fwd_noalloc(
+        ctypes.byref(desc), _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(tau), _stream(stream)))
 
 
 # ---------------------------------------------------------------- tensor conveniences

@@ -132,6 +132,30 @@ entmax_status entmax_last_device_status(const entmax_attn_desc *desc, const void
 entmax_status entmax_attn_block_mask(const entmax_attn_desc *desc, const void *workspace,
                                      uint32_t *M, int *stats, void *stream);
 
+/* Forward for callers that cannot allocate device memory. Some callers are handed
+ * only their input and output buffers: a plugin inside a host framework that owns
+ * every device allocation and gives the plugin no allocator, or a latency-critical
+ * loop that must not call cudaMalloc after start-up (cudaMalloc can synchronise the
+ * device). This call runs the same forward as entmax_attn_fwd, with the same arguments
+ * minus the workspace. Its scratch is a fixed array of ENTMAX_NOALLOC_SCRATCH_BYTES
+ * that the library keeps on every GPU that loads it, until the process exits.
+ * The paper has no counterpart to this entry point; it exists for deployment only.
+ *   - Limit: entmax_attn_workspace_bytes(desc) must not exceed
+ *     ENTMAX_NOALLOC_SCRATCH_BYTES (16 MiB, roughly B*H*L <= 63000 rows). A larger
+ *     problem returns ENTMAX_EUNSUPPORTED before anything is launched.
+ *   - Allocates nothing: no cudaMalloc, no cudaFree, no allocating library routine.
+ *   - The first call on a device looks up the device address of the scratch array
+ *     while that device is current. Make that first call before any stream capture.
+ *   - All calls on a device share the one scratch array, and it keeps the last
+ *     call's contents. Each call clears the parts that must start at zero. Calls whose
+ *     GPU work overlaps (different streams, or host threads without ordering) race on
+ *     the array and give undefined results, so serialise them.
+ *   - Forward only: no workspace remains to pass to entmax_attn_bwd, and
+ *     entmax_last_device_status / entmax_attn_block_mask cannot see this scratch. */
+#define ENTMAX_NOALLOC_SCRATCH_BYTES (16u << 20)
+entmax_status entmax_attn_fwd_noalloc(const entmax_attn_desc *desc, const void *Q, const void *K,
+                                      const void *V, float *O, float *tau, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
