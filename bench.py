@@ -37,7 +37,7 @@ L2_BYTES = 126 * 1024 * 1024
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="long_causal_L8192")
@@ -46,6 +46,24 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU-oracle sample time")
     return ap.parse_args()
+
+
+def ncu_traffic(kernel: str, workload: str, alpha: float):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, or None when the
+    kernel source has changed since that capture (or no capture exists)."""
+    import hashlib
+
+    path = os.path.join(ROOT, "profiles", "traffic_per_launch.txt")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f).get(kernel)
+    if not rec or rec.get("workload") != workload or rec.get("alpha") != alpha:
+        return None
+    with open(os.path.join(ROOT, rec["source"]), "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest()[:16] != rec["sha256_16"]:
+            return None
+    return rec["bytes_per_launch"]
 
 
 def load_peaks():
@@ -303,7 +321,8 @@ def run_ours(args):
         "roofline": {"bound": "tensor", "kernel": f"entmax {dom} (algorithmic bf16 tile products)",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "peak_source": f"{peaks['source']} bf16 sustained (cuBLAS loop under the power cap)",
-                     "traffic": None},
+                     "traffic": ncu_traffic(dom, w.name, alpha),
+                     "traffic_unit": "bytes per launch (ncu dram read+write; null if the kernel changed)"},
         "clocks": clk,
         "gpu_launches": 3 * args.steps,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
