@@ -12,13 +12,16 @@
 // One CTA per (batch*head, 128-key tile). K_j and V_j stay in shared memory; the
 // flagged query tiles stream through a 2-stage ring of (Q_i, dO_i). Per query tile the
 // tensor cores compute S = Q_i K_j^T and dA = dO_i V_j^T into TMEM (M = queries).
-// Warps 0-3 (one query row per thread) form A and dS as two-term bf16 splits
-// (hi + lo, about fp32 accuracy in the products) into swizzled shared-memory buffers.
-// Those buffers then feed dV += A^T dO_i and dK += dS^T Q_i as MN-major operands
-// (M = keys, accumulated in TMEM), and dQ_i = dS K_j as a K-major operand
-// (double-buffered in TMEM). The row owners add dQ_i to global memory with
-// vector reductions. TMEM: [0,128) S, [128,256) dA, [256,320) dV, [320,384) dK,
-// [384,512) dQ x2.
+// Warps 0-7 are row owners: warp w reads TMEM lanes 32(w%4)..+31 (one query row per
+// lane) and the columns of keys [64(w/4), 64(w/4)+64). Once a warp holds its S and dA
+// values in registers it releases them, so the MMA warp computes S and dA of the next
+// query tile while the row owners form A and dS. A and dS are written as two-term bf16
+// splits (hi + lo, about fp32 accuracy in the products) into swizzled shared-memory
+// buffers. Those buffers then feed dV += A^T dO_i and dK += dS^T Q_i as MN-major
+// operands (M = keys, accumulated in TMEM), and dQ_i = dS K_j as a K-major operand
+// (double-buffered in TMEM). The row owners add dQ_i to global memory with vector
+// reductions. Warp 8 issues the TMA loads, warp 9 the MMAs.
+// TMEM: [0,128) S, [128,256) dA, [256,320) dV, [320,384) dK, [384,512) dQ x2.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -26,13 +29,15 @@ namespace entmax {
 
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
 constexpr int kStages = 2;
 constexpr int kPairBytes = 2 * kTileBytes;   // Q_i and dO_i
 
 struct Shared {
   uint64_t full[kStages], empty[kStages];
-  uint64_t bar_kv, s_full, p_ready, mma2_done;
+  uint64_t bar_kv, s_full, sda_free, p_ready, mma2_done;
   uint32_t tmem_base;
   int abort_flag;
   uint32_t qlist[kMaskWords];
@@ -81,13 +86,14 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     }
     mbar_init(&sh.bar_kv, 1);
     mbar_init(&sh.s_full, 1);
-    mbar_init(&sh.p_ready, 4);
+    mbar_init(&sh.sda_free, 8);
+    mbar_init(&sh.p_ready, 8);
     mbar_init(&sh.mma2_done, 1);
     sh.abort_flag = 0;
     fence_mbar_init();
   }
   if (tid < kMaskWords) sh.qlist[tid] = (tid < p.Wr) ? p.MT[((size_t)bh * p.Tc + kt) * p.Wr + tid] : 0u;
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(&sh.tmem_base, 512);
     tmem_relinquish();
   }
@@ -101,7 +107,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
 #pragma unroll
   for (int w = 0; w < kMaskWords; ++w) nq += __popc(qlist[w]);
 
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0 && nq > 0) {
       tma_prefetch_desc(&p.tQ);
@@ -123,7 +129,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
         mbar_wait(&sh.full[k % kStages], (k / kStages) & 1, status, &no_abort);
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------- MMA issuer
     if (lane == 0 && nq > 0) {
       const uint32_t id128 = idesc_bf16(128, 128, 0, 0);
@@ -132,12 +138,12 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       const uint32_t kA = smem_u32(sK), vA = smem_u32(sV);
       const uint32_t aH = smem_u32(sA), aL = smem_u32(sAl), dH = smem_u32(sdS), dL = smem_u32(sdSl);
       mbar_wait(&sh.bar_kv, 0, status, abrt);
-      uint32_t seq = 0;
-      for_each_bit(qlist, kMaskWords, [&](int) {
-        const int st = seq % kStages;
+      // S = Q_s K^T and dA = dO_s V^T into TMEM [0,256).
+      auto issue_sda = [&](int s) {
+        const int st = s % kStages;
         const uint32_t qA = smem_u32(ring + st * kPairBytes), oA = qA + kTileBytes;
-        // S and dA of the previous step were consumed before its p_ready, waited below.
-        mbar_wait(&sh.full[st], (seq / kStages) & 1, status, abrt);
+        mbar_wait(&sh.full[st], (s / kStages) & 1, status, abrt);
+        if (s > 0) mbar_wait(&sh.sda_free, (s - 1) & 1, status, abrt);   // S, dA of s-1 are in registers
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -145,19 +151,25 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
           mma_ss(T + 128, sdesc_sw128(oA + k * 32, 16, 1024), sdesc_sw128(vA + k * 32, 16, 1024), id128, k > 0);
         }
         mma_commit(&sh.s_full);
-        mbar_wait(&sh.p_ready, seq & 1, status, abrt);   // A and dS in shared memory
+      };
+      issue_sda(0);
+      for (int s = 0; s < nq; ++s) {
+        if (s + 1 < nq) issue_sda(s + 1);   // overlaps the row owners' work on tile s
+        const int st = s % kStages;
+        const uint32_t qA = smem_u32(ring + st * kPairBytes), oA = qA + kTileBytes;
+        mbar_wait(&sh.p_ready, s & 1, status, abrt);   // A and dS of tile s in shared memory
         tc_fence_after();
-        const uint32_t dq = T + 384 + (seq & 1) * 64;
+        const uint32_t dq = T + 384 + (s & 1) * 64;
 #pragma unroll
         for (int t = 0; t < 8; ++t) {
-          // dV += A^T dO_i and dK += dS^T Q_i: K = queries (16 per step), M = keys.
-          const uint32_t acc = (seq > 0 || t > 0) ? 1u : 0u;
+          // dV += A^T dO_s and dK += dS^T Q_s: K = queries (16 per step), M = keys.
+          const uint32_t acc = (s > 0 || t > 0) ? 1u : 0u;
           const uint64_t bO = sdesc_sw128(oA + t * 2048, 8192, 1024), bQ = sdesc_sw128(qA + t * 2048, 8192, 1024);
           mma_ss(T + 256, sdesc_sw128(aH + t * 2048, 16384, 1024), bO, idMN, acc);
           mma_ss(T + 256, sdesc_sw128(aL + t * 2048, 16384, 1024), bO, idMN, 1u);
           mma_ss(T + 320, sdesc_sw128(dH + t * 2048, 16384, 1024), bQ, idMN, acc);
           mma_ss(T + 320, sdesc_sw128(dL + t * 2048, 16384, 1024), bQ, idMN, 1u);
-          // dQ_i = dS K_j: K = keys (16 per step; panel t/4), M = queries.
+          // dQ_s = dS K_j: K = keys (16 per step; panel t/4), M = queries.
           const uint32_t koff = (t >> 2) * kTileBytes + (t & 3) * 32;
           const uint64_t bK = sdesc_sw128(kA + t * 2048, 8192, 1024);
           mma_ss(dq, sdesc_sw128(dH + koff, 16, 1024), bK, idQ, t > 0 ? 1u : 0u);
@@ -165,39 +177,31 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
         }
         mma_commit(&sh.empty[st]);
         mma_commit(&sh.mma2_done);
-        ++seq;
-      });
+      }
     }
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- row owners
-    const int row = tid;
-    const uint32_t tl = T + ((uint32_t)(warp * 32) << 16);
+    const int quad = warp & 3, hf = warp >> 2;   // TMEM lane quadrant, key half
+    const int row = quad * 32 + lane;
+    const uint32_t tl = T + ((uint32_t)(quad * 32) << 16);
     const float cz = p.cz;
     uint32_t seq = 0;
     int prev_i = -1;
-    // Adds dQ of the query tile handled at step `s` (TMEM buffer s & 1) to global memory.
-    // Each mma2_done phase is waited on exactly once: inside the loop the wait before
-    // the shared-memory writes of step s+1 already covers step s.
-    auto flush_dq = [&](uint32_t s, int irow, bool wait) {
-      if (wait) warp_wait(&sh.mma2_done, s & 1, status, abrt);
+    // Adds this thread's 32 columns of dQ for the query tile of step `s` (TMEM buffer
+    // s % 2) to global memory. The caller has already waited for that step's MMAs.
+    auto flush_dq = [&](uint32_t s, int irow) {
       tc_fence_after();
-      const uint32_t dq = tl + 384 + (s & 1) * 64;
-      uint32_t a[32], c[32];
-      tmem_ld32(dq, a);
-      tmem_ld32(dq + 32, c);
+      uint32_t a[32];
+      tmem_ld32(tl + 384 + (s & 1) * 64 + hf * 32, a);
       tmem_wait_ld();
       if (irow < p.L) {
-        float* dst = p.dQ + ((size_t)bh * p.L + irow) * kD;
+        float* dst = p.dQ + ((size_t)bh * p.L + irow) * kD + hf * 32;
         const float sc = p.scale;
 #pragma unroll
         for (int k = 0; k < 8; ++k)
           red_add_v4(dst + 4 * k, sc * __uint_as_float(a[4 * k]), sc * __uint_as_float(a[4 * k + 1]),
                      sc * __uint_as_float(a[4 * k + 2]), sc * __uint_as_float(a[4 * k + 3]));
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-          red_add_v4(dst + 32 + 4 * k, sc * __uint_as_float(c[4 * k]), sc * __uint_as_float(c[4 * k + 1]),
-                     sc * __uint_as_float(c[4 * k + 2]), sc * __uint_as_float(c[4 * k + 3]));
       }
       __syncwarp();
     };
@@ -208,90 +212,94 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       const float dl = valid ? p.delta[(size_t)bh * p.L + i] : 0.f;
       const bool full = pat.block_full(it * kTile, min(p.L, it * kTile + kTile), j0, j0 + kTile);
       warp_wait(&sh.s_full, seq & 1, status, abrt);
+      tc_fence_after();
+      uint32_t sr[64], ar[64];
+      tmem_ld32(tl + hf * 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(tl + hf * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_ld32(tl + 128 + hf * 64, *reinterpret_cast<uint32_t(*)[32]>(&ar[0]));
+      tmem_ld32(tl + 128 + hf * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&ar[32]));
+      tmem_wait_ld();
+      tc_fence_before();
+      warp_arrive(&sh.sda_free);
       // The previous tile's dV/dK/dQ MMAs must be done reading sA / sdS.
       if (seq > 0) warp_wait(&sh.mma2_done, (seq - 1) & 1, status, abrt);
-      tc_fence_after();
-#pragma unroll 1
-      for (int q = 0; q < 4; ++q) {
-        uint32_t sr[32], ar[32];
-        tmem_ld32(tl + q * 32, sr);
-        tmem_ld32(tl + 128 + q * 32, ar);
-        tmem_wait_ld();
-        uint32_t ah[16], al[16], dh[16], dl2[16];
+      // Keys [64 hf, 64 hf + 64) of row `row`: panel hf, 16-byte chunks 0..7.
+      const int pan = hf * kTileBytes;
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          float s0 = __uint_as_float(sr[2 * c]), s1 = __uint_as_float(sr[2 * c + 1]);
+      for (int ch = 0; ch < 8; ++ch) {
+        uint32_t ah[4], al[4], dh[4], dl2[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int c = ch * 8 + 2 * e;
+          float s0 = __uint_as_float(sr[c]), s1 = __uint_as_float(sr[c + 1]);
           if (!full) {
-            const int jj = j0 + q * 32 + 2 * c;
+            const int jj = j0 + hf * 64 + c;
             if (!pat.active(i, jj)) s0 = -INFINITY;
             if (!pat.active(i, jj + 1)) s1 = -INFINITY;
           }
-          const float u0 = fmaf(s0, cz, -tau), u1 = fmaf(s1, cz, -tau);
-          const float v0 = fmaxf(u0, 0.f), v1 = fmaxf(u1, 0.f);
-          const float d0 = __uint_as_float(ar[2 * c]) - dl, d1 = __uint_as_float(ar[2 * c + 1]) - dl;
+          const float2 u = __ffma2_rn(make_float2(s0, s1), make_float2(cz, cz), make_float2(-tau, -tau));
+          const float v0 = fmaxf(u.x, 0.f), v1 = fmaxf(u.y, 0.f);
+          const float d0 = __uint_as_float(ar[c]) - dl, d1 = __uint_as_float(ar[c + 1]) - dl;
           if (AK == kAlpha15) {
-            split_bf16x2(v0 * v0, v1 * v1, ah[c], al[c]);
-            split_bf16x2(v0 * d0, v1 * d1, dh[c], dl2[c]);
+            const float2 a = __fmul2_rn(make_float2(v0, v1), make_float2(v0, v1));
+            const float2 ds = __fmul2_rn(make_float2(v0, v1), make_float2(d0, d1));
+            split_bf16x2(a.x, a.y, ah[e], al[e]);
+            split_bf16x2(ds.x, ds.y, dh[e], dl2[e]);
           } else {
-            split_bf16x2(v0, v1, ah[c], al[c]);
-            split_bf16x2(u0 > 0.f ? d0 : 0.f, u1 > 0.f ? d1 : 0.f, dh[c], dl2[c]);
+            split_bf16x2(v0, v1, ah[e], al[e]);
+            split_bf16x2(u.x > 0.f ? d0 : 0.f, u.y > 0.f ? d1 : 0.f, dh[e], dl2[e]);
           }
         }
-        // Keys q*32 .. q*32+31 -> panel q/2, 16-byte chunks (q%2)*4 .. +3 of row `row`.
-        const int pan = (q >> 1) * kTileBytes;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint32_t off = pan + sw128_offset(row, (q & 1) * 32 + k * 8);
-          *reinterpret_cast<uint4*>(sA + off) = make_uint4(ah[4 * k], ah[4 * k + 1], ah[4 * k + 2], ah[4 * k + 3]);
-          *reinterpret_cast<uint4*>(sAl + off) = make_uint4(al[4 * k], al[4 * k + 1], al[4 * k + 2], al[4 * k + 3]);
-          *reinterpret_cast<uint4*>(sdS + off) = make_uint4(dh[4 * k], dh[4 * k + 1], dh[4 * k + 2], dh[4 * k + 3]);
-          *reinterpret_cast<uint4*>(sdSl + off) =
-              make_uint4(dl2[4 * k], dl2[4 * k + 1], dl2[4 * k + 2], dl2[4 * k + 3]);
-        }
+        const uint32_t off = pan + sw128_offset(row, ch * 8);
+        *reinterpret_cast<uint4*>(sA + off) = make_uint4(ah[0], ah[1], ah[2], ah[3]);
+        *reinterpret_cast<uint4*>(sAl + off) = make_uint4(al[0], al[1], al[2], al[3]);
+        *reinterpret_cast<uint4*>(sdS + off) = make_uint4(dh[0], dh[1], dh[2], dh[3]);
+        *reinterpret_cast<uint4*>(sdSl + off) = make_uint4(dl2[0], dl2[1], dl2[2], dl2[3]);
       }
       fence_proxy_async_smem();
-      tc_fence_before();
       warp_arrive(&sh.p_ready);
-      if (seq > 0) flush_dq(seq - 1, prev_i, false);
+      if (seq > 0) flush_dq(seq - 1, prev_i);   // its MMAs were waited for above
       prev_i = i;
       ++seq;
     });
-    if (seq > 0) flush_dq(seq - 1, prev_i, true);
-    // dK and dV of this key tile (TMEM lane = key). Every lane executes the TMEM loads
-    // (.sync.aligned); only the global stores depend on the key being inside L.
+    if (seq > 0) {
+      warp_wait(&sh.mma2_done, (seq - 1) & 1, status, abrt);
+      flush_dq(seq - 1, prev_i);
+    }
+    // dK and dV of this key tile (TMEM lane = key); each thread writes 32 of the 64
+    // columns. Every lane executes the TMEM loads (.sync.aligned); only the global stores
+    // depend on the key being inside L.
     const int j = j0 + row;
     const bool jvalid = j < p.L;
-    float* dk = p.dK + ((size_t)bh * p.L + (jvalid ? j : 0)) * kD;
-    float* dv = p.dV + ((size_t)bh * p.L + (jvalid ? j : 0)) * kD;
+    float* dk = p.dK + ((size_t)bh * p.L + (jvalid ? j : 0)) * kD + hf * 32;
+    float* dv = p.dV + ((size_t)bh * p.L + (jvalid ? j : 0)) * kD + hf * 32;
     const float sc = p.scale;
-    for (int h = 0; h < 2; ++h) {
-      uint32_t a[32], c[32];
-      if (seq > 0) {
-        tmem_ld32(tl + 256 + h * 32, a);
-        tmem_ld32(tl + 320 + h * 32, c);
-        tmem_wait_ld();
-      } else {
+    uint32_t a[32], c[32];
+    if (seq > 0) {
+      tc_fence_after();
+      tmem_ld32(tl + 256 + hf * 32, a);
+      tmem_ld32(tl + 320 + hf * 32, c);
+      tmem_wait_ld();
+    } else {
 #pragma unroll
-        for (int k = 0; k < 32; ++k) a[k] = c[k] = 0u;
-      }
-      if (jvalid) {
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          reinterpret_cast<float4*>(dv + h * 32)[k] =
-              make_float4(__uint_as_float(a[4 * k]), __uint_as_float(a[4 * k + 1]), __uint_as_float(a[4 * k + 2]),
-                          __uint_as_float(a[4 * k + 3]));
-          reinterpret_cast<float4*>(dk + h * 32)[k] =
-              make_float4(sc * __uint_as_float(c[4 * k]), sc * __uint_as_float(c[4 * k + 1]),
-                          sc * __uint_as_float(c[4 * k + 2]), sc * __uint_as_float(c[4 * k + 3]));
-        }
-      }
-      __syncwarp();
+      for (int k = 0; k < 32; ++k) a[k] = c[k] = 0u;
     }
+    if (jvalid) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        reinterpret_cast<float4*>(dv)[k] = make_float4(__uint_as_float(a[4 * k]), __uint_as_float(a[4 * k + 1]),
+                                                       __uint_as_float(a[4 * k + 2]), __uint_as_float(a[4 * k + 3]));
+        reinterpret_cast<float4*>(dk)[k] =
+            make_float4(sc * __uint_as_float(c[4 * k]), sc * __uint_as_float(c[4 * k + 1]),
+                        sc * __uint_as_float(c[4 * k + 2]), sc * __uint_as_float(c[4 * k + 3]));
+      }
+    }
+    __syncwarp();
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) tmem_dealloc(T, 512);
+  if (warp == kMmaWarp) tmem_dealloc(T, 512);
 }
 
 cudaError_t launch_bwd(bool alpha15, const BwdParams& p, int grid, cudaStream_t s) {

@@ -70,12 +70,13 @@ __device__ __forceinline__ void for_each_bit(const uint32_t* words, int nwords, 
   }
 }
 
-// Vote among the 128 row-owner threads (warps 0-3): true if any passes `pred`.
-// votes[r] must be zero before decision r; each decision uses its own slot.
-__device__ __forceinline__ bool rows_any(bool pred, int* votes, int r, int lane) {
+// Vote among the `nthreads` row-owner threads (warps 0..nthreads/32-1, named barrier 2):
+// true if any passes `pred`. votes[r] must be zero before decision r; each decision
+// uses its own slot.
+__device__ __forceinline__ bool rows_any(bool pred, int* votes, int r, int lane, int nthreads) {
   const unsigned bal = __ballot_sync(0xffffffffu, pred);
   if (lane == 0 && bal) atomicAdd(&votes[r], 1);
-  named_bar(2, 128);
+  named_bar(2, nthreads);
   return *reinterpret_cast<volatile int*>(&votes[r]) > 0;
 }
 

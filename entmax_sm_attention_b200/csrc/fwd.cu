@@ -1,37 +1,42 @@
 // fwd.cu -- fused alpha-entmax attention forward for sm_100a.
 //
-// One CTA per (batch*head, 128-row query tile) computes the four phases of
-// "AdaSplash-2: Faster Differentiable Sparse Attention", §3.3:
+// One CTA per (batch*head, 128-row query tile) computes the phases of "AdaSplash-2:
+// Faster Differentiable Sparse Attention", §3.3:
 //   Phase 1 (maximum): stream the structurally active key tiles; S = Q K^T on the
-//     tensor cores (tcgen05, accumulator in TMEM). Each row keeps its running max and
-//     its max in every key tile (kept in shared memory).
+//     tensor cores (tcgen05, accumulator in TMEM). Each row keeps its max in every key
+//     tile, in shared memory.
 //   Initial threshold: the row's tau restricted to its key-tile maxima. Entmax on a
 //     subset of the scores has a smaller threshold than on all of them (fewer
-//     nonnegative terms in Eq. 4), so this is a lower bound on tau*. It plays the role
-//     the paper gives its on-chip histogram (Phase 2): it costs no extra pass over K,
-//     because the tile maxima come out of Phase 1.
-//   Phase 3 (refinement): full sweeps over the key tiles that can still hold support
-//     (tile max above the row's current tau). Per row they accumulate count, S1 =
-//     sum u, S2 = sum u^2 with u = [z - tau]_+, then take a Newton step on Eq. 4,
-//     safeguarded by the bracket of §2.4 with bisection when the step leaves it (§3.2
-//     "safeguarded hybrid solver"). Eq. 4 is convex and decreasing for alpha <= 2, so
-//     Newton from the left never overshoots. A row stops when |f(tau)| <= kTolF; then
-//     one last Newton correction is applied without another sweep.
+//     nonnegative terms in Eq. 4), so this is a lower bound tau_T <= tau*. It plays the
+//     role the paper gives its on-chip histogram (Phase 2), without an extra pass over K.
+//   Phase 3 (refinement): one sweep at tau_T accumulates count, S1 = sum u, S2 = sum u^2
+//     (u = [z - tau]_+) and copies every score with u > 0 (the only candidates for the
+//     support, since tau* >= tau_T) into shared memory. Rows whose candidates fit are
+//     solved exactly on chip: safeguarded Newton on Eq. 4 (§3.2), finished by the exact
+//     root of the current support's piece (alpha = 2: (S1-1)/C; alpha = 1.5: the smaller
+//     root of C d^2 - 2 S1 d + S2 - 1 = 0) once no candidate leaves the support. Rows
+//     whose candidates overflow take Newton steps bracketed by §2.4, one full sweep each.
 //   Block mask: bit (query tile, key tile) = some row has a key-tile max above its
-//     final tau. Packed 32 key tiles per uint32 (Appendix C.4), plus the transpose
-//     for the backward.
+//     final tau. Packed 32 key tiles per uint32 (Appendix C.4), plus the transpose for
+//     the backward.
 //   Phase 4 (output): only the flagged key tiles. Recompute S and form
 //     A = u^{1/(alpha-1)} and g = u^{(2-alpha)/(alpha-1)}. Each is written to TMEM as a
 //     two-term bf16 split (hi + lo); A goes over the S columns it replaces. Then the
-//     tensor cores compute O += A V and Ot += g V, reading the A operand from TMEM.
-//     The split keeps the products at about fp32 accuracy: a single bf16 term (2^-8
-//     relative) would cost more than the gradient tolerance once it reaches dK through
-//     delta. sum_j g_ij is kept per row for the backward.
+//     tensor cores compute O += A V and Ot += g V, reading the A operand from TMEM. The
+//     split keeps the products at about fp32 accuracy: a single bf16 term (2^-8 relative)
+//     would cost more than the gradient tolerance once it reaches dK through delta.
+//     sum_j g_ij is kept per row for the backward.
 //
-// Roles: warps 0-3 own one query row per thread (TMEM lane = row); warp 4 issues the
-// TMA loads (a 3-slot ring of 16 KB K/V tiles); warp 5 owns TMEM and issues the MMAs.
-// TMEM (512 columns): [0,128) S tile, overwritten by A hi/lo; [128,256) g hi/lo;
-// [256,320) O; [320,384) Ot. Per 32-key quarter q: hi at +32q, lo at +32q+16.
+// Roles (320 threads): warps 0-7 are row owners. Warp w reads TMEM lanes 32(w%4)..+31
+// (one query row per lane) and columns [64(w/4), 64(w/4)+64) of every S tile, so two
+// threads share a row and combine partial sums in shared memory. Warp 8 issues TMA
+// loads into a 4-slot ring of 16 KB K/V tiles. Warp 9 owns TMEM and issues the MMAs.
+// TMEM (512 columns): during the sweeps, four S buffers at 0/128/256/384, so the MMA
+// warp runs up to three tiles ahead. During the output pass:
+//   - two S buffers at 0 and 384; A hi/lo overwrite each buffer per 32-key quarter q
+//     (hi at 32q, lo at 32q+16);
+//   - g hi/lo at 128 + (same layout);
+//   - O at [256,320) and Ot at [320,384).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -39,9 +44,14 @@ namespace entmax {
 
 namespace {
 
-constexpr int kThreads = 192;
-constexpr int kSlots = 3;
-constexpr float kTolF = 3e-5f;   // stop when |f(tau)| = |sum p - 1| <= kTolF
+constexpr int kThreads = 320;
+constexpr int kMathThreads = 256;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kSlots = 4;
+constexpr int kSBufs = 4;
+constexpr int kCandPerThread = 32;     // candidates per (row, column half); 64 per row
+constexpr float kTolF = 3e-5f;         // |f(tau)| = |sum p - 1| small enough to stop sweeping
 constexpr int kMaxVotes = 72;
 
 constexpr int kKindSweep = 0;
@@ -49,7 +59,9 @@ constexpr int kKindOutput = 1;
 
 struct Shared {
   uint64_t full[kSlots], empty[kSlots];
-  uint64_t bar_q, s_full, s_free, pv_done;
+  uint64_t bar_q;
+  uint64_t s_full[kSBufs], s_free[kSBufs];     // sweeps: MMA -> rows, rows -> MMA
+  uint64_t o_full[2], o_ready[2], pv_done[2];  // output pass ping-pong
   uint32_t tmem_base;
   int abort_flag;
   int ctl_kind, ctl_buf;
@@ -61,6 +73,13 @@ struct Shared {
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
+
+// Order-preserving float <-> int map (shared-memory atomicMax on floats).
+__device__ __forceinline__ int f2ord(float f) {
+  const int i = __float_as_int(f);
+  return i >= 0 ? i : i ^ 0x7fffffff;
+}
+__device__ __forceinline__ float ord2f(int i) { return __int_as_float(i >= 0 ? i : i ^ 0x7fffffff); }
 
 // Load 64 consecutive fp32 TMEM columns of this thread's lane.
 __device__ __forceinline__ void ld64(uint32_t taddr, float (&s)[64]) {
@@ -75,35 +94,52 @@ __device__ __forceinline__ void ld64(uint32_t taddr, float (&s)[64]) {
   }
 }
 
-// tau on the key-tile maxima of one row (a lower bound of the row's tau*, see above):
-// Newton on Eq. 4 from the bracket's left end, where f >= 0.
+__device__ __forceinline__ void accumulate(float u, float& S1, float& S2, float& C, float& umin) {
+  if (u > 0.f) {
+    S1 += u;
+    S2 = fmaf(u, u, S2);
+    C += 1.f;
+    umin = fminf(umin, u);
+  }
+}
+
+// Safeguarded solve of Eq. 4 for one row over raw scores vals0[k*stride] (k < n0) and
+// vals1[k*stride] (k < n1), which must hold every score that can be in the support.
+// u = fma(s, cz, -t). Starts at t (a lower bound) inside [lo, hi]; on success returns
+// true with the exact root up to fp32 rounding.
 template <int AK>
-__device__ float tau_on_tile_maxima(const float* tmax, const uint32_t (&act)[kMaskWords], int row, float cz,
-                                    float lo) {
-  float t = lo;
-  for (int it = 0; it < 40; ++it) {
-    float S1 = 0.f, S2 = 0.f, C = 0.f;
-    for (int w = 0; w < kMaskWords; ++w) {
-      uint32_t bits = act[w];
-      while (bits) {
-        int jt = w * 32 + __ffs(bits) - 1;
-        bits &= bits - 1;
-        float u = fmaf(tmax[jt * kTile + row], cz, -t);
-        if (u > 0.f) {
-          S1 += u;
-          S2 = fmaf(u, u, S2);
-          C += 1.f;
-        }
+__device__ bool solve_list(const float* vals0, int n0, const float* vals1, int n1, int stride, float cz, float t,
+                           float lo, float hi, float& t_out) {
+  for (int it = 0; it < 48; ++it) {
+    float S1 = 0.f, S2 = 0.f, C = 0.f, umin = INFINITY;
+    for (int k = 0; k < n0; ++k) accumulate(fmaf(vals0[k * stride], cz, -t), S1, S2, C, umin);
+    for (int k = 0; k < n1; ++k) accumulate(fmaf(vals1[k * stride], cz, -t), S1, S2, C, umin);
+    const float f = (AK == kAlpha15) ? S2 - 1.f : S1 - 1.f;
+    const float fp = (AK == kAlpha15) ? 2.f * S1 : C;   // |f'(t)|
+    if (C > 0.f) {
+      float d = -1.f;
+      if (AK == kAlpha15) {
+        const float disc = S1 * S1 - C * (S2 - 1.f);
+        if (disc >= 0.f) d = (S2 - 1.f) / (S1 + sqrtf(disc));   // = (S1 - sqrt(disc)) / C
+      } else {
+        d = (S1 - 1.f) / C;
+      }
+      if (d >= 0.f && d < umin) {   // no candidate leaves the support at t + d: exact
+        t_out = t + d;
+        return true;
       }
     }
-    float f = (AK == kAlpha15) ? S2 - 1.f : S1 - 1.f;
-    float fp = (AK == kAlpha15) ? 2.f * S1 : C;
-    if (!(fp > 0.f)) break;
-    float step = f / fp;
-    t += step;
-    if (fabsf(f) <= 1e-6f) break;
+    if (fabsf(f) <= 1e-7f && fp > 0.f) {
+      t_out = t + f / fp;
+      return true;
+    }
+    if (f > 0.f) lo = t; else hi = t;
+    float tn = t + f / fp;
+    if (!(tn > lo && tn < hi)) tn = 0.5f * (lo + hi);
+    t = tn;
   }
-  return t;
+  t_out = t;
+  return false;
 }
 
 }  // namespace
@@ -115,7 +151,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
   uint8_t* dsm = align1024(dsm_raw);
   uint8_t* sQ = dsm;
   uint8_t* ring = dsm + kTileBytes;
-  float* tmax = reinterpret_cast<float*>(dsm + kTileBytes * (1 + kSlots));  // [Tc][128]
+  int* tmax = reinterpret_cast<int*>(dsm + kTileBytes * (1 + kSlots));   // [Tc][128], f2ord
+  float* cand = reinterpret_cast<float*>(tmax + p.Tc * kTile);           // [2 halves][32][128]
+  float* part = cand + 2 * kCandPerThread * kTile;                       // [2 halves][4][128]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bh = blockIdx.x % p.BH;
@@ -132,9 +170,15 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       mbar_init(&sh.empty[s], 1);
     }
     mbar_init(&sh.bar_q, 1);
-    mbar_init(&sh.s_full, 1);
-    mbar_init(&sh.s_free, 4);
-    mbar_init(&sh.pv_done, 1);
+    for (int s = 0; s < kSBufs; ++s) {
+      mbar_init(&sh.s_full[s], 1);
+      mbar_init(&sh.s_free[s], 8);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sh.o_full[s], 1);
+      mbar_init(&sh.o_ready[s], 8);
+      mbar_init(&sh.pv_done[s], 1);
+    }
     sh.abort_flag = 0;
     fence_mbar_init();
   }
@@ -144,7 +188,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     sh.lists[1][tid] = 0;
   }
   for (int v = tid; v < kMaxVotes; v += kThreads) sh.votes[v] = 0;
-  if (warp == 5) {
+  for (int e = tid; e < p.Tc * kTile; e += kThreads) tmax[e] = f2ord(-INFINITY);
+  if (warp == kMmaWarp) {
     tmem_alloc(&sh.tmem_base, 512);
     tmem_relinquish();
   }
@@ -159,8 +204,10 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
 #pragma unroll
   for (int w = 0; w < kMaskWords; ++w) act[w] = sh.act[w];
 
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------------------ TMA producer
+    // Ring positions are taken in program order: every tile of phase 1 and of each
+    // sweep is one K load; the output pass loads K_k, V_k, K_{k+1}, V_{k+1}, ...
     uint32_t seq = 0;
     auto load = [&](const CUtensorMap* map, int jt) {
       const int slot = seq % kSlots;
@@ -199,36 +246,41 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     }
     // Make sure no copy is still in flight when the CTA retires.
     if (lane == 0) {
-      for (uint32_t k = (seq > kSlots ? seq - kSlots : 0); k < seq; ++k) {
-        volatile int no_abort = 0;
+      volatile int no_abort = 0;
+      for (uint32_t k = (seq > kSlots ? seq - kSlots : 0); k < seq; ++k)
         mbar_wait(&sh.full[k % kSlots], (k / kSlots) & 1, status, &no_abort);
-      }
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------- MMA issuer
-    uint32_t seq = 0, n_s = 0, n_pv = 0;
+    uint32_t seq = 0;            // next ring position (sweeps consume in order)
+    uint32_t sfree_par = 0;      // per sweep S buffer: parity of its uses so far (bit b)
+    uint32_t sbuf = 0;           // next sweep S buffer
     const uint32_t idS = idesc_bf16(128, 128, 0, 0);
     const uint32_t idO = idesc_bf16(128, 64, 0, 1);
     const uint32_t sQa = smem_u32(sQ);
-    auto issue_s = [&]() {
-      const int slot = seq % kSlots;
-      mbar_wait(&sh.full[slot], (seq / kSlots) & 1, status, abrt);
-      if (n_s > 0) mbar_wait(&sh.s_free, (n_s - 1) & 1, status, abrt);
-      if (n_pv > 0) mbar_wait(&sh.pv_done, (n_pv - 1) & 1, status, abrt);
+    // S = Q K^T from ring position `pos` into TMEM columns [dcol, dcol+128).
+    auto mma_s = [&](uint32_t pos, uint32_t dcol) {
+      const int slot = pos % kSlots;
+      mbar_wait(&sh.full[slot], (pos / kSlots) & 1, status, abrt);
       tc_fence_after();
       const uint32_t kb = smem_u32(ring + slot * kTileBytes);
 #pragma unroll
       for (int k = 0; k < 4; ++k)
-        mma_ss(T, sdesc_sw128(sQa + k * 32, 16, 1024), sdesc_sw128(kb + k * 32, 16, 1024), idS, k > 0);
+        mma_ss(T + dcol, sdesc_sw128(sQa + k * 32, 16, 1024), sdesc_sw128(kb + k * 32, 16, 1024), idS, k > 0);
       mma_commit(&sh.empty[slot]);
-      mma_commit(&sh.s_full);
-      ++n_s;
-      ++seq;
+    };
+    auto sweep_tile = [&]() {
+      const uint32_t bf = sbuf;
+      mbar_wait(&sh.s_free[bf], ((sfree_par >> bf) & 1) ^ 1, status, abrt);   // buffer consumed
+      sfree_par ^= 1u << bf;
+      mma_s(seq++, bf * 128);
+      mma_commit(&sh.s_full[bf]);
+      sbuf = (sbuf + 1) & (kSBufs - 1);
     };
     if (lane == 0) {
       mbar_wait(&sh.bar_q, 0, status, abrt);
-      for_each_bit(act, kMaskWords, [&](int) { issue_s(); });
+      for_each_bit(act, kMaskWords, [&](int) { sweep_tile(); });
     }
     __syncwarp();
     while (true) {
@@ -239,31 +291,47 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       for (int w = 0; w < kMaskWords; ++w) list[w] = sh.lists[sh.ctl_buf][w];
       if (lane == 0) {
         if (kind == kKindSweep) {
-          for_each_bit(list, kMaskWords, [&](int) { issue_s(); });
+          sbuf = 0;
+          for_each_bit(list, kMaskWords, [&](int) { sweep_tile(); });
         } else {
-          for_each_bit(list, kMaskWords, [&](int) {
-            issue_s();
-            const int slot = seq % kSlots;
-            mbar_wait(&sh.full[slot], (seq / kSlots) & 1, status, abrt);
-            mbar_wait(&sh.s_free, (n_s - 1) & 1, status, abrt);   // A and g written
+          // Output pass. S of tile k+1 is issued before PV of tile k, so it overlaps the
+          // row owners' work on tile k. Buffer c = k % 2 sits at TMEM column 0 or 384.
+          // K_k is at ring position base + 2k, V_k at base + 2k + 1.
+          int n = 0;
+#pragma unroll
+          for (int w = 0; w < kMaskWords; ++w) n += __popc(list[w]);
+          const uint32_t base = seq;
+          auto issue_s = [&](int k) {
+            const int c = k & 1;
+            if (k >= 2) mbar_wait(&sh.pv_done[c], ((k - 2) >> 1) & 1, status, abrt);   // buffer c free
+            mma_s(base + 2 * k, c ? 384u : 0u);
+            mma_commit(&sh.o_full[c]);
+          };
+          if (n > 0) issue_s(0);
+          for (int k = 0; k < n; ++k) {
+            if (k + 1 < n) issue_s(k + 1);
+            const int c = k & 1;
+            const uint32_t pa = c ? 384u : 0u;
+            const uint32_t vpos = base + 2 * k + 1;
+            const int vslot = vpos % kSlots;
+            mbar_wait(&sh.full[vslot], (vpos / kSlots) & 1, status, abrt);
+            mbar_wait(&sh.o_ready[c], (k >> 1) & 1, status, abrt);   // A and g of tile k written
             tc_fence_after();
-            const uint32_t vb = smem_u32(ring + slot * kTileBytes);
+            const uint32_t vb = smem_u32(ring + vslot * kTileBytes);
 #pragma unroll
             for (int t = 0; t < 8; ++t) {
-              // key step t = quarter t/2, half t%2; hi at +0, lo at +16 within the quarter
-              const uint32_t col = (t >> 1) * 32 + (t & 1) * 8;
+              const uint32_t col = (t >> 1) * 32 + (t & 1) * 8;   // key quarter t/2, half t%2
               const uint64_t bd = sdesc_sw128(vb + t * 2048, 8192, 1024);
-              const uint32_t acc = (n_pv > 0 || t > 0) ? 1u : 0u;
-              mma_ts(T + 256, T + col, bd, idO, acc);
-              mma_ts(T + 256, T + col + 16, bd, idO, 1u);
+              const uint32_t acc = (k > 0 || t > 0) ? 1u : 0u;
+              mma_ts(T + 256, T + pa + col, bd, idO, acc);
+              mma_ts(T + 256, T + pa + col + 16, bd, idO, 1u);
               mma_ts(T + 320, T + 128 + col, bd, idO, acc);
               if (AK == kAlpha15) mma_ts(T + 320, T + 128 + col + 16, bd, idO, 1u);
             }
-            mma_commit(&sh.empty[slot]);
-            mma_commit(&sh.pv_done);
-            ++n_pv;
-            ++seq;
-          });
+            mma_commit(&sh.empty[vslot]);
+            mma_commit(&sh.pv_done[c]);
+          }
+          seq = base + 2 * n;
         }
       }
       __syncwarp();
@@ -271,71 +339,93 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     }
   } else {
     // ---------------------------------------------------------------- row owners
-    const int row = tid;
+    const int quad = warp & 3, hf = warp >> 2;   // TMEM lane quadrant, column half
+    const int row = quad * 32 + lane;
     const int i = i0 + row;
     const bool valid = i < p.L;
-    const uint32_t tl = T + ((uint32_t)(warp * 32) << 16);
+    const uint32_t tl = T + ((uint32_t)(quad * 32) << 16);
     const float cz = p.cz;
-    uint32_t n_s = 0;
+    uint32_t sfull_par = 0, sbuf = 0;
     float m = -INFINITY;
 
-    // Phase 1: row max and per-key-tile maxima.
+    // Phase 1: per-key-tile row maxima over this thread's column half (combined in smem).
     for_each_bit(act, kMaskWords, [&](int jt) {
-      warp_wait(&sh.s_full, n_s & 1, status, abrt);
+      const uint32_t bf = sbuf;
+      warp_wait(&sh.s_full[bf], (sfull_par >> bf) & 1, status, abrt);
+      sfull_par ^= 1u << bf;
       tc_fence_after();
-      const int j0 = jt * kTile;
-      const bool full = pat.block_full(i0, i1, j0, j0 + kTile);
-      float tm = -INFINITY;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        float s[64];
-        ld64(tl + h * 64, s);
-        if (full) {
-#pragma unroll
-          for (int c = 0; c < 64; ++c) tm = fmaxf(tm, s[c]);
-        } else {
-#pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if (pat.active(i, j0 + h * 64 + c)) tm = fmaxf(tm, s[c]);
-        }
-      }
+      const int j0 = jt * kTile + hf * 64;
+      float s[64];
+      ld64(tl + bf * 128 + hf * 64, s);
       tc_fence_before();
-      warp_arrive(&sh.s_free);
-      tmax[jt * kTile + row] = tm;
+      warp_arrive(&sh.s_free[bf]);
+      if (!pat.block_full(i0, i1, jt * kTile, jt * kTile + kTile)) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          if (!pat.active(i, j0 + c)) s[c] = -INFINITY;
+      }
+      float t8[8];   // eight independent max chains
+#pragma unroll
+      for (int c = 0; c < 8; ++c) t8[c] = s[c];
+#pragma unroll
+      for (int c = 8; c < 64; ++c) t8[c & 7] = fmaxf(t8[c & 7], s[c]);
+      const float tm = fmaxf(fmaxf(fmaxf(t8[0], t8[1]), fmaxf(t8[2], t8[3])),
+                             fmaxf(fmaxf(t8[4], t8[5]), fmaxf(t8[6], t8[7])));
+      atomicMax(&tmax[jt * kTile + row], f2ord(tm));
       m = fmaxf(m, tm);
-      ++n_s;
+      sbuf = (sbuf + 1) & (kSBufs - 1);
     });
+    // Row max over both column halves.
+    part[hf * 4 * kTile + row] = m;
+    named_bar(3, kMathThreads);
+    m = fmaxf(part[row], part[4 * kTile + row]);
 
-    // Bracket (§2.4) and the tile-maxima lower bound.
+    // Bracket (§2.4) and the tile-maxima lower bound (identical in both threads of a row).
     const int n_act = valid ? pat.count(i) : 1;
     const float mz = m * cz;
     float lo = mz - 1.f;
     float hi = mz - ((AK == kAlpha15) ? rsqrtf((float)n_act) : 1.f / (float)n_act);
-    float tau = valid ? tau_on_tile_maxima<AK>(tmax, act, row, cz, lo) : INFINITY;
-    tau = fminf(fmaxf(tau, lo), hi);
-    if (!valid) tau = INFINITY;
+    float tau = INFINITY;
     bool done = !valid;
-    float sg = 0.f;
+    if (valid) {
+      // Only tile maxima above lo = m - 1 can be in the support of the maxima problem.
+      // Gather up to 32 of them into this thread's candidate area (unused until the
+      // first sweep). Entmax on any subset of the scores has a threshold <= tau*, so
+      // keeping only the first 32 still gives a lower bound.
+      float* mylist = cand + hf * kCandPerThread * kTile + row;
+      int nl = 0;
+      for_each_bit(act, kMaskWords, [&](int jt) {
+        const float v = ord2f(tmax[jt * kTile + row]);
+        if (nl < kCandPerThread && fmaf(v, cz, -lo) > 0.f) mylist[nl++ * kTile] = v;
+      });
+      float t = lo;
+      solve_list<AK>(mylist, nl, mylist, 0, kTile, cz, lo, lo, hi, t);
+      tau = fminf(fmaxf(t, lo), hi);
+    }
+    float2 sg2 = make_float2(0.f, 0.f);   // sum_j g_ij, two chains
     int sweeps = 0;
+    uint32_t n_s = 0;   // S tiles computed (phase 1, sweeps, output) for the counters
+    for_each_bit(act, kMaskWords, [&](int) { ++n_s; });
 
     // Decision points: publish either one more refinement sweep or the final mask.
     for (int r = 0;; ++r) {
       const int buf = r & 1;
       const bool need = !done && sweeps < p.max_sweeps;
-      const bool final_mask = !rows_any(need, sh.votes, r, lane);
-      // Tiles that some row still needs (refinement) or that hold a nonzero (mask).
-      for_each_bit(act, kMaskWords, [&](int jt) {
-        const bool take = final_mask ? valid : !done;
-        const bool hit = take && fmaf(tmax[jt * kTile + row], cz, -tau) > 0.f;
-        const uint32_t bal = __ballot_sync(0xffffffffu, hit);
-        if (lane == 0 && bal) atomicOr(&sh.lists[buf][jt >> 5], 1u << (jt & 31));
-      });
-      named_bar(2, 128);
+      const bool final_mask = !rows_any(need, sh.votes, r, lane, kMathThreads);
+      if (hf == 0) {
+        // Tiles that some row still needs (refinement) or that hold a nonzero (mask).
+        for_each_bit(act, kMaskWords, [&](int jt) {
+          const bool take = final_mask ? valid : !done;
+          const bool hit = take && fmaf(ord2f(tmax[jt * kTile + row]), cz, -tau) > 0.f;
+          const uint32_t bal = __ballot_sync(0xffffffffu, hit);
+          if (lane == 0 && bal) atomicOr(&sh.lists[buf][jt >> 5], 1u << (jt & 31));
+        });
+      }
+      named_bar(2, kMathThreads);
       if (tid == 0) {
         sh.ctl_kind = final_mask ? kKindOutput : kKindSweep;
         sh.ctl_buf = buf;
-        // clear the other buffer for the next decision (nobody reads it any more)
-        for (int w = 0; w < kMaskWords; ++w) sh.lists[buf ^ 1][w] = 0;
+        for (int w = 0; w < kMaskWords; ++w) sh.lists[buf ^ 1][w] = 0;   // for the next decision
       }
       uint32_t list[kMaskWords];
 #pragma unroll
@@ -343,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       named_bar(1, kThreads);
 
       if (final_mask) {
-        if (!done) atomicOr(status, kStatusNoConverge);   // cap reached; tau stays bracketed
+        if (!done && hf == 0) atomicOr(status, kStatusNoConverge);   // cap reached; tau stays bracketed
         // Block mask row of this query tile and the transposed bits (Appendix C.4).
         if (tid < p.Wc) p.M[((size_t)bh * p.Tr + qt) * p.Wc + tid] = list[tid];
         if (tid == 0) {
@@ -351,123 +441,208 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
             atomicOr(&p.MT[((size_t)bh * p.Tc + jt) * p.Wr + (qt >> 5)], 1u << (qt & 31));
           });
         }
-        // Phase 4: output sweep over the flagged tiles.
-        int n_out = 0;
+        // Phase 4: output pass over the flagged tiles, ping-pong buffers c = k % 2.
+        int k = 0;
         for_each_bit(list, kMaskWords, [&](int jt) {
-          warp_wait(&sh.s_full, n_s & 1, status, abrt);
+          const int c = k & 1;
+          const uint32_t pa = c ? 384u : 0u;
+          warp_wait(&sh.o_full[c], (k >> 1) & 1, status, abrt);
           tc_fence_after();
-          const int j0 = jt * kTile;
-          const bool full = pat.block_full(i0, i1, j0, j0 + kTile);
+          const int j0 = jt * kTile + hf * 64;
+          float s[64];
+          ld64(tl + pa + hf * 64, s);
+          if (!pat.block_full(i0, i1, jt * kTile, jt * kTile + kTile)) {
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            float s[64];
-            ld64(tl + h * 64, s);
-            if (!full) {
+            for (int cc = 0; cc < 64; ++cc)
+              if (!pat.active(i, j0 + cc)) s[cc] = -INFINITY;
+          }
 #pragma unroll
-              for (int c = 0; c < 64; ++c)
-                if (!pat.active(i, j0 + h * 64 + c)) s[c] = -INFINITY;
-            }
+          for (int q = 0; q < 2; ++q) {
+            uint32_t ah[16], al[16];
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
-              uint32_t ah[16], al[16], gh[16], gl[16];
-#pragma unroll
-              for (int c = 0; c < 16; ++c) {
-                const float u0 = fmaf(s[q * 32 + 2 * c], cz, -tau);
-                const float u1 = fmaf(s[q * 32 + 2 * c + 1], cz, -tau);
-                const float v0 = fmaxf(u0, 0.f), v1 = fmaxf(u1, 0.f);
-                if (AK == kAlpha15) {
-                  split_bf16x2(v0 * v0, v1 * v1, ah[c], al[c]);
-                  split_bf16x2(v0, v1, gh[c], gl[c]);
-                  sg += v0 + v1;
-                } else {
-                  const float g0 = u0 > 0.f ? 1.f : 0.f, g1 = u1 > 0.f ? 1.f : 0.f;
-                  split_bf16x2(v0, v1, ah[c], al[c]);
-                  gh[c] = pack_bf16(g0, g1);   // 0 and 1 are exact in bf16
-                  sg += g0 + g1;
-                }
+            for (int cc = 0; cc < 16; ++cc) {
+              const float2 u = __ffma2_rn(make_float2(s[q * 32 + 2 * cc], s[q * 32 + 2 * cc + 1]),
+                                          make_float2(cz, cz), make_float2(-tau, -tau));
+              const float v0 = fmaxf(u.x, 0.f), v1 = fmaxf(u.y, 0.f);
+              if (AK == kAlpha15) {
+                const float2 a = __fmul2_rn(make_float2(v0, v1), make_float2(v0, v1));
+                split_bf16x2(a.x, a.y, ah[cc], al[cc]);
+              } else {
+                split_bf16x2(v0, v1, ah[cc], al[cc]);
               }
-              const uint32_t col = h * 64 + q * 32;   // key quarter (2h + q)
-              tmem_st16(tl + col, ah);
-              tmem_st16(tl + col + 16, al);
-              tmem_st16(tl + 128 + col, gh);
-              if (AK == kAlpha15) tmem_st16(tl + 128 + col + 16, gl);
             }
+            const uint32_t col = hf * 64 + q * 32;   // key quarter 2hf + q
+            tmem_st16(tl + pa + col, ah);
+            tmem_st16(tl + pa + col + 16, al);
+          }
+          // g shares one TMEM region across tiles: PV of tile k-1 must have read it.
+          if (k >= 1) warp_wait(&sh.pv_done[(k - 1) & 1], ((k - 1) >> 1) & 1, status, abrt);
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            uint32_t gh[16], gl[16];
+#pragma unroll
+            for (int cc = 0; cc < 16; ++cc) {
+              const float2 u = __ffma2_rn(make_float2(s[q * 32 + 2 * cc], s[q * 32 + 2 * cc + 1]),
+                                          make_float2(cz, cz), make_float2(-tau, -tau));
+              const float v0 = fmaxf(u.x, 0.f), v1 = fmaxf(u.y, 0.f);
+              if (AK == kAlpha15) {
+                split_bf16x2(v0, v1, gh[cc], gl[cc]);
+                sg2 = __fadd2_rn(sg2, make_float2(v0, v1));
+              } else {
+                const float g0 = u.x > 0.f ? 1.f : 0.f, g1 = u.y > 0.f ? 1.f : 0.f;
+                gh[cc] = pack_bf16(g0, g1);   // 0 and 1 are exact in bf16
+                sg2 = __fadd2_rn(sg2, make_float2(g0, g1));
+              }
+            }
+            const uint32_t col = hf * 64 + q * 32;
+            tmem_st16(tl + 128 + col, gh);
+            if (AK == kAlpha15) tmem_st16(tl + 128 + col + 16, gl);
           }
           tmem_wait_st();
           tc_fence_before();
-          warp_arrive(&sh.s_free);
+          warp_arrive(&sh.o_ready[c]);
+          ++k;
           ++n_s;
-          ++n_out;
         });
-        // Epilogue: O and Ot from TMEM.
-        warp_wait(&sh.pv_done, (n_out - 1) & 1, status, abrt);
+        const int n_out = k;
+        // Epilogue: O and Ot from TMEM (each thread of a row writes 32 of the 64 columns).
+        warp_wait(&sh.pv_done[(n_out - 1) & 1], ((n_out - 1) >> 1) & 1, status, abrt);
         tc_fence_after();
-        float o[64];
-        ld64(tl + 256, o);
+        part[(hf * 4 + 1) * kTile + row] = sg2.x + sg2.y;
+        uint32_t o[32];
+        tmem_ld32(tl + 256 + hf * 32, o);
+        tmem_wait_ld();
         if (valid) {
-          float4* dst = reinterpret_cast<float4*>(p.O + ((size_t)bh * p.L + i) * kD);
+          float4* dst = reinterpret_cast<float4*>(p.O + ((size_t)bh * p.L + i) * kD + hf * 32);
 #pragma unroll
-          for (int c = 0; c < 16; ++c) dst[c] = make_float4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+          for (int cc = 0; cc < 8; ++cc)
+            dst[cc] = make_float4(__uint_as_float(o[4 * cc]), __uint_as_float(o[4 * cc + 1]),
+                                  __uint_as_float(o[4 * cc + 2]), __uint_as_float(o[4 * cc + 3]));
         }
         __syncwarp();
-        ld64(tl + 320, o);
+        tmem_ld32(tl + 320 + hf * 32, o);
+        tmem_wait_ld();
         if (valid) {
-          float4* dst = reinterpret_cast<float4*>(p.Ot + ((size_t)bh * p.L + i) * kD);
+          float4* dst = reinterpret_cast<float4*>(p.Ot + ((size_t)bh * p.L + i) * kD + hf * 32);
 #pragma unroll
-          for (int c = 0; c < 16; ++c) dst[c] = make_float4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+          for (int cc = 0; cc < 8; ++cc)
+            dst[cc] = make_float4(__uint_as_float(o[4 * cc]), __uint_as_float(o[4 * cc + 1]),
+                                  __uint_as_float(o[4 * cc + 2]), __uint_as_float(o[4 * cc + 3]));
+        }
+        named_bar(3, kMathThreads);
+        if (valid && hf == 0) {
           p.tau[(size_t)bh * p.L + i] = tau;
-          p.sumg[(size_t)bh * p.L + i] = sg;
+          p.sumg[(size_t)bh * p.L + i] = part[1 * kTile + row] + part[5 * kTile + row];
         }
         if (tid == 0) {
-          int n_act = 0;
-          for (int w = 0; w < kMaskWords; ++w) n_act += __popc(act[w]);
+          int na = 0;
+          for (int w = 0; w < kMaskWords; ++w) na += __popc(act[w]);
           int4* st = reinterpret_cast<int4*>(p.stats) + (size_t)bh * p.Tr + qt;
-          *st = make_int4(sweeps, (int)n_s, n_out, n_act);
+          *st = make_int4(sweeps, (int)n_s, n_out, na);
         }
         break;
       }
 
-      // Phase 3: one refinement sweep.
+      // Phase 3: one refinement sweep at the current tau. The first one (at tau_T) also
+      // collects this thread's candidates u > 0.
+      const bool collect = (sweeps == 0);
       float S1 = 0.f, S2 = 0.f, C = 0.f;
+      int nc = 0;
+      float* mycand = cand + hf * kCandPerThread * kTile + row;
+      sbuf = 0;
       for_each_bit(list, kMaskWords, [&](int jt) {
-        warp_wait(&sh.s_full, n_s & 1, status, abrt);
+        const uint32_t bf = sbuf;
+        warp_wait(&sh.s_full[bf], (sfull_par >> bf) & 1, status, abrt);
+        sfull_par ^= 1u << bf;
         tc_fence_after();
-        const int j0 = jt * kTile;
-        const bool full = pat.block_full(i0, i1, j0, j0 + kTile);
+        const int j0 = jt * kTile + hf * 64;
+        float s[64];
+        ld64(tl + bf * 128 + hf * 64, s);
+        tc_fence_before();
+        warp_arrive(&sh.s_free[bf]);
+        if (!pat.block_full(i0, i1, jt * kTile, jt * kTile + kTile)) {
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          float s[64];
-          ld64(tl + h * 64, s);
-          if (!full) {
+          for (int cc = 0; cc < 64; ++cc)
+            if (!pat.active(i, j0 + cc)) s[cc] = -INFINITY;
+        }
+        float2 s1[4], s2[4];
+        int cnt[4];
 #pragma unroll
-            for (int c = 0; c < 64; ++c)
-              if (!pat.active(i, j0 + h * 64 + c)) s[c] = -INFINITY;
+        for (int a = 0; a < 4; ++a) {
+          s1[a] = make_float2(0.f, 0.f);
+          s2[a] = make_float2(0.f, 0.f);
+          cnt[a] = 0;
+        }
+        if (collect) {
+#pragma unroll
+          for (int cc = 0; cc < 64; cc += 2) {
+            const float2 u = __ffma2_rn(make_float2(s[cc], s[cc + 1]), make_float2(cz, cz), make_float2(-tau, -tau));
+            const float2 v = make_float2(fmaxf(u.x, 0.f), fmaxf(u.y, 0.f));
+            const int a = (cc >> 1) & 3;
+            s1[a] = __fadd2_rn(s1[a], v);
+            s2[a] = __ffma2_rn(v, v, s2[a]);
+            // Candidates: predicated stores, no branches (the store slot is clamped).
+            if (u.x > 0.f) mycand[min(nc, kCandPerThread - 1) * kTile] = s[cc];
+            nc += u.x > 0.f;
+            if (u.y > 0.f) mycand[min(nc, kCandPerThread - 1) * kTile] = s[cc + 1];
+            nc += u.y > 0.f;
           }
+        } else {
 #pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            const float u = fmaf(s[c], cz, -tau);
-            const float v = fmaxf(u, 0.f);
-            S1 += v;
-            S2 = fmaf(v, v, S2);
-            C += u > 0.f ? 1.f : 0.f;
+          for (int cc = 0; cc < 64; cc += 2) {
+            const float2 u = __ffma2_rn(make_float2(s[cc], s[cc + 1]), make_float2(cz, cz), make_float2(-tau, -tau));
+            const float2 v = make_float2(fmaxf(u.x, 0.f), fmaxf(u.y, 0.f));
+            const int a = (cc >> 1) & 3;
+            s1[a] = __fadd2_rn(s1[a], v);
+            s2[a] = __ffma2_rn(v, v, s2[a]);
+            cnt[a] += (u.x > 0.f) + (u.y > 0.f);
           }
         }
-        tc_fence_before();
-        warp_arrive(&sh.s_free);
+        C += (float)(cnt[0] + cnt[1] + cnt[2] + cnt[3]);
+        const float2 s1t = __fadd2_rn(__fadd2_rn(s1[0], s1[1]), __fadd2_rn(s1[2], s1[3]));
+        const float2 s2t = __fadd2_rn(__fadd2_rn(s2[0], s2[1]), __fadd2_rn(s2[2], s2[3]));
+        S1 += s1t.x + s1t.y;
+        S2 += s2t.x + s2t.y;
         ++n_s;
+        sbuf = (sbuf + 1) & (kSBufs - 1);
       });
+      // Combine the two column halves of each row.
+      float* mp = part + hf * 4 * kTile + row;
+      mp[0] = S1;
+      mp[kTile] = S2;
+      mp[2 * kTile] = collect ? (float)nc : C;
+      mp[3 * kTile] = (float)nc;
+      named_bar(3, kMathThreads);
+      const float* p0 = part + row;
+      const float* p1 = part + 4 * kTile + row;
+      S1 = p0[0] + p1[0];
+      S2 = p0[kTile] + p1[kTile];
+      C = p0[2 * kTile] + p1[2 * kTile];
+      const int nc0 = (int)p0[3 * kTile], nc1 = (int)p1[3 * kTile];
+      named_bar(3, kMathThreads);   // partials consumed before anyone rewrites them
       ++sweeps;
       if (!done) {
         const float f = (AK == kAlpha15) ? S2 - 1.f : S1 - 1.f;
         const float fp = (AK == kAlpha15) ? 2.f * S1 : C;   // |f'(tau)|
-        if (fabsf(f) <= kTolF && fp > 0.f) {
-          tau += f / fp;     // final Newton correction, no further sweep needed
-          done = true;
-        } else {
-          if (f > 0.f) lo = tau; else hi = tau;
-          float t = tau + f / fp;
-          if (!(t > lo && t < hi)) t = 0.5f * (lo + hi);   // bisection safeguard
-          tau = t;
+        if (f > 0.f) lo = fmaxf(lo, tau); else hi = fminf(hi, tau);
+        if (collect && nc0 <= kCandPerThread && nc1 <= kCandPerThread) {
+          // Every score above tau_T <= tau* is in the two candidate lists: exact on chip.
+          float t;
+          if (solve_list<AK>(cand + row, nc0, cand + kCandPerThread * kTile + row, nc1, kTile, cz, tau, lo, hi,
+                             t)) {
+            tau = t;
+            done = true;
+          }
+        }
+        if (!done) {
+          if (fabsf(f) <= kTolF && fp > 0.f) {
+            tau += f / fp;   // final Newton correction, no further sweep needed
+            done = true;
+          } else {
+            float t = tau + f / fp;
+            if (!(t > lo && t < hi)) t = 0.5f * (lo + hi);   // bisection safeguard
+            tau = t;
+          }
         }
       }
     }
@@ -475,13 +650,11 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) tmem_dealloc(T, 512);
+  if (warp == kMmaWarp) tmem_dealloc(T, 512);
 }
 
-// At least 120 KB, so that one CTA holds an SM: it allocates all 512 TMEM columns.
 int fwd_smem_bytes(int Tc) {
-  const int need = 1024 + kTileBytes * (1 + kSlots) + Tc * kTile * 4;
-  return need > 120 * 1024 ? need : 120 * 1024;
+  return 1024 + kTileBytes * (1 + kSlots) + Tc * kTile * 4 + 2 * kCandPerThread * kTile * 4 + 8 * kTile * 4;
 }
 
 cudaError_t launch_fwd(bool alpha15, const FwdParams& p, int grid, cudaStream_t s) {

@@ -78,13 +78,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* s
   }
 }
 
-// Warp-wide variants for code that all 32 lanes execute. Each lane polls the barrier on
-// its own, so lanes can leave the wait at different times; the __syncwarp reconverges
-// the warp before the .sync.aligned tcgen05 instructions and bar.sync that follow.
+// Warp-wide variant for code that all 32 lanes execute: lane 0 polls the barrier (the
+// other lanes do not spin on shared memory), then __syncwarp reconverges the warp before
+// the .sync.aligned tcgen05 instructions and bar.sync that follow, and makes the
+// barrier's completion (and the memory it guards) visible to every lane.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, int* status, volatile int* abort) {
-  const bool ok = mbar_wait(bar, parity, status, abort);
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, status, abort) ? 1 : 0;
   __syncwarp();
-  return ok;
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  return ok != 0;
 }
 // One arrival per warp (lane 0), with the warp converged before and after.
 __device__ __forceinline__ void warp_arrive(uint64_t* bar) {
