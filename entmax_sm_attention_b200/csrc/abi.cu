@@ -66,7 +66,6 @@ entmax_status check_desc(const entmax_attn_desc* d) {
   if (d->d != kD) return ENTMAX_EUNSUPPORTED;
   if (d->L > ENTMAX_MAX_L) return ENTMAX_EUNSUPPORTED;
   if (d->alpha != 1.5f && d->alpha != 2.0f) return ENTMAX_EUNSUPPORTED;
-  if (d->dtype == ENTMAX_FP32) return ENTMAX_EUNSUPPORTED;
   return ENTMAX_OK;
 }
 
@@ -117,6 +116,34 @@ extern "C" entmax_status entmax_attn_fwd(const entmax_attn_desc* d, const void* 
   layout_of(d, &l);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* w = static_cast<uint8_t*>(ws);
+  if (cudaMemsetAsync(w + l.off_status, 0, 256, s) != cudaSuccess) return ENTMAX_ECUDA;
+  if (cudaMemsetAsync(w + l.off_MT, 0, l.bytes_MT, s) != cudaSuccess) return ENTMAX_ECUDA;
+  if (d->dtype == ENTMAX_FP32) {
+    FwdF32Params q;
+    std::memset(&q, 0, sizeof(q));
+    q.Q = static_cast<const float*>(Q);
+    q.K = static_cast<const float*>(K);
+    q.V = static_cast<const float*>(V);
+    q.O = O;
+    q.tau = tau;
+    q.M = reinterpret_cast<uint32_t*>(w + l.off_M);
+    q.MT = reinterpret_cast<uint32_t*>(w + l.off_MT);
+    q.stats = reinterpret_cast<int*>(w + l.off_stats);
+    q.status = reinterpret_cast<int*>(w + l.off_status);
+    q.kv_len = d->kv_len;
+    q.H = d->H;
+    q.L = d->L;
+    q.Tr = l.Tr;
+    q.Tc = l.Tc;
+    q.Wc = l.Wc;
+    q.Wr = l.Wr;
+    q.BH = l.BH;
+    q.cz = (d->alpha - 1.0f) * d->scale;
+    q.causal = d->causal || d->window >= 0;
+    q.window = d->window < 0 ? -1 : d->window;
+    q.max_sweeps = d->max_sweeps == 0 ? kDefaultSweeps : d->max_sweeps;
+    return launch_fwd_f32(d->alpha == 1.5f, q, l.BH * l.Tr, s) == cudaSuccess ? ENTMAX_OK : ENTMAX_ECUDA;
+  }
   FwdParams p;
   std::memset(&p, 0, sizeof(p));
   if (!make_map(&p.tQ, Q, d->L, l.BH) || !make_map(&p.tK, K, d->L, l.BH) || !make_map(&p.tV, V, d->L, l.BH))
@@ -141,8 +168,6 @@ extern "C" entmax_status entmax_attn_fwd(const entmax_attn_desc* d, const void* 
   p.causal = d->causal || d->window >= 0;
   p.window = d->window < 0 ? -1 : d->window;
   p.max_sweeps = d->max_sweeps == 0 ? kDefaultSweeps : d->max_sweeps;
-  if (cudaMemsetAsync(w + l.off_status, 0, 256, s) != cudaSuccess) return ENTMAX_ECUDA;
-  if (cudaMemsetAsync(p.MT, 0, l.bytes_MT, s) != cudaSuccess) return ENTMAX_ECUDA;
   return launch_fwd(d->alpha == 1.5f, p, l.BH * l.Tr, s) == cudaSuccess ? ENTMAX_OK : ENTMAX_ECUDA;
 }
 
@@ -151,6 +176,7 @@ extern "C" entmax_status entmax_attn_bwd(const entmax_attn_desc* d, const void* 
                                          float* dV, void* stream) {
   entmax_status st = check_desc(d);
   if (st != ENTMAX_OK) return st;
+  if (d->dtype != ENTMAX_BF16) return ENTMAX_EUNSUPPORTED;   // the fp32 path is forward-only
   if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(dO, 16) || !aligned(tau, 4) ||
       !aligned(ws, 256) || !aligned(dQ, 16) || !aligned(dK, 16) || !aligned(dV, 16))
     return ENTMAX_EINVAL;

@@ -38,11 +38,28 @@ struct BwdParams {
   int causal, window;
 };
 
+struct FwdF32Params {
+  const float* Q;           // fp32 [B*H][L][64]
+  const float* K;
+  const float* V;
+  float* O;
+  float* tau;
+  uint32_t* M;
+  uint32_t* MT;
+  int* stats;
+  int* status;
+  const int* kv_len;
+  int H, L, Tr, Tc, Wc, Wr, BH;
+  float cz;
+  int causal, window, max_sweeps;
+};
+
 // Host-side launchers (each defined next to its kernel). They set the kernel's
 // dynamic shared-memory limit and launch on `s`; they return the launch error.
 int fwd_smem_bytes(int Tc);
 int bwd_smem_bytes();
 cudaError_t launch_fwd(bool alpha15, const FwdParams& p, int grid, cudaStream_t s);
+cudaError_t launch_fwd_f32(bool alpha15, const FwdF32Params& p, int grid, cudaStream_t s);
 cudaError_t launch_bwd(bool alpha15, const BwdParams& p, int grid, cudaStream_t s);
 cudaError_t launch_delta(const uint16_t* dO, const float* Ot, const float* sumg, float* delta, long rows,
                          cudaStream_t s);

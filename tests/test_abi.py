@@ -61,6 +61,7 @@ def test_workspace_bytes_valid_and_invalid(lib):
 @pytest.mark.parametrize("bad,code", [
     (dict(d=128), eb.ENTMAX_EUNSUPPORTED),
     (dict(alpha=3.0), eb.ENTMAX_EUNSUPPORTED),
+    (dict(dtype=9), eb.ENTMAX_EINVAL),
     (dict(L=eb.ENTMAX_MAX_L + 128), eb.ENTMAX_EUNSUPPORTED),
     (dict(B=-1), eb.ENTMAX_EINVAL),
     (dict(scale=float("nan")), eb.ENTMAX_EINVAL),

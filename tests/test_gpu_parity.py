@@ -79,3 +79,35 @@ def test_repeatable():
     for k in ("O", "tau", "dK", "dV", "M"):
         assert np.array_equal(a[k], b[k]), k
     assert np.abs(a["dQ"] - b["dQ"]).max() < 1e-5
+
+
+def test_single_head_fp32_workload():
+    """B=H=1, L=128, fp32 Q, K, V, non-causal: forward against the oracle, plus
+    entmax_rows on the same 128 x 128 score matrix S = Q K^T / sqrt(d)."""
+    from entmax_sm_attention_b200.workloads import WORKLOADS, make_inputs
+    from parity import check_mask, gpu_run, oracle_problem
+
+    w = WORKLOADS["single_head_L128_fp32"]
+    inp = make_inputs(w, seed=0)
+    assert inp["Q"].dtype == torch.float32
+    g = gpu_run(inp, w, 1.5, backward=False)
+    assert g["status"][0] == eb.ENTMAX_OK
+    pr = oracle_problem(inp, w, 1.5)
+    ref = pr.forward()
+    assert np.abs(g["tau"] - ref["tau"]).max() <= TOL_TAU
+    assert np.abs(g["O"] - ref["O"]).max() <= 1e-2
+    assert check_mask(pr, ref["tau"], g["M"])[0] == 0
+    # entmax_rows on the explicit scores (computed in fp32 on the GPU by torch: plumbing)
+    S = (inp["Q"][0, 0].cuda() @ inp["K"][0, 0].cuda().T) * w.scale
+    P, tau = eb.rows(S.contiguous(), 1.5)
+    Pr, taur = oracle.entmax_rows(S.cpu(), 1.5)
+    assert np.abs(tau.cpu().numpy() - taur).max() <= 1e-5
+    assert np.abs(P.cpu().numpy() - Pr).max() <= 1e-5
+
+
+def test_fp32_backward_is_rejected():
+    d = {k: torch.zeros(1, 1, 128, 64, device="cuda") for k in ("Q", "K", "V", "dO")}
+    O, tau, ctx = eb.forward(d["Q"], d["K"], d["V"])
+    with pytest.raises(eb.EntmaxError) as e:
+        eb.backward(ctx, d["Q"], d["K"], d["V"], d["dO"], tau)
+    assert e.value.code == eb.ENTMAX_EUNSUPPORTED
