@@ -15,9 +15,10 @@ import torch
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libentmax_attn.so")
 
-ENTMAX_OK, ENTMAX_EINVAL, ENTMAX_EUNSUPPORTED, ENTMAX_ECUDA, ENTMAX_ENOCONVERGE, ENTMAX_ETIMEOUT = range(6)
+(ENTMAX_OK, ENTMAX_EINVAL, ENTMAX_EUNSUPPORTED, ENTMAX_ECUDA, ENTMAX_ENOCONVERGE, ENTMAX_ETIMEOUT,
+ ENTMAX_ERANGE) = range(7)
 STATUS_NAMES = {0: "ENTMAX_OK", 1: "ENTMAX_EINVAL", 2: "ENTMAX_EUNSUPPORTED", 3: "ENTMAX_ECUDA",
-                4: "ENTMAX_ENOCONVERGE", 5: "ENTMAX_ETIMEOUT"}
+                4: "ENTMAX_ENOCONVERGE", 5: "ENTMAX_ETIMEOUT", 6: "ENTMAX_ERANGE"}
 ENTMAX_BF16, ENTMAX_FP32 = 0, 1
 ENTMAX_MAX_L = 16384
 ENTMAX_TILE = 128
@@ -143,7 +144,7 @@ def entmax_last_device_status(desc: AttnDesc, workspace, stream=None) -> tuple[i
     word = ctypes.c_int(0)
     code = load_library().entmax_last_device_status(ctypes.byref(desc), _ptr(workspace), ctypes.byref(word),
                                                      _stream(stream))
-    _check("entmax_last_device_status", code, ok=(ENTMAX_OK, ENTMAX_ENOCONVERGE, ENTMAX_ETIMEOUT))
+    _check("entmax_last_device_status", code, ok=(ENTMAX_OK, ENTMAX_ENOCONVERGE, ENTMAX_ETIMEOUT, ENTMAX_ERANGE))
     return code, word.value
 
 

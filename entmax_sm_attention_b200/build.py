@@ -12,7 +12,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libentmax_attn.so")
-SOURCES = ["abi.cu", "fwd.cu", "fwd_f32.cu", "bwd.cu", "rows.cu", "noalloc.cu"]
+SOURCES = ["abi.cu", "convert.cu", "fwd.cu", "fwd_f32.cu", "bwd.cu", "rows.cu", "noalloc.cu"]
 HEADERS = ["common.cuh", "sm100.cuh", "kernels.h"]
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

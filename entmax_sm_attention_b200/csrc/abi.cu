@@ -22,7 +22,7 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct Layout {
   int BH, Tr, Tc, Wc, Wr;
-  size_t off_status, off_M, off_MT, off_sumg, off_Ot, off_delta, off_stats, total;
+  size_t off_status, off_M, off_MT, off_sumg, off_Ot, off_delta, off_stats, off_v16, off_do16, total;
   size_t bytes_M, bytes_MT, bytes_stats;
 };
 
@@ -51,6 +51,10 @@ bool layout_of(const entmax_attn_desc* d, Layout* l) {
   l->off_stats = off;
   l->bytes_stats = (size_t)l->BH * l->Tr * 16;
   off += align256(l->bytes_stats);
+  l->off_v16 = off;
+  off += align256(rows * kD * 2);
+  l->off_do16 = off;
+  off += align256(rows * kD * 2);
   l->total = off;
   return true;
 }
@@ -83,15 +87,16 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// bf16 [BH][L][64] viewed as a 3-D tensor; box = one 128 x 64 tile, 128-byte swizzle.
+// [BH][L][64] 16-bit tensor viewed as 3-D; box = one 128 x 64 tile, 128-byte swizzle.
 // Rows past L read as zeros.
-bool make_map(CUtensorMap* m, const void* base, int L, int BH) {
+bool make_map(CUtensorMap* m, const void* base, int L, int BH, bool f16 = false) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)L, (cuuint64_t)BH};
   cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)L * kD * 2};
   cuuint32_t box[3] = {(cuuint32_t)kD, (cuuint32_t)kTile, 1}, es[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+  return fn(m, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base),
+            dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -146,7 +151,10 @@ extern "C" entmax_status entmax_attn_fwd(const entmax_attn_desc* d, const void* 
   }
   FwdParams p;
   std::memset(&p, 0, sizeof(p));
-  if (!make_map(&p.tQ, Q, d->L, l.BH) || !make_map(&p.tK, K, d->L, l.BH) || !make_map(&p.tV, V, d->L, l.BH))
+  void* v16 = w + l.off_v16;
+  if (!make_map(&p.tQ, Q, d->L, l.BH) || !make_map(&p.tK, K, d->L, l.BH) || !make_map(&p.tV, v16, d->L, l.BH, true))
+    return ENTMAX_ECUDA;
+  if (launch_bf16_to_f16(V, v16, (long)l.BH * d->L * kD, reinterpret_cast<int*>(w + l.off_status), s) != cudaSuccess)
     return ENTMAX_ECUDA;
   p.O = O;
   p.tau = tau;
@@ -186,8 +194,10 @@ extern "C" entmax_status entmax_attn_bwd(const entmax_attn_desc* d, const void* 
   uint8_t* w = static_cast<uint8_t*>(ws);
   BwdParams p;
   std::memset(&p, 0, sizeof(p));
-  if (!make_map(&p.tQ, Q, d->L, l.BH) || !make_map(&p.tK, K, d->L, l.BH) || !make_map(&p.tV, V, d->L, l.BH) ||
-      !make_map(&p.tdO, dO, d->L, l.BH))
+  // V's fp16 copy was made by the forward (same workspace); dO gets one here.
+  void* do16 = w + l.off_do16;
+  if (!make_map(&p.tQ, Q, d->L, l.BH) || !make_map(&p.tK, K, d->L, l.BH) ||
+      !make_map(&p.tV, w + l.off_v16, d->L, l.BH, true) || !make_map(&p.tdO, do16, d->L, l.BH, true))
     return ENTMAX_ECUDA;
   float* delta = reinterpret_cast<float*>(w + l.off_delta);
   p.tau = tau;
@@ -210,6 +220,8 @@ extern "C" entmax_status entmax_attn_bwd(const entmax_attn_desc* d, const void* 
   p.window = d->window < 0 ? -1 : d->window;
   const long rows = (long)l.BH * d->L;
   if (cudaMemsetAsync(dQ, 0, (size_t)rows * kD * 4, s) != cudaSuccess) return ENTMAX_ECUDA;
+  if (launch_bf16_to_f16(dO, do16, rows * kD, reinterpret_cast<int*>(w + l.off_status), s) != cudaSuccess)
+    return ENTMAX_ECUDA;
   if (launch_delta(static_cast<const uint16_t*>(dO), reinterpret_cast<const float*>(w + l.off_Ot),
                    reinterpret_cast<const float*>(w + l.off_sumg), delta, rows, s) != cudaSuccess)
     return ENTMAX_ECUDA;
@@ -235,6 +247,7 @@ extern "C" entmax_status entmax_last_device_status(const entmax_attn_desc* d, co
   if (cudaMemcpy(&word, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return ENTMAX_ECUDA;
   *status_out = word;
   if (word & kStatusTimeout) return ENTMAX_ETIMEOUT;
+  if (word & kStatusRange) return ENTMAX_ERANGE;
   if (word & kStatusNoConverge) return ENTMAX_ENOCONVERGE;
   return ENTMAX_OK;
 }

@@ -15,11 +15,13 @@
 // Warps 0-7 are row owners: warp w reads TMEM lanes 32(w%4)..+31 (one query row per
 // lane) and the columns of keys [64(w/4), 64(w/4)+64). Once a warp holds its S and dA
 // values in registers it releases them, so the MMA warp computes S and dA of the next
-// query tile while the row owners form A and dS. A and dS are written as two-term bf16
-// splits (hi + lo, about fp32 accuracy in the products) into swizzled shared-memory
-// buffers. Those buffers then feed dV += A^T dO_i and dK += dS^T Q_i as MN-major
-// operands (M = keys, accumulated in TMEM), and dQ_i = dS K_j as a K-major operand
-// (double-buffered in TMEM). The row owners add dQ_i to global memory with vector
+// query tile while the row owners form A and dS. Both go to swizzled shared-memory
+// buffers: A in fp16 (with the fp16 copy of dO; 2^-11 rounding), dS as a two-term
+// bf16 split (hi + lo, about fp32 accuracy in its products). A single 16-bit dS costs
+// too much in dK at large query variance. Those buffers then feed dV += A^T dO_i and
+// dK += dS^T Q_i as MN-major operands (M = keys, accumulated in TMEM), and
+// dQ_i = dS K_j as a K-major operand (double-buffered in TMEM). dA = dO_i V_j^T uses the
+// fp16 copies of dO and V (exact conversions of the bf16 inputs). The row owners add dQ_i to global memory with vector
 // reductions. Warp 8 issues the TMA loads, warp 9 the MMAs.
 // TMEM: [0,128) S, [128,256) dA, [256,320) dV, [320,384) dK, [384,512) dQ x2.
 #include "common.cuh"
@@ -54,7 +56,7 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
 
 }  // namespace
 
-int bwd_smem_bytes() { return 1024 + 2 * kTileBytes + kStages * kPairBytes + 8 * kTileBytes; }
+int bwd_smem_bytes() { return 1024 + 2 * kTileBytes + kStages * kPairBytes + 6 * kTileBytes; }
 
 template <int AK>
 __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant__ BwdParams p) {
@@ -64,10 +66,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
   uint8_t* sK = dsm;
   uint8_t* sV = dsm + kTileBytes;
   uint8_t* ring = dsm + 2 * kTileBytes;                       // stage s: Q at +0, dO at +16 KB
-  // [128 q][128 k] bf16 matrices, each as 2 swizzled panels of 64 keys: A hi, A lo, dS hi, dS lo
+  // [128 q][128 k] 16-bit matrices, each as 2 swizzled panels of 64 keys: A (fp16),
+  // dS hi, dS lo (bf16)
   uint8_t* sA = ring + kStages * kPairBytes;
-  uint8_t* sAl = sA + 2 * kTileBytes;
-  uint8_t* sdS = sAl + 2 * kTileBytes;
+  uint8_t* sdS = sA + 2 * kTileBytes;
   uint8_t* sdSl = sdS + 2 * kTileBytes;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -132,11 +134,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------- MMA issuer
     if (lane == 0 && nq > 0) {
-      const uint32_t id128 = idesc_bf16(128, 128, 0, 0);
-      const uint32_t idMN = idesc_bf16(128, 64, 1, 1);   // A MN-major (from sA/sdS), B MN-major
-      const uint32_t idQ = idesc_bf16(128, 64, 0, 1);    // A K-major (sdS), B MN-major (K_j)
+      const uint32_t idS = idesc_bf16(128, 128, 0, 0);    // S = Q K^T
+      const uint32_t idA = idesc_f16(128, 128, 0, 0);     // dA = dO V^T (fp16 copies)
+      const uint32_t idV = idesc_f16(128, 64, 1, 1);      // dV += A^T dO: A MN-major (sA), B MN-major
+      const uint32_t idK = idesc_bf16(128, 64, 1, 1);     // dK += dS^T Q: A MN-major (sdS), B MN-major
+      const uint32_t idQ = idesc_bf16(128, 64, 0, 1);     // dQ = dS K: A K-major (sdS), B MN-major (K_j)
       const uint32_t kA = smem_u32(sK), vA = smem_u32(sV);
-      const uint32_t aH = smem_u32(sA), aL = smem_u32(sAl), dH = smem_u32(sdS), dL = smem_u32(sdSl);
+      const uint32_t aH = smem_u32(sA), dH = smem_u32(sdS), dL = smem_u32(sdSl);
       mbar_wait(&sh.bar_kv, 0, status, abrt);
       // S = Q_s K^T and dA = dO_s V^T into TMEM [0,256).
       auto issue_sda = [&](int s) {
@@ -147,8 +151,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          mma_ss(T, sdesc_sw128(qA + k * 32, 16, 1024), sdesc_sw128(kA + k * 32, 16, 1024), id128, k > 0);
-          mma_ss(T + 128, sdesc_sw128(oA + k * 32, 16, 1024), sdesc_sw128(vA + k * 32, 16, 1024), id128, k > 0);
+          mma_ss(T, sdesc_sw128(qA + k * 32, 16, 1024), sdesc_sw128(kA + k * 32, 16, 1024), idS, k > 0);
+          mma_ss(T + 128, sdesc_sw128(oA + k * 32, 16, 1024), sdesc_sw128(vA + k * 32, 16, 1024), idA, k > 0);
         }
         mma_commit(&sh.s_full);
       };
@@ -165,10 +169,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
           // dV += A^T dO_s and dK += dS^T Q_s: K = queries (16 per step), M = keys.
           const uint32_t acc = (s > 0 || t > 0) ? 1u : 0u;
           const uint64_t bO = sdesc_sw128(oA + t * 2048, 8192, 1024), bQ = sdesc_sw128(qA + t * 2048, 8192, 1024);
-          mma_ss(T + 256, sdesc_sw128(aH + t * 2048, 16384, 1024), bO, idMN, acc);
-          mma_ss(T + 256, sdesc_sw128(aL + t * 2048, 16384, 1024), bO, idMN, 1u);
-          mma_ss(T + 320, sdesc_sw128(dH + t * 2048, 16384, 1024), bQ, idMN, acc);
-          mma_ss(T + 320, sdesc_sw128(dL + t * 2048, 16384, 1024), bQ, idMN, 1u);
+          mma_ss(T + 256, sdesc_sw128(aH + t * 2048, 16384, 1024), bO, idV, acc);
+          mma_ss(T + 320, sdesc_sw128(dH + t * 2048, 16384, 1024), bQ, idK, acc);
+          mma_ss(T + 320, sdesc_sw128(dL + t * 2048, 16384, 1024), bQ, idK, 1u);
           // dQ_s = dS K_j: K = keys (16 per step; panel t/4), M = queries.
           const uint32_t koff = (t >> 2) * kTileBytes + (t & 3) * 32;
           const uint64_t bK = sdesc_sw128(kA + t * 2048, 8192, 1024);
@@ -227,7 +230,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       const int pan = hf * kTileBytes;
 #pragma unroll
       for (int ch = 0; ch < 8; ++ch) {
-        uint32_t ah[4], al[4], dh[4], dl2[4];
+        uint32_t ah[4], dh[4], dl2[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int c = ch * 8 + 2 * e;
@@ -243,16 +246,15 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
           if (AK == kAlpha15) {
             const float2 a = __fmul2_rn(make_float2(v0, v1), make_float2(v0, v1));
             const float2 ds = __fmul2_rn(make_float2(v0, v1), make_float2(d0, d1));
-            split_bf16x2(a.x, a.y, ah[e], al[e]);
+            ah[e] = pack_f16(a.x, a.y);
             split_bf16x2(ds.x, ds.y, dh[e], dl2[e]);
           } else {
-            split_bf16x2(v0, v1, ah[e], al[e]);
+            ah[e] = pack_f16(v0, v1);
             split_bf16x2(u.x > 0.f ? d0 : 0.f, u.y > 0.f ? d1 : 0.f, dh[e], dl2[e]);
           }
         }
         const uint32_t off = pan + sw128_offset(row, ch * 8);
         *reinterpret_cast<uint4*>(sA + off) = make_uint4(ah[0], ah[1], ah[2], ah[3]);
-        *reinterpret_cast<uint4*>(sAl + off) = make_uint4(al[0], al[1], al[2], al[3]);
         *reinterpret_cast<uint4*>(sdS + off) = make_uint4(dh[0], dh[1], dh[2], dh[3]);
         *reinterpret_cast<uint4*>(sdSl + off) = make_uint4(dl2[0], dl2[1], dl2[2], dl2[3]);
       }

@@ -20,12 +20,12 @@
 //     final tau. Packed 32 key tiles per uint32 (Appendix C.4), plus the transpose for
 //     the backward.
 //   Phase 4 (output): only the flagged key tiles. Recompute S and form
-//     A = u^{1/(alpha-1)} and g = u^{(2-alpha)/(alpha-1)}. Each is written to TMEM as a
-//     two-term bf16 split (hi + lo); A goes over the S columns it replaces. Then the
-//     tensor cores compute O += A V and Ot += g V, reading the A operand from TMEM. The
-//     split keeps the products at about fp32 accuracy: a single bf16 term (2^-8 relative)
-//     would cost more than the gradient tolerance once it reaches dK through delta.
-//     sum_j g_ij is kept per row for the backward.
+//     A = u^{1/(alpha-1)} and g = u^{(2-alpha)/(alpha-1)}. Both go to TMEM in fp16,
+//     over the S columns they replace. Then the tensor cores compute O += A V and
+//     Ot += g V, reading the A operand from TMEM, with B an fp16 copy of V. fp16 rounds
+//     at 2^-11; a bf16 A or g (2^-8) would cost more than the output and gradient
+//     tolerances once g reaches dK through delta. sum_j g_ij is kept per row for the
+//     backward.
 //
 // Roles (320 threads): warps 0-7 are row owners. Warp w reads TMEM lanes 32(w%4)..+31
 // (one query row per lane) and columns [64(w/4), 64(w/4)+64) of every S tile, so two
@@ -33,9 +33,8 @@
 // loads into a 4-slot ring of 16 KB K/V tiles. Warp 9 owns TMEM and issues the MMAs.
 // TMEM (512 columns): during the sweeps, four S buffers at 0/128/256/384, so the MMA
 // warp runs up to three tiles ahead. During the output pass:
-//   - two S buffers at 0 and 384; A hi/lo overwrite each buffer per 32-key quarter q
-//     (hi at 32q, lo at 32q+16);
-//   - g hi/lo at 128 + (same layout);
+//   - two S buffers at 0 and 384. The thread owning key half h overwrites its 64 S
+//     columns [64h, 64h+64) with A (fp16 pairs) at 64h and g at 64h + 32;
 //   - O at [256,320) and Ot at [320,384).
 #include "common.cuh"
 #include "kernels.h"
@@ -257,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     uint32_t sfree_par = 0;      // per sweep S buffer: parity of its uses so far (bit b)
     uint32_t sbuf = 0;           // next sweep S buffer
     const uint32_t idS = idesc_bf16(128, 128, 0, 0);
-    const uint32_t idO = idesc_bf16(128, 64, 0, 1);
+    const uint32_t idO = idesc_f16(128, 64, 0, 1);   // A (TMEM) and V copy, both fp16
     const uint32_t sQa = smem_u32(sQ);
     // S = Q K^T from ring position `pos` into TMEM columns [dcol, dcol+128).
     auto mma_s = [&](uint32_t pos, uint32_t dcol) {
@@ -320,13 +319,12 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
             const uint32_t vb = smem_u32(ring + vslot * kTileBytes);
 #pragma unroll
             for (int t = 0; t < 8; ++t) {
-              const uint32_t col = (t >> 1) * 32 + (t & 1) * 8;   // key quarter t/2, half t%2
+              // keys 16t..16t+15: half t/4, pair columns 8(t%4) within the half's A / g blocks
+              const uint32_t col = pa + (t >> 2) * 64 + (t & 3) * 8;
               const uint64_t bd = sdesc_sw128(vb + t * 2048, 8192, 1024);
               const uint32_t acc = (k > 0 || t > 0) ? 1u : 0u;
-              mma_ts(T + 256, T + pa + col, bd, idO, acc);
-              mma_ts(T + 256, T + pa + col + 16, bd, idO, 1u);
-              mma_ts(T + 320, T + 128 + col, bd, idO, acc);
-              if (AK == kAlpha15) mma_ts(T + 320, T + 128 + col + 16, bd, idO, 1u);
+              mma_ts(T + 256, T + col, bd, idO, acc);
+              mma_ts(T + 320, T + col + 32, bd, idO, acc);
             }
             mma_commit(&sh.empty[vslot]);
             mma_commit(&sh.pv_done[c]);
@@ -456,48 +454,29 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
             for (int cc = 0; cc < 64; ++cc)
               if (!pat.active(i, j0 + cc)) s[cc] = -INFINITY;
           }
+          uint32_t aw[32], gw[32];
 #pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            uint32_t ah[16], al[16];
-#pragma unroll
-            for (int cc = 0; cc < 16; ++cc) {
-              const float2 u = __ffma2_rn(make_float2(s[q * 32 + 2 * cc], s[q * 32 + 2 * cc + 1]),
-                                          make_float2(cz, cz), make_float2(-tau, -tau));
-              const float v0 = fmaxf(u.x, 0.f), v1 = fmaxf(u.y, 0.f);
-              if (AK == kAlpha15) {
-                const float2 a = __fmul2_rn(make_float2(v0, v1), make_float2(v0, v1));
-                split_bf16x2(a.x, a.y, ah[cc], al[cc]);
-              } else {
-                split_bf16x2(v0, v1, ah[cc], al[cc]);
-              }
+          for (int cc = 0; cc < 32; ++cc) {
+            const float2 u = __ffma2_rn(make_float2(s[2 * cc], s[2 * cc + 1]), make_float2(cz, cz),
+                                        make_float2(-tau, -tau));
+            const float v0 = fmaxf(u.x, 0.f), v1 = fmaxf(u.y, 0.f);
+            if (AK == kAlpha15) {
+              const float2 a = __fmul2_rn(make_float2(v0, v1), make_float2(v0, v1));
+              aw[cc] = pack_f16(a.x, a.y);
+              gw[cc] = pack_f16(v0, v1);
+              sg2 = __fadd2_rn(sg2, make_float2(v0, v1));
+            } else {
+              const float g0 = u.x > 0.f ? 1.f : 0.f, g1 = u.y > 0.f ? 1.f : 0.f;
+              aw[cc] = pack_f16(v0, v1);
+              gw[cc] = pack_f16(g0, g1);
+              sg2 = __fadd2_rn(sg2, make_float2(g0, g1));
             }
-            const uint32_t col = hf * 64 + q * 32;   // key quarter 2hf + q
-            tmem_st16(tl + pa + col, ah);
-            tmem_st16(tl + pa + col + 16, al);
           }
-          // g shares one TMEM region across tiles: PV of tile k-1 must have read it.
-          if (k >= 1) warp_wait(&sh.pv_done[(k - 1) & 1], ((k - 1) >> 1) & 1, status, abrt);
-#pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            uint32_t gh[16], gl[16];
-#pragma unroll
-            for (int cc = 0; cc < 16; ++cc) {
-              const float2 u = __ffma2_rn(make_float2(s[q * 32 + 2 * cc], s[q * 32 + 2 * cc + 1]),
-                                          make_float2(cz, cz), make_float2(-tau, -tau));
-              const float v0 = fmaxf(u.x, 0.f), v1 = fmaxf(u.y, 0.f);
-              if (AK == kAlpha15) {
-                split_bf16x2(v0, v1, gh[cc], gl[cc]);
-                sg2 = __fadd2_rn(sg2, make_float2(v0, v1));
-              } else {
-                const float g0 = u.x > 0.f ? 1.f : 0.f, g1 = u.y > 0.f ? 1.f : 0.f;
-                gh[cc] = pack_bf16(g0, g1);   // 0 and 1 are exact in bf16
-                sg2 = __fadd2_rn(sg2, make_float2(g0, g1));
-              }
-            }
-            const uint32_t col = hf * 64 + q * 32;
-            tmem_st16(tl + 128 + col, gh);
-            if (AK == kAlpha15) tmem_st16(tl + 128 + col + 16, gl);
-          }
+          const uint32_t col = pa + hf * 64;
+          tmem_st16(tl + col, *reinterpret_cast<uint32_t(*)[16]>(&aw[0]));
+          tmem_st16(tl + col + 16, *reinterpret_cast<uint32_t(*)[16]>(&aw[16]));
+          tmem_st16(tl + col + 32, *reinterpret_cast<uint32_t(*)[16]>(&gw[0]));
+          tmem_st16(tl + col + 48, *reinterpret_cast<uint32_t(*)[16]>(&gw[16]));
           tmem_wait_st();
           tc_fence_before();
           warp_arrive(&sh.o_ready[c]);

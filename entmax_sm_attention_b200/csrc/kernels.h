@@ -7,7 +7,7 @@
 namespace entmax {
 
 struct FwdParams {
-  CUtensorMap tQ, tK, tV;   // bf16 [B*H][L][64], box 64 x 128 x 1, 128-byte swizzle
+  CUtensorMap tQ, tK, tV;   // [B*H][L][64], box 64 x 128 x 1, 128-byte swizzle (Q, K bf16; V fp16)
   float* O;                 // [B*H][L][64]
   float* tau;               // [B*H][L]
   float* sumg;              // [B*H][L]      sum_j g_ij
@@ -23,7 +23,7 @@ struct FwdParams {
 };
 
 struct BwdParams {
-  CUtensorMap tQ, tK, tV, tdO;   // bf16 [B*H][L][64]
+  CUtensorMap tQ, tK, tV, tdO;   // [B*H][L][64]: Q, K bf16; V, dO fp16
   const float* tau;              // [B*H][L]
   const float* delta;            // [B*H][L]
   const uint32_t* MT;            // [B*H][Tc][Wr]
@@ -61,6 +61,7 @@ int bwd_smem_bytes();
 cudaError_t launch_fwd(bool alpha15, const FwdParams& p, int grid, cudaStream_t s);
 cudaError_t launch_fwd_f32(bool alpha15, const FwdF32Params& p, int grid, cudaStream_t s);
 cudaError_t launch_bwd(bool alpha15, const BwdParams& p, int grid, cudaStream_t s);
+cudaError_t launch_bf16_to_f16(const void* src, void* dst, long elems, int* status, cudaStream_t s);
 cudaError_t launch_delta(const uint16_t* dO, const float* Ot, const float* sumg, float* delta, long rows,
                          cudaStream_t s);
 cudaError_t launch_rows(bool alpha15, const float* S, int rows, int n, long ld, float* P, float* tau,

@@ -38,7 +38,9 @@
  *     ENTMAX_ECUDA. Conditions found on the device (solver cap reached, a bounded wait
  *     that expired) are recorded in the workspace status word and read back with
  *     entmax_last_device_status. Nothing throws across the ABI.
- *   - Non-finite inputs give undefined results.
+ *   - Non-finite inputs give undefined results. The probability-side products (O = A V,
+ *     Ot = g V, dV = A^T dO, dA = dO V^T) run in fp16, so bf16 V and dO must lie within
+ *     the fp16 range (|x| <= 65504); a value outside it sets ENTMAX_ERANGE.
  */
 #ifndef ENTMAX_ATTN_H
 #define ENTMAX_ATTN_H
@@ -56,7 +58,8 @@ typedef enum {
     ENTMAX_EUNSUPPORTED = 2,  /* valid request that this build does not implement         */
     ENTMAX_ECUDA = 3,         /* a CUDA call or kernel launch failed                      */
     ENTMAX_ENOCONVERGE = 4,   /* device: a row hit the refinement cap (tau kept bracketed) */
-    ENTMAX_ETIMEOUT = 5       /* device: a bounded wait inside a kernel expired            */
+    ENTMAX_ETIMEOUT = 5,      /* device: a bounded wait inside a kernel expired            */
+    ENTMAX_ERANGE = 6         /* device: a bf16 V or dO value beyond fp16 range (|x|>65504) */
 } entmax_status;
 
 typedef enum { ENTMAX_BF16 = 0, ENTMAX_FP32 = 1 } entmax_dtype;
@@ -82,8 +85,8 @@ typedef struct {
 
 /* Bytes of device workspace needed by entmax_attn_fwd / entmax_attn_bwd for *desc.
  * The workspace holds the status word, the block mask M and its transpose M^T, the
- * per-row sum_j g_ij and Ot_i = sum_j g_ij V_j, delta_i, per-tile counters
- * and, for fp32 inputs, split copies of Q, K and V. Returns 0 for an invalid
+ * per-row sum_j g_ij and Ot_i = sum_j g_ij V_j, delta_i, per-tile counters and fp16
+ * copies of V and dO. Returns 0 for an invalid
  * descriptor. The base address must be 256-byte aligned; the fwd -> bwd pair must use
  * the same workspace, and the caller keeps it alive in between. */
 size_t entmax_attn_workspace_bytes(const entmax_attn_desc *desc);
@@ -115,8 +118,9 @@ entmax_status entmax_rows(const float *S, int rows, int n, int ld, float alpha, 
                           float *tau, void *stream);
 
 /* Synchronises `stream`, then reads the workspace status word left by the last
- * fwd/bwd: ENTMAX_OK, ENTMAX_ENOCONVERGE or ENTMAX_ETIMEOUT. *status_out receives the
- * raw word: bit 0 = no convergence, bit 1 = wait timeout. */
+ * fwd/bwd: ENTMAX_OK, ENTMAX_ENOCONVERGE, ENTMAX_ETIMEOUT or ENTMAX_ERANGE. *status_out receives the
+ * raw word: bit 0 = no convergence, bit 1 = wait timeout, bit 2 = a V or dO value outside
+ * the fp16 range (ENTMAX_ERANGE; the results of that call are then undefined). */
 entmax_status entmax_last_device_status(const entmax_attn_desc *desc, const void *workspace,
                                         int *status_out, void *stream);
 
@@ -141,7 +145,7 @@ entmax_status entmax_attn_block_mask(const entmax_attn_desc *desc, const void *w
  * that the library keeps on every GPU that loads it, until the process exits.
  * The paper has no counterpart to this entry point; it exists for deployment only.
  *   - Limit: entmax_attn_workspace_bytes(desc) must not exceed
- *     ENTMAX_NOALLOC_SCRATCH_BYTES (16 MiB, roughly B*H*L <= 63000 rows). A larger
+ *     ENTMAX_NOALLOC_SCRATCH_BYTES (16 MiB, roughly B*H*L <= 32000 rows). A larger
  *     problem returns ENTMAX_EUNSUPPORTED before anything is launched.
  *   - Allocates nothing: no cudaMalloc, no cudaFree, no allocating library routine.
  *   - The first call on a device looks up the device address of the scratch array

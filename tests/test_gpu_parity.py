@@ -111,3 +111,21 @@ def test_fp32_backward_is_rejected():
     with pytest.raises(eb.EntmaxError) as e:
         eb.backward(ctx, d["Q"], d["K"], d["V"], d["dO"], tau)
     assert e.value.code == eb.ENTMAX_EUNSUPPORTED
+
+
+def test_out_of_fp16_range_is_reported():
+    """V and dO feed fp16 products; a bf16 value beyond fp16's range is flagged."""
+    from entmax_sm_attention_b200.workloads import make_inputs
+
+    w = small_case("range", L=256)
+    d = {k: v.cuda() for k, v in make_inputs(w).items()}
+    d["V"][0, 1, 7, 3] = 1.0e5
+    O, tau, ctx = eb.forward(d["Q"], d["K"], d["V"], alpha=1.5, scale=w.scale)
+    code, word = eb.entmax_last_device_status(*ctx)
+    assert code == eb.ENTMAX_ERANGE and word & 4
+    d["V"][0, 1, 7, 3] = 0.5
+    O, tau, ctx = eb.forward(d["Q"], d["K"], d["V"], alpha=1.5, scale=w.scale)
+    assert eb.entmax_last_device_status(*ctx)[0] == eb.ENTMAX_OK
+    d["dO"][0, 0, 3, 1] = -7.0e4
+    eb.backward(ctx, d["Q"], d["K"], d["V"], d["dO"], tau)
+    assert eb.entmax_last_device_status(*ctx)[0] == eb.ENTMAX_ERANGE
