@@ -101,6 +101,19 @@ bool make_map(CUtensorMap* m, const void* base, int L, int BH, bool f16 = false)
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// fp32 [BH][L][64] as 3-D with a 32 x 128 box (128-byte rows, 128-byte swizzle): the
+// target of the backward's dQ reduce-adds.
+bool make_map_f32_half(CUtensorMap* m, void* base, int L, int BH) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)L, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)kD * 4, (cuuint64_t)L * kD * 4};
+  cuuint32_t box[3] = {32, (cuuint32_t)kTile, 1}, es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 extern "C" size_t entmax_attn_workspace_bytes(const entmax_attn_desc* d) {
@@ -197,7 +210,8 @@ extern "C" entmax_status entmax_attn_bwd(const entmax_attn_desc* d, const void* 
   // V's fp16 copy was made by the forward (same workspace); dO gets one here.
   void* do16 = w + l.off_do16;
   if (!make_map(&p.tQ, Q, d->L, l.BH) || !make_map(&p.tK, K, d->L, l.BH) ||
-      !make_map(&p.tV, w + l.off_v16, d->L, l.BH, true) || !make_map(&p.tdO, do16, d->L, l.BH, true))
+      !make_map(&p.tV, w + l.off_v16, d->L, l.BH, true) || !make_map(&p.tdO, do16, d->L, l.BH, true) ||
+      !make_map_f32_half(&p.tdQ, dQ, d->L, l.BH))
     return ENTMAX_ECUDA;
   float* delta = reinterpret_cast<float*>(w + l.off_delta);
   p.tau = tau;

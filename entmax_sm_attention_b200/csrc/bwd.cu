@@ -49,14 +49,10 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
-               : "memory");
-}
 
 }  // namespace
 
-int bwd_smem_bytes() { return 1024 + 2 * kTileBytes + kStages * kPairBytes + 6 * kTileBytes; }
+int bwd_smem_bytes() { return 1024 + 2 * kTileBytes + kStages * kPairBytes + 6 * kTileBytes + 2 * kTileBytes; }
 
 template <int AK>
 __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant__ BwdParams p) {
@@ -71,10 +67,12 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
   uint8_t* sA = ring + kStages * kPairBytes;
   uint8_t* sdS = sA + 2 * kTileBytes;
   uint8_t* sdSl = sdS + 2 * kTileBytes;
+  uint8_t* sStage = sdSl + 2 * kTileBytes;   // dQ tile: two [128][32] fp32 boxes, 128-byte swizzle
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bh = blockIdx.x % p.BH;
   const int kt = blockIdx.x / p.BH;          // key tile (low key tiles have the most query tiles)
+  const int kMathThreads = 256;
   const int b = bh / p.H;
   const Pattern pat{p.L, p.kv_len ? min(max(p.kv_len[b], 1), p.L) : p.L, p.causal, p.window};
   const int j0 = kt * kTile;
@@ -190,23 +188,33 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     const uint32_t tl = T + ((uint32_t)(quad * 32) << 16);
     const float cz = p.cz;
     uint32_t seq = 0;
-    int prev_i = -1;
-    // Adds this thread's 32 columns of dQ for the query tile of step `s` (TMEM buffer
-    // s % 2) to global memory. The caller has already waited for that step's MMAs.
-    auto flush_dq = [&](uint32_t s, int irow) {
+    int prev_it = -1;
+    // Adds dQ of the query tile `it` handled at step `s` (TMEM buffer s % 2) to global
+    // memory. The caller has already waited for that step's MMAs. Each thread stages its
+    // 32 columns (scaled) in the swizzled box of its column half; then thread 0 issues
+    // one TMA reduce-add per box. The staging buffer is reused only after the previous
+    // reduce-adds have read it.
+    auto flush_dq = [&](uint32_t s, int it) {
+      if (tid == 0) bulk_wait_read_all();
+      named_bar(1, kMathThreads);
       tc_fence_after();
       uint32_t a[32];
       tmem_ld32(tl + 384 + (s & 1) * 64 + hf * 32, a);
       tmem_wait_ld();
-      if (irow < p.L) {
-        float* dst = p.dQ + ((size_t)bh * p.L + irow) * kD + hf * 32;
-        const float sc = p.scale;
+      uint8_t* box = sStage + hf * kTileBytes + row * 128;
+      const float sc = p.scale;
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-          red_add_v4(dst + 4 * k, sc * __uint_as_float(a[4 * k]), sc * __uint_as_float(a[4 * k + 1]),
-                     sc * __uint_as_float(a[4 * k + 2]), sc * __uint_as_float(a[4 * k + 3]));
+      for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<float4*>(box + ((c ^ (row & 7)) << 4)) =
+            make_float4(sc * __uint_as_float(a[4 * c]), sc * __uint_as_float(a[4 * c + 1]),
+                        sc * __uint_as_float(a[4 * c + 2]), sc * __uint_as_float(a[4 * c + 3]));
+      fence_proxy_async_smem();
+      named_bar(1, kMathThreads);
+      if (tid == 0) {
+        tma_reduce_add_3d(&p.tdQ, sStage, 0, it * kTile, bh);
+        tma_reduce_add_3d(&p.tdQ, sStage + kTileBytes, 32, it * kTile, bh);
+        bulk_commit();
       }
-      __syncwarp();
     };
     for_each_bit(qlist, kMaskWords, [&](int it) {
       const int i = it * kTile + row;
@@ -260,14 +268,15 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       }
       fence_proxy_async_smem();
       warp_arrive(&sh.p_ready);
-      if (seq > 0) flush_dq(seq - 1, prev_i);   // its MMAs were waited for above
-      prev_i = i;
+      if (seq > 0) flush_dq(seq - 1, prev_it);   // its MMAs were waited for above
+      prev_it = it;
       ++seq;
     });
     if (seq > 0) {
       warp_wait(&sh.mma2_done, (seq - 1) & 1, status, abrt);
-      flush_dq(seq - 1, prev_i);
+      flush_dq(seq - 1, prev_it);
     }
+    if (tid == 0) bulk_wait_all();   // the last reduce-adds complete before the CTA retires
     // dK and dV of this key tile (TMEM lane = key); each thread writes 32 of the 64
     // columns. Every lane executes the TMEM loads (.sync.aligned); only the global stores
     // depend on the key being inside L.

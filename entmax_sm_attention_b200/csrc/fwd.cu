@@ -553,18 +553,29 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           cnt[a] = 0;
         }
         if (collect) {
+          // Groups of 8 scores: u+ summed per group (feeds S1); only a group with a
+          // positive sum (rare: a support candidate) is scanned element by element.
 #pragma unroll
-          for (int cc = 0; cc < 64; cc += 2) {
-            const float2 u = __ffma2_rn(make_float2(s[cc], s[cc + 1]), make_float2(cz, cz), make_float2(-tau, -tau));
-            const float2 v = make_float2(fmaxf(u.x, 0.f), fmaxf(u.y, 0.f));
-            const int a = (cc >> 1) & 3;
-            s1[a] = __fadd2_rn(s1[a], v);
-            s2[a] = __ffma2_rn(v, v, s2[a]);
-            // Candidates: predicated stores, no branches (the store slot is clamped).
-            if (u.x > 0.f) mycand[min(nc, kCandPerThread - 1) * kTile] = s[cc];
-            nc += u.x > 0.f;
-            if (u.y > 0.f) mycand[min(nc, kCandPerThread - 1) * kTile] = s[cc + 1];
-            nc += u.y > 0.f;
+          for (int g = 0; g < 8; ++g) {
+            float2 v[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 u = __ffma2_rn(make_float2(s[8 * g + 2 * e], s[8 * g + 2 * e + 1]), make_float2(cz, cz),
+                                          make_float2(-tau, -tau));
+              v[e] = make_float2(fmaxf(u.x, 0.f), fmaxf(u.y, 0.f));
+              s2[e] = __ffma2_rn(v[e], v[e], s2[e]);
+            }
+            const float2 gs = __fadd2_rn(__fadd2_rn(v[0], v[1]), __fadd2_rn(v[2], v[3]));
+            s1[g & 3] = __fadd2_rn(s1[g & 3], gs);
+            if (gs.x + gs.y > 0.f) {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                if (fmaf(s[8 * g + e], cz, -tau) > 0.f) {
+                  if (nc < kCandPerThread) mycand[nc * kTile] = s[8 * g + e];
+                  ++nc;
+                }
+              }
+            }
           }
         } else {
 #pragma unroll

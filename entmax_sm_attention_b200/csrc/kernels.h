@@ -24,6 +24,7 @@ struct FwdParams {
 
 struct BwdParams {
   CUtensorMap tQ, tK, tV, tdO;   // [B*H][L][64]: Q, K bf16; V, dO fp16
+  CUtensorMap tdQ;               // fp32 [B*H][L][64], box 32 x 128 x 1, 128-byte swizzle (reduce-add)
   const float* tau;              // [B*H][L]
   const float* delta;            // [B*H][L]
   const uint32_t* MT;            // [B*H][Tc][Wr]
