@@ -30,11 +30,14 @@
 // Roles (320 threads): warps 0-7 are row owners. Warp w reads TMEM lanes 32(w%4)..+31
 // (one query row per lane) and columns [64(w/4), 64(w/4)+64) of every S tile, so two
 // threads share a row and combine partial sums in shared memory. Warp 8 issues TMA
-// loads into a 4-slot ring of 16 KB K/V tiles. Warp 9 owns TMEM and issues the MMAs.
+// loads into a 4-slot ring of 16 KB K/V tiles. Warp 9 owns TMEM and issues the MMAs;
+// in the output pass warp 10 issues the Ot = g V chain, because one thread cannot
+// issue N=64 MMAs as fast as the tensor cores retire them.
 // TMEM (512 columns): during the sweeps, four S buffers at 0/128/256/384, so the MMA
 // warp runs up to three tiles ahead. During the output pass:
-//   - two S buffers at 0 and 384. The thread owning key half h overwrites its 64 S
-//     columns [64h, 64h+64) with A (fp16 pairs) at 64h and g at 64h + 32;
+//   - three S buffers at 0, 128 and 384 (tile k in buffer k % 3). The thread owning key
+//     half h overwrites its 64 S columns [64h, 64h+64) with A (fp16 pairs) at 64h and
+//     g at 64h + 32;
 //   - O at [256,320) and Ot at [320,384).
 #include "common.cuh"
 #include "kernels.h"
@@ -43,10 +46,12 @@ namespace entmax {
 
 namespace {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;
 constexpr int kMathThreads = 256;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
+constexpr int kMma2Warp = 10;   // second MMA issuer: the Ot = g V chain of the output pass
+constexpr int kOBufs = 3;       // S/A buffers in the output pass (TMEM columns 0, 128, 384)
 constexpr int kSlots = 4;
 constexpr int kSBufs = 4;
 constexpr int kCandPerThread = 32;     // candidates per (row, column half); 64 per row
@@ -60,7 +65,7 @@ struct Shared {
   uint64_t full[kSlots], empty[kSlots];
   uint64_t bar_q;
   uint64_t s_full[kSBufs], s_free[kSBufs];     // sweeps: MMA -> rows, rows -> MMA
-  uint64_t o_full[2], o_ready[2], pv_done[2];  // output pass ping-pong
+  uint64_t o_full[kOBufs], o_ready[kOBufs], pv_done[kOBufs];  // output pass, buffer c = k % 3
   uint32_t tmem_base;
   int abort_flag;
   int ctl_kind, ctl_buf;
@@ -166,17 +171,17 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
   if (tid == 0) {
     for (int s = 0; s < kSlots; ++s) {
       mbar_init(&sh.full[s], 1);
-      mbar_init(&sh.empty[s], 1);
+      mbar_init(&sh.empty[s], 2);   // two commits: one per MMA issuer reading the slot
     }
     mbar_init(&sh.bar_q, 1);
     for (int s = 0; s < kSBufs; ++s) {
       mbar_init(&sh.s_full[s], 1);
       mbar_init(&sh.s_free[s], 8);
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kOBufs; ++s) {
       mbar_init(&sh.o_full[s], 1);
       mbar_init(&sh.o_ready[s], 8);
-      mbar_init(&sh.pv_done[s], 1);
+      mbar_init(&sh.pv_done[s], 2);   // O chain and Ot chain
     }
     sh.abort_flag = 0;
     fence_mbar_init();
@@ -267,6 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
 #pragma unroll
       for (int k = 0; k < 4; ++k)
         mma_ss(T + dcol, sdesc_sw128(sQa + k * 32, 16, 1024), sdesc_sw128(kb + k * 32, 16, 1024), idS, k > 0);
+      mma_commit(&sh.empty[slot]);   // a K slot is read by this issuer only: both arrivals here
       mma_commit(&sh.empty[slot]);
     };
     auto sweep_tile = [&]() {
@@ -293,43 +299,79 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           sbuf = 0;
           for_each_bit(list, kMaskWords, [&](int) { sweep_tile(); });
         } else {
-          // Output pass. S of tile k+1 is issued before PV of tile k, so it overlaps the
-          // row owners' work on tile k. Buffer c = k % 2 sits at TMEM column 0 or 384.
-          // K_k is at ring position base + 2k, V_k at base + 2k + 1.
+          // Output pass. S of tile k+1 is issued before O += A V of tile k, so it overlaps
+          // the row owners' work on tile k. Tile k uses buffer c = k % 3 at TMEM column
+          // 0, 128 or 384. K_k is at ring position base + 2k, V_k at base + 2k + 1.
           int n = 0;
 #pragma unroll
           for (int w = 0; w < kMaskWords; ++w) n += __popc(list[w]);
           const uint32_t base = seq;
           auto issue_s = [&](int k) {
-            const int c = k & 1;
-            if (k >= 2) mbar_wait(&sh.pv_done[c], ((k - 2) >> 1) & 1, status, abrt);   // buffer c free
-            mma_s(base + 2 * k, c ? 384u : 0u);
+            const int c = k % kOBufs;
+            if (k >= kOBufs) mbar_wait(&sh.pv_done[c], ((k - kOBufs) / kOBufs) & 1, status, abrt);   // buffer free
+            mma_s(base + 2 * k, c == 0 ? 0u : (c == 1 ? 128u : 384u));
             mma_commit(&sh.o_full[c]);
           };
           if (n > 0) issue_s(0);
           for (int k = 0; k < n; ++k) {
             if (k + 1 < n) issue_s(k + 1);
-            const int c = k & 1;
-            const uint32_t pa = c ? 384u : 0u;
+            const int c = k % kOBufs;
+            const uint32_t pa = c == 0 ? 0u : (c == 1 ? 128u : 384u);
             const uint32_t vpos = base + 2 * k + 1;
             const int vslot = vpos % kSlots;
             mbar_wait(&sh.full[vslot], (vpos / kSlots) & 1, status, abrt);
-            mbar_wait(&sh.o_ready[c], (k >> 1) & 1, status, abrt);   // A and g of tile k written
+            mbar_wait(&sh.o_ready[c], (k / kOBufs) & 1, status, abrt);   // A and g of tile k written
             tc_fence_after();
             const uint32_t vb = smem_u32(ring + vslot * kTileBytes);
 #pragma unroll
             for (int t = 0; t < 8; ++t) {
-              // keys 16t..16t+15: half t/4, pair columns 8(t%4) within the half's A / g blocks
+              // keys 16t..16t+15: half t/4, pair columns 8(t%4) within the half's A block
               const uint32_t col = pa + (t >> 2) * 64 + (t & 3) * 8;
-              const uint64_t bd = sdesc_sw128(vb + t * 2048, 8192, 1024);
-              const uint32_t acc = (k > 0 || t > 0) ? 1u : 0u;
-              mma_ts(T + 256, T + col, bd, idO, acc);
-              mma_ts(T + 320, T + col + 32, bd, idO, acc);
+              mma_ts(T + 256, T + col, sdesc_sw128(vb + t * 2048, 8192, 1024), idO, (k > 0 || t > 0) ? 1u : 0u);
             }
             mma_commit(&sh.empty[vslot]);
             mma_commit(&sh.pv_done[c]);
           }
           seq = base + 2 * n;
+        }
+      }
+      __syncwarp();
+      if (kind != kKindSweep) break;
+    }
+  } else if (warp == kMma2Warp) {
+    // ------------------------------------------------ second MMA issuer (output pass)
+    const uint32_t idO = idesc_f16(128, 64, 0, 1);
+    uint32_t seq = 0;   // ring positions, tracked exactly like the producer's
+    for_each_bit(act, kMaskWords, [&](int) { ++seq; });
+    while (true) {
+      named_bar(1, kThreads);
+      const int kind = sh.ctl_kind;
+      uint32_t list[kMaskWords];
+#pragma unroll
+      for (int w = 0; w < kMaskWords; ++w) list[w] = sh.lists[sh.ctl_buf][w];
+      int n = 0;
+#pragma unroll
+      for (int w = 0; w < kMaskWords; ++w) n += __popc(list[w]);
+      if (kind == kKindSweep) {
+        seq += n;
+      } else if (lane == 0) {
+        const uint32_t base = seq;
+        for (int k = 0; k < n; ++k) {
+          const int c = k % kOBufs;
+          const uint32_t pa = c == 0 ? 0u : (c == 1 ? 128u : 384u);
+          const uint32_t vpos = base + 2 * k + 1;
+          const int vslot = vpos % kSlots;
+          mbar_wait(&sh.full[vslot], (vpos / kSlots) & 1, status, abrt);
+          mbar_wait(&sh.o_ready[c], (k / kOBufs) & 1, status, abrt);
+          tc_fence_after();
+          const uint32_t vb = smem_u32(ring + vslot * kTileBytes);
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            const uint32_t col = pa + (t >> 2) * 64 + (t & 3) * 8 + 32;   // g block of the half
+            mma_ts(T + 320, T + col, sdesc_sw128(vb + t * 2048, 8192, 1024), idO, (k > 0 || t > 0) ? 1u : 0u);
+          }
+          mma_commit(&sh.empty[vslot]);
+          mma_commit(&sh.pv_done[c]);
         }
       }
       __syncwarp();
@@ -439,12 +481,12 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
             atomicOr(&p.MT[((size_t)bh * p.Tc + jt) * p.Wr + (qt >> 5)], 1u << (qt & 31));
           });
         }
-        // Phase 4: output pass over the flagged tiles, ping-pong buffers c = k % 2.
+        // Phase 4: output pass over the flagged tiles, buffers c = k % 3.
         int k = 0;
         for_each_bit(list, kMaskWords, [&](int jt) {
-          const int c = k & 1;
-          const uint32_t pa = c ? 384u : 0u;
-          warp_wait(&sh.o_full[c], (k >> 1) & 1, status, abrt);
+          const int c = k % kOBufs;
+          const uint32_t pa = c == 0 ? 0u : (c == 1 ? 128u : 384u);
+          warp_wait(&sh.o_full[c], (k / kOBufs) & 1, status, abrt);
           tc_fence_after();
           const int j0 = jt * kTile + hf * 64;
           float s[64];
@@ -485,7 +527,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         });
         const int n_out = k;
         // Epilogue: O and Ot from TMEM (each thread of a row writes 32 of the 64 columns).
-        warp_wait(&sh.pv_done[(n_out - 1) & 1], ((n_out - 1) >> 1) & 1, status, abrt);
+        warp_wait(&sh.pv_done[(n_out - 1) % kOBufs], ((n_out - 1) / kOBufs) & 1, status, abrt);
         tc_fence_after();
         part[(hf * 4 + 1) * kTile + row] = sg2.x + sg2.y;
         uint32_t o[32];
