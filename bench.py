@@ -45,6 +45,7 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU-oracle sample time")
+    ap.add_argument("--no-sweeps", action="store_true", help="skip the block-sparsity sweeps")
     return ap.parse_args()
 
 
@@ -340,6 +341,8 @@ def run_ours(args):
             "memsets_per_step": 3,
         },
     }
+    if rank == 0 and world == 1 and not args.no_sweeps:
+        result["detail"]["sparsity_sweeps"] = sparsity_sweeps(w, alpha, dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, cores, sample = cpu_oracle_sample(w, alpha, args.seed, args.cpu_seconds)
         result["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
@@ -347,6 +350,61 @@ def run_ours(args):
         print(json.dumps(result), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+def sparsity_sweeps(w, alpha, dev, steps: int = 10):
+    """Wall time against measured block sparsity on the same shape as the timed workload.
+    (a) planted block structure with rho in {1, 1/2, 1/4, 1/8, 1/16} (block sparsity about
+    1 - rho); (b) iid Gaussian inputs with query scale sigma_Q in {1, 3, 8, 24} (AdaSplash-2
+    §4.2's knob). Each point: 2 warm-up and `steps` timed forward+backward steps, L2 flushed
+    before each step."""
+    import torch
+
+    from entmax_sm_attention_b200 import binding as eb
+    from entmax_sm_attention_b200.workloads import make_inputs, make_planted_inputs
+
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    desc = eb.make_desc(w.B, w.H, w.L, w.d, alpha=alpha, scale=w.scale, causal=w.causal, window=w.window)
+    ws = eb.alloc_workspace(desc, dev)
+    shp = (w.B, w.H, w.L, w.d)
+    O = torch.empty(shp, dtype=torch.float32, device=dev)
+    tau = torch.empty(shp[:3], dtype=torch.float32, device=dev)
+    dQ, dK, dV = (torch.empty(shp, dtype=torch.float32, device=dev) for _ in range(3))
+
+    def point(inp):
+        d = {k: v.to(dev) for k, v in inp.items()}
+        fwd, bwd = [], []
+        for k in range(2 + steps):
+            flush.zero_()
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            e[0].record(stream)
+            eb.entmax_attn_fwd(desc, d["Q"], d["K"], d["V"], O, tau, ws, stream)
+            e[1].record(stream)
+            eb.entmax_attn_bwd(desc, d["Q"], d["K"], d["V"], d["dO"], tau, ws, dQ, dK, dV, stream)
+            e[2].record(stream)
+            torch.cuda.synchronize(dev)
+            if k >= 2:
+                fwd.append(e[0].elapsed_time(e[1]))
+                bwd.append(e[1].elapsed_time(e[2]))
+        _, st = eb.block_mask((desc, ws))
+        st = st.cpu().long()
+        return {"block_sparsity_128": 1.0 - float(st[..., 2].sum()) / max(1, int(st[..., 3].sum())),
+                "fwd_ms": statistics.mean(fwd), "bwd_ms": statistics.mean(bwd),
+                "ms": statistics.mean(fwd) + statistics.mean(bwd)}
+
+    planted = []
+    for rho in (1.0, 0.5, 0.25, 0.125, 0.0625):
+        r = point(make_planted_inputs(w, rho, seed=7))
+        r["rho"] = rho
+        planted.append(r)
+    sigma = []
+    for sq in (1.0, 3.0, 8.0, 24.0):
+        r = point(make_inputs(w.with_(sigma_q=sq), seed=7))
+        r["sigma_q"] = sq
+        sigma.append(r)
+    return {"planted_rho": planted, "iid_sigma_q": sigma,
+            "note": "same shape as the timed workload; planted inputs are a builder-added family"}
 
 
 def act_pairs(w) -> int:

@@ -108,3 +108,40 @@ def small_case(name: str, *, B=1, H=2, L=300, d=64, dtype="bf16", causal=False, 
     """A reduced workload the oracle finishes in seconds: several tiles plus a ragged tail."""
     return Workload(name, B=B, H=H, L=L, d=d, dtype=dtype, causal=causal, window=window,
                     kv_len=kv_len, sigma_q=sigma_q, alphas=alphas)
+
+
+def make_planted_inputs(w: Workload, rho: float, seed: int = 0, gamma: float = 3.0) -> dict:
+    """Block-structured inputs whose support lies in a chosen fraction rho of the key tiles.
+
+    This family is not on the pages. It stands in for the trained models whose block
+    sparsity AdaSplash-2 §4.2 and Fig. 7 report, which iid Gaussian inputs do not reach at
+    128 x 128 tiles. Every key tile t of every (b, h) gets a centre c_t ~ N(0, I), and its
+    keys are K_j = c_t + 0.3 N(0, I). Each query tile picks max(1, round(rho * n)) of the
+    n key tiles it may attend to (causal: tiles 0..it). Each query row aims at one of the
+    picked tiles t*: Q_i = gamma * c_{t*} + 0.5 N(0, I). With gamma = 3 and d = 64 a key of
+    the chosen tile scores about gamma |c|^2 / sqrt(d) = 24 and any other key about
+    N(0, gamma^2) = N(0, 9), so the support, and with it the flagged blocks, stays in the
+    picked tiles (block sparsity about 1 - rho). V and dO ~ N(0, 1).
+    """
+    g = torch.Generator().manual_seed(seed)
+    B, H, L, d, T = w.B, w.H, w.L, w.d, 128
+    nT = -(-L // T)
+    centres = torch.randn((B, H, nT, d), generator=g)
+    tile_of = torch.arange(L) // T
+    K = centres[:, :, tile_of, :] + 0.3 * torch.randn((B, H, L, d), generator=g)
+    Q = 0.5 * torch.randn((B, H, L, d), generator=g)
+    for it in range(nT):
+        n_allowed = it + 1 if w.causal else nT
+        n_pick = max(1, int(round(rho * n_allowed)))
+        rows = slice(it * T, min(L, (it + 1) * T))
+        nrows = rows.stop - rows.start
+        for b in range(B):
+            for h in range(H):
+                picked = torch.randperm(n_allowed, generator=g)[:n_pick]
+                choice = picked[torch.randint(0, n_pick, (nrows,), generator=g)]
+                Q[b, h, rows] += gamma * centres[b, h, choice]
+    V = torch.randn((B, H, L, d), generator=g)
+    dO = torch.randn((B, H, L, d), generator=g)
+    dt = w.torch_dtype
+    return {"Q": Q.to(dt).contiguous(), "K": K.to(dt).contiguous(), "V": V.to(dt).contiguous(),
+            "dO": dO.to(dt).contiguous()}

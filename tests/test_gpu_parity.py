@@ -129,3 +129,26 @@ def test_out_of_fp16_range_is_reported():
     d["dO"][0, 0, 3, 1] = -7.0e4
     eb.backward(ctx, d["Q"], d["K"], d["V"], d["dO"], tau)
     assert eb.entmax_last_device_status(*ctx)[0] == eb.ENTMAX_ERANGE
+
+
+@pytest.mark.parametrize("alpha", [1.5, 2.0])
+def test_planted_block_structure(alpha):
+    """Block-structured inputs (support confined to a fraction rho of the key tiles):
+    parity with the oracle, an exact mask, real block sparsity, and a backward that
+    visits only the flagged tiles."""
+    from entmax_sm_attention_b200.workloads import make_planted_inputs
+    from parity import check_mask, gpu_run, oracle_problem
+
+    w = small_case("planted", B=1, H=2, L=1100, causal=True)
+    inp = make_planted_inputs(w, 0.25, seed=3)
+    g = gpu_run(inp, w, alpha, backward=True)
+    pr = oracle_problem(inp, w, alpha)
+    ref = pr.backward()
+    assert np.abs(g["tau"] - ref["tau"]).max() <= TOL_TAU
+    assert np.abs(g["O"] - ref["O"]).max() <= 1e-2
+    for k in ("dQ", "dK", "dV"):
+        assert np.abs(g[k] - ref[k]).max() <= 2e-2, k
+    assert check_mask(pr, ref["tau"], g["M"])[0] == 0
+    st = g["stats"].reshape(-1, 4)
+    sparsity = 1.0 - st[:, 2].sum() / st[:, 3].sum()
+    assert sparsity > 0.5, sparsity
