@@ -291,14 +291,14 @@ def run_ours(args):
     st = st.cpu().long()
     n_sweeps, n_s, n_out, n_act = (st[..., c] for c in range(4))
     s_tiles, out_tiles, act_tiles = int(n_s.sum()), int(n_out.sum()), int(n_act.sum())
-    # Algorithmic tensor work (SURVEY-style count, tile granularity): forward = every
-    # S tile computed (max pass + refinement passes + output pass) + O and Ot products
-    # on flagged tiles; backward = S, dA, dV, dK, dQ on every flagged tile pair.
+    # Algorithmic tensor work at tile granularity: forward = every S tile computed (max
+    # pass + refinement passes + output pass) + the A V and g V products on flagged
+    # tiles; backward = S, dA, dV, dK, dQ on every flagged tile pair.
     fwd_flops = UNIT_FLOP * (s_tiles + 2 * out_tiles)
     bwd_flops = UNIT_FLOP * 5 * out_tiles
-    # Issued tensor work, counting the two-term (hi + lo) splits.
-    fwd_issued = UNIT_FLOP * (s_tiles + (4 if alpha == 1.5 else 3) * out_tiles)
-    bwd_issued = UNIT_FLOP * 8 * out_tiles
+    # Issued tensor work: the backward feeds dS as two bf16 terms (hi + lo) to dK and dQ.
+    fwd_issued = UNIT_FLOP * (s_tiles + 2 * out_tiles)
+    bwd_issued = UNIT_FLOP * 7 * out_tiles
     fwd_avg, bwd_avg = statistics.mean(fwd_ms), statistics.mean(bwd_ms)
     peaks = load_peaks()
     peak = peaks["bf16_tflops_sustained"]
@@ -325,7 +325,8 @@ def run_ours(args):
                      "traffic": ncu_traffic(dom, w.name, alpha),
                      "traffic_unit": "bytes per launch (ncu dram read+write; null if the kernel changed)"},
         "clocks": clk,
-        "gpu_launches": 3 * args.steps,
+        # per step: V -> fp16 copy, forward, dO -> fp16 copy, delta, backward
+        "gpu_launches": 5 * args.steps,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "detail": {
             "fwd_ms": fwd_avg, "bwd_ms": bwd_avg,
@@ -390,6 +391,8 @@ def sparsity_sweeps(w, alpha, dev, steps: int = 10):
         _, st = eb.block_mask((desc, ws))
         st = st.cpu().long()
         return {"block_sparsity_128": 1.0 - float(st[..., 2].sum()) / max(1, int(st[..., 3].sum())),
+                "refine_sweeps_mean": float(st[..., 0].float().mean()),
+                "s_tiles_per_active": float(st[..., 1].sum()) / max(1, int(st[..., 3].sum())),
                 "fwd_ms": statistics.mean(fwd), "bwd_ms": statistics.mean(bwd),
                 "ms": statistics.mean(fwd) + statistics.mean(bwd)}
 

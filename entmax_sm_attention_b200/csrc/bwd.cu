@@ -21,8 +21,10 @@
 // too much in dK at large query variance. Those buffers then feed dV += A^T dO_i and
 // dK += dS^T Q_i as MN-major operands (M = keys, accumulated in TMEM), and
 // dQ_i = dS K_j as a K-major operand (double-buffered in TMEM). dA = dO_i V_j^T uses the
-// fp16 copies of dO and V (exact conversions of the bf16 inputs). The row owners add dQ_i to global memory with vector
-// reductions. Warp 8 issues the TMA loads, warp 9 the MMAs.
+// fp16 copies of dO and V (exact conversions of the bf16 inputs). The row owners copy
+// dQ_i from TMEM into a swizzled fp32 staging tile in shared memory, and one thread adds
+// it to global dQ with a TMA reduce-add (cp.reduce.async.bulk.tensor .add), one query
+// tile behind the MMAs. Warp 8 issues the TMA loads, warp 9 the MMAs.
 // TMEM: [0,128) S, [128,256) dA, [256,320) dV, [320,384) dK, [384,512) dQ x2.
 #include "common.cuh"
 #include "kernels.h"

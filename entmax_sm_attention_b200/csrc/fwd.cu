@@ -9,13 +9,16 @@
 //     subset of the scores has a smaller threshold than on all of them (fewer
 //     nonnegative terms in Eq. 4), so this is a lower bound tau_T <= tau*. It plays the
 //     role the paper gives its on-chip histogram (Phase 2), without an extra pass over K.
-//   Phase 3 (refinement): one sweep at tau_T accumulates count, S1 = sum u, S2 = sum u^2
-//     (u = [z - tau]_+) and copies every score with u > 0 (the only candidates for the
-//     support, since tau* >= tau_T) into shared memory. Rows whose candidates fit are
-//     solved exactly on chip: safeguarded Newton on Eq. 4 (§3.2), finished by the exact
-//     root of the current support's piece (alpha = 2: (S1-1)/C; alpha = 1.5: the smaller
-//     root of C d^2 - 2 S1 d + S2 - 1 = 0) once no candidate leaves the support. Rows
-//     whose candidates overflow take Newton steps bracketed by §2.4, one full sweep each.
+//   Phase 3 (refinement): a sweep at tau accumulates S1 = sum u, S2 = sum u^2 and the
+//     count (u = [z - tau]_+) and copies every score with u > 0 into shared memory
+//     (64 per row and column half). While tau <= tau* (f(tau) >= 0, true at tau_T) those
+//     copies hold the whole support, so a row whose copies fit is solved exactly on
+//     chip: safeguarded Newton on Eq. 4 (§3.2), finished by the exact root of the
+//     current support's piece (alpha = 2: (S1-1)/C; alpha = 1.5: the smaller root of
+//     C d^2 - 2 S1 d + S2 - 1 = 0) once no candidate leaves the support. A row whose
+//     copies overflow takes one Newton step bracketed by §2.4 and sweeps again. Eq. 4's
+//     f is convex and decreasing in tau, so a Newton step from tau <= tau* stays
+//     <= tau*, and the next sweep's copies (fewer, above a higher tau) again qualify.
 //   Block mask: bit (query tile, key tile) = some row has a key-tile max above its
 //     final tau. Packed 32 key tiles per uint32 (Appendix C.4), plus the transpose for
 //     the backward.
@@ -27,7 +30,7 @@
 //     tolerances once g reaches dK through delta. sum_j g_ij is kept per row for the
 //     backward.
 //
-// Roles (320 threads): warps 0-7 are row owners. Warp w reads TMEM lanes 32(w%4)..+31
+// Roles (352 threads): warps 0-7 are row owners. Warp w reads TMEM lanes 32(w%4)..+31
 // (one query row per lane) and columns [64(w/4), 64(w/4)+64) of every S tile, so two
 // threads share a row and combine partial sums in shared memory. Warp 8 issues TMA
 // loads into a 4-slot ring of 16 KB K/V tiles. Warp 9 owns TMEM and issues the MMAs;
@@ -54,7 +57,7 @@ constexpr int kMma2Warp = 10;   // second MMA issuer: the Ot = g V chain of the 
 constexpr int kOBufs = 3;       // S/A buffers in the output pass (TMEM columns 0, 128, 384)
 constexpr int kSlots = 4;
 constexpr int kSBufs = 4;
-constexpr int kCandPerThread = 32;     // candidates per (row, column half); 64 per row
+constexpr int kCandPerThread = 64;     // candidates per (row, column half); 128 per row
 constexpr float kTolF = 3e-5f;         // |f(tau)| = |sum p - 1| small enough to stop sweeping
 constexpr int kMaxVotes = 72;
 
@@ -564,10 +567,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         break;
       }
 
-      // Phase 3: one refinement sweep at the current tau. The first one (at tau_T) also
-      // collects this thread's candidates u > 0.
-      const bool collect = (sweeps == 0);
-      float S1 = 0.f, S2 = 0.f, C = 0.f;
+      // Phase 3: one refinement sweep at the current tau. Every sweep also collects this
+      // thread's candidates u > 0: when tau <= tau* (f >= 0) they hold the whole support.
+      float S1 = 0.f, S2 = 0.f;
       int nc = 0;
       float* mycand = cand + hf * kCandPerThread * kTile + row;
       sbuf = 0;
@@ -587,50 +589,35 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
             if (!pat.active(i, j0 + cc)) s[cc] = -INFINITY;
         }
         float2 s1[4], s2[4];
-        int cnt[4];
 #pragma unroll
         for (int a = 0; a < 4; ++a) {
           s1[a] = make_float2(0.f, 0.f);
           s2[a] = make_float2(0.f, 0.f);
-          cnt[a] = 0;
         }
-        if (collect) {
-          // Groups of 8 scores: u+ summed per group (feeds S1); only a group with a
-          // positive sum (rare: a support candidate) is scanned element by element.
+        // Groups of 8 scores: u+ summed per group (feeds S1); only a group with a
+        // positive sum (rare: a support candidate) is scanned element by element.
 #pragma unroll
-          for (int g = 0; g < 8; ++g) {
-            float2 v[4];
+        for (int g = 0; g < 8; ++g) {
+          float2 v[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 u = __ffma2_rn(make_float2(s[8 * g + 2 * e], s[8 * g + 2 * e + 1]), make_float2(cz, cz),
-                                          make_float2(-tau, -tau));
-              v[e] = make_float2(fmaxf(u.x, 0.f), fmaxf(u.y, 0.f));
-              s2[e] = __ffma2_rn(v[e], v[e], s2[e]);
-            }
-            const float2 gs = __fadd2_rn(__fadd2_rn(v[0], v[1]), __fadd2_rn(v[2], v[3]));
-            s1[g & 3] = __fadd2_rn(s1[g & 3], gs);
-            if (gs.x + gs.y > 0.f) {
+          for (int e = 0; e < 4; ++e) {
+            const float2 u = __ffma2_rn(make_float2(s[8 * g + 2 * e], s[8 * g + 2 * e + 1]), make_float2(cz, cz),
+                                        make_float2(-tau, -tau));
+            v[e] = make_float2(fmaxf(u.x, 0.f), fmaxf(u.y, 0.f));
+            s2[e] = __ffma2_rn(v[e], v[e], s2[e]);
+          }
+          const float2 gs = __fadd2_rn(__fadd2_rn(v[0], v[1]), __fadd2_rn(v[2], v[3]));
+          s1[g & 3] = __fadd2_rn(s1[g & 3], gs);
+          if (gs.x + gs.y > 0.f) {
 #pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                if (fmaf(s[8 * g + e], cz, -tau) > 0.f) {
-                  if (nc < kCandPerThread) mycand[nc * kTile] = s[8 * g + e];
-                  ++nc;
-                }
+            for (int e = 0; e < 8; ++e) {
+              if (fmaf(s[8 * g + e], cz, -tau) > 0.f) {
+                if (nc < kCandPerThread) mycand[nc * kTile] = s[8 * g + e];
+                ++nc;
               }
             }
           }
-        } else {
-#pragma unroll
-          for (int cc = 0; cc < 64; cc += 2) {
-            const float2 u = __ffma2_rn(make_float2(s[cc], s[cc + 1]), make_float2(cz, cz), make_float2(-tau, -tau));
-            const float2 v = make_float2(fmaxf(u.x, 0.f), fmaxf(u.y, 0.f));
-            const int a = (cc >> 1) & 3;
-            s1[a] = __fadd2_rn(s1[a], v);
-            s2[a] = __ffma2_rn(v, v, s2[a]);
-            cnt[a] += (u.x > 0.f) + (u.y > 0.f);
-          }
         }
-        C += (float)(cnt[0] + cnt[1] + cnt[2] + cnt[3]);
         const float2 s1t = __fadd2_rn(__fadd2_rn(s1[0], s1[1]), __fadd2_rn(s1[2], s1[3]));
         const float2 s2t = __fadd2_rn(__fadd2_rn(s2[0], s2[1]), __fadd2_rn(s2[2], s2[3]));
         S1 += s1t.x + s1t.y;
@@ -642,23 +629,23 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       float* mp = part + hf * 4 * kTile + row;
       mp[0] = S1;
       mp[kTile] = S2;
-      mp[2 * kTile] = collect ? (float)nc : C;
-      mp[3 * kTile] = (float)nc;
+      mp[2 * kTile] = (float)nc;
       named_bar(3, kMathThreads);
       const float* p0 = part + row;
       const float* p1 = part + 4 * kTile + row;
       S1 = p0[0] + p1[0];
       S2 = p0[kTile] + p1[kTile];
-      C = p0[2 * kTile] + p1[2 * kTile];
-      const int nc0 = (int)p0[3 * kTile], nc1 = (int)p1[3 * kTile];
+      const int nc0 = (int)p0[2 * kTile], nc1 = (int)p1[2 * kTile];
+      const float C = (float)(nc0 + nc1);   // support size at tau (alpha = 2: |f'(tau)|)
       named_bar(3, kMathThreads);   // partials consumed before anyone rewrites them
       ++sweeps;
       if (!done) {
         const float f = (AK == kAlpha15) ? S2 - 1.f : S1 - 1.f;
         const float fp = (AK == kAlpha15) ? 2.f * S1 : C;   // |f'(tau)|
         if (f > 0.f) lo = fmaxf(lo, tau); else hi = fminf(hi, tau);
-        if (collect && nc0 <= kCandPerThread && nc1 <= kCandPerThread) {
-          // Every score above tau_T <= tau* is in the two candidate lists: exact on chip.
+        if (f >= 0.f && nc0 <= kCandPerThread && nc1 <= kCandPerThread) {
+          // tau <= tau*, so every score of the support is in the two candidate lists: the
+          // exact solve on chip ends the refinement.
           float t;
           if (solve_list<AK>(cand + row, nc0, cand + kCandPerThread * kTile + row, nc1, kTile, cz, tau, lo, hi,
                              t)) {
