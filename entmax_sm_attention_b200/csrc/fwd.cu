@@ -142,7 +142,7 @@ __device__ bool solve_list(const float* vals0, int n0, const float* vals1, int n
     }
     if (f > 0.f) lo = t; else hi = t;
     float tn = t + f / fp;
-    if (!(tn > lo && tn < hi)) tn = 0.5f * (lo + hi);
+    if (!(tn > lo && tn <= hi && tn != t)) tn = 0.5f * (lo + hi);   // the root may sit at hi; a stalled step bisects
     t = tn;
   }
   t_out = t;
@@ -654,12 +654,14 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           }
         }
         if (!done) {
-          if (fabsf(f) <= kTolF && fp > 0.f) {
+          // f is a sum of C positive terms in fp32; its rounding error grows with C.
+          const float tolf = fmaxf(kTolF, C * 0x1p-22f);
+          if (fabsf(f) <= tolf && fp > 0.f) {
             tau += f / fp;   // final Newton correction, no further sweep needed
             done = true;
           } else {
             float t = tau + f / fp;
-            if (!(t > lo && t < hi)) t = 0.5f * (lo + hi);   // bisection safeguard
+            if (!(t > lo && t <= hi && t != tau)) t = 0.5f * (lo + hi);   // safeguard; the root may sit at hi
             tau = t;
           }
         }

@@ -59,7 +59,7 @@ __device__ bool solve32(const float* vals, int n, int stride, float cz, float t,
     }
     if (f > 0.f) lo = t; else hi = t;
     float tn = t + f / fp;
-    if (!(tn > lo && tn < hi)) tn = 0.5f * (lo + hi);
+    if (!(tn > lo && tn <= hi && tn != t)) tn = 0.5f * (lo + hi);   // the root may sit at hi (uniform scores); a stalled step bisects
     t = tn;
   }
   out = t;
@@ -201,7 +201,7 @@ __global__ void __launch_bounds__(kThreads32) fwd_f32_kernel(const FwdF32Params 
         done = true;
       } else {
         float tn = tau + f / fp;
-        if (!(tn > lo && tn < hi)) tn = 0.5f * (lo + hi);
+        if (!(tn > lo && tn <= hi && tn != tau)) tn = 0.5f * (lo + hi);   // the root may sit at hi (uniform scores); a stalled step bisects
         tau = tn;
       }
     }

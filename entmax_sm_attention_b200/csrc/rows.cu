@@ -116,7 +116,7 @@ __global__ void __launch_bounds__(kRowThreads) rows_kernel(const float* __restri
     }
     if (f > 0.f) lo = t; else hi = t;
     float tn = t + f / fp;
-    if (!(tn > lo && tn < hi)) tn = 0.5f * (lo + hi);
+    if (!(tn > lo && tn <= hi && tn != t)) tn = 0.5f * (lo + hi);   // the root may sit at hi (uniform scores); a stalled step bisects
     t = tn;
   }
   if (threadIdx.x == 0) tau_out[blockIdx.x] = t;

@@ -28,9 +28,13 @@ CASES = [
     small_case("padded_short_kv", B=1, L=260, kv_len=5),
     small_case("window0_L200", L=200, causal=True, window=0),
     small_case("wide_sigma8_L384", L=384, causal=True, sigma_q=8.0),
-    # Near-uniform rows: almost every key is in the support, so the candidate copies
-    # overflow and the threshold takes several Newton sweeps.
+    # Near-uniform rows: at alpha = 1.5 almost every key is in the support, so the
+    # candidate lists overflow and the threshold takes Newton sweeps; at alpha = 2 the
+    # support (28+ keys) still fits and is solved in the max pass.
     small_case("flat_sigma005_L512", L=512, sigma_q=0.05),
+    # Exactly uniform rows (Q = 0, all scores tie): p = 1/n, tau = -n^{1-alpha}; every key is
+    # in the support, so both alphas take the sweep path.
+    small_case("uniform_sigma0_L512", L=512, sigma_q=0.0),
 ]
 
 
@@ -58,13 +62,22 @@ def test_entmax_rows(alpha):
         z = (alpha - 1) * S.double().numpy()
         decided = np.abs(z - taur[:, None]) > 1e-3
         assert np.array_equal((P > 0)[decided], (Pr > 0)[decided])
+    # Uniform rows (all scores tie): p = 1/n and tau = (alpha-1) s - n^{1-alpha}, the upper
+    # end of the §2.4 bracket.
+    for n, v in ((300, 0.0), (1000, 3.7)):
+        S = torch.full((3, n), v, dtype=torch.float32)
+        P, tau = eb.rows(S.cuda(), alpha)
+        P, tau = P.cpu().double().numpy(), tau.cpu().double().numpy()
+        assert np.abs(P - 1.0 / n).max() <= 1e-6
+        assert np.abs(tau - ((alpha - 1) * v - n ** (1 - alpha))).max() <= 1e-5
 
 
 def test_refinement_cap_reports_no_convergence():
     """Refinement capped at one sweep on rows that need several (near-uniform rows whose
-    support overflows the on-chip candidate copies): the status word says so. Per §2.4
-    tau stays inside the bracket, so O stays finite."""
-    w = small_case("capped", L=512, causal=False, sigma_q=0.05)
+    support, 174+ keys per column half at both alphas, overflows the on-chip candidate
+    lists): the status word says so. Per §2.4 tau stays inside the bracket, so O stays
+    finite."""
+    w = small_case("capped", L=512, causal=False, sigma_q=0.002)
     from parity import gpu_run
     from entmax_sm_attention_b200.workloads import make_inputs
     for alpha in (1.5, 2.0):
@@ -111,6 +124,23 @@ def test_single_head_fp32_workload():
     Pr, taur = oracle.entmax_rows(S.cpu(), 1.5)
     assert np.abs(tau.cpu().numpy() - taur).max() <= 1e-5
     assert np.abs(P.cpu().numpy() - Pr).max() <= 1e-5
+
+
+def test_fp32_uniform_rows():
+    """fp32 forward on exactly uniform rows (Q = 0): tau sits at the upper end of the
+    bracket, -n^{1-alpha}, and O is the mean of the active values."""
+    from parity import gpu_run, oracle_problem
+    from entmax_sm_attention_b200.workloads import make_inputs
+
+    for causal in (False, True):
+        w = small_case("uniform_fp32", L=200, dtype="fp32", sigma_q=0.0, causal=causal)
+        inp = make_inputs(w)
+        for alpha in (1.5, 2.0):
+            g = gpu_run(inp, w, alpha, backward=False)
+            assert g["status"][0] == eb.ENTMAX_OK
+            ref = oracle_problem(inp, w, alpha).forward()
+            assert np.abs(g["tau"] - ref["tau"]).max() <= TOL_TAU
+            assert np.abs(g["O"] - ref["O"]).max() <= 1e-2
 
 
 def test_fp32_backward_is_rejected():
