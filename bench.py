@@ -77,6 +77,28 @@ def load_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+# ------------------------------------------------------------ multi-rank plumbing
+def rank_seed(seed: int, rank: int) -> int:
+    """Seed of a rank's batch: every rank works on its own independent batch."""
+    return seed + rank
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The slowest rank's value (timings are taken as the max over ranks)."""
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, tokens_per_step: int, steps: int, max_ms: float) -> float:
+    """Whole-job tokens/s: the tokens all ranks processed over the slowest rank's time."""
+    return world * tokens_per_step * steps / (max_ms / 1e3)
+
+
 # ------------------------------------------------------------------ clock sampling
 class ClockSampler:
     """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
@@ -208,7 +230,7 @@ def run_ours(args):
     w = WORKLOADS[args.workload]
     alpha = args.alpha
 
-    host = make_inputs(w, seed=args.seed + rank)
+    host = make_inputs(w, seed=rank_seed(args.seed, rank))
     pinned = {k: v.pin_memory() for k, v in host.items()}
     d = {k: v.to(dev) for k, v in host.items()}
     kv = None if w.kv_len is None else torch.tensor(w.kv_len_list(), dtype=torch.int32, device=dev)
@@ -256,14 +278,10 @@ def run_ours(args):
     clk = clocks.stop()
     fwd_ms = [e[0].elapsed_time(e[1]) for e in ev]
     bwd_ms = [e[1].elapsed_time(e[2]) for e in ev]
-    total_ms = sum(fwd_ms) + sum(bwd_ms)
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(fwd_ms) + sum(bwd_ms), world, dev)
     ms_per_step = total_ms / args.steps
     tokens_per_step = w.B * w.L
-    value = world * tokens_per_step * args.steps / (total_ms / 1e3)
+    value = job_throughput(world, tokens_per_step, args.steps, total_ms)
 
     # ---- end to end through the public API: pinned host -> device, fwd+bwd, device -> host
     out_host = {k: torch.empty(shp, dtype=torch.float32).pin_memory() for k in ("O", "dQ", "dK", "dV")}
@@ -281,10 +299,8 @@ def run_ours(args):
             out_host[k].copy_(src, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-    e2e_value = world * tokens_per_step * args.steps / (float(e2e_ms.item()) / 1e3)
+    e2e_value = job_throughput(world, tokens_per_step, args.steps,
+                               max_over_ranks(e0.elapsed_time(e1), world, dev))
 
     # ---- work actually done (per-tile counters written by the forward)
     M, st = eb.block_mask((desc, ws))
