@@ -30,12 +30,14 @@
 //     tolerances once g reaches dK through delta. sum_j g_ij is kept per row for the
 //     backward.
 //
-// Roles (352 threads): warps 0-7 are row owners. Warp w reads TMEM lanes 32(w%4)..+31
+// Roles (384 threads): warps 0-7 are row owners. Warp w reads TMEM lanes 32(w%4)..+31
 // (one query row per lane) and columns [64(w/4), 64(w/4)+64) of every S tile, so two
 // threads share a row and combine partial sums in shared memory. Warp 8 issues TMA
-// loads into a 4-slot ring of 16 KB K/V tiles. Warp 9 owns TMEM and issues the MMAs;
-// in the output pass warp 10 issues the Ot = g V chain, because one thread cannot
-// issue N=64 MMAs as fast as the tensor cores retire them.
+// loads into a 4-slot ring of 16 KB K/V tiles. Warp 9 owns TMEM and issues the S = Q K^T
+// MMAs of every phase; in the output pass warp 11 issues the O = A V chain and warp 10
+// the Ot = g V chain. One thread issues an N=64 MMA only every ~54 cycles and each
+// mbarrier wait costs ~200 cycles even when the phase is complete, so one issuer per
+// chain keeps each below the tile's tensor time.
 // TMEM (512 columns): during the sweeps, four S buffers at 0/128/256/384, so the MMA
 // warp runs up to three tiles ahead. During the output pass:
 //   - three S buffers at 0, 128 and 384 (tile k in buffer k % 3). The thread owning key
@@ -49,11 +51,12 @@ namespace entmax {
 
 namespace {
 
-constexpr int kThreads = 352;
+constexpr int kThreads = 384;
 constexpr int kMathThreads = 256;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kMma2Warp = 10;   // second MMA issuer: the Ot = g V chain of the output pass
+constexpr int kMma3Warp = 11;   // third MMA issuer: the O = A V chain of the output pass
 constexpr int kOBufs = 3;       // S/A buffers in the output pass (TMEM columns 0, 128, 384)
 constexpr int kSlots = 4;
 constexpr int kSBufs = 4;
@@ -302,38 +305,18 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           sbuf = 0;
           for_each_bit(list, kMaskWords, [&](int) { sweep_tile(); });
         } else {
-          // Output pass. S of tile k+1 is issued before O += A V of tile k, so it overlaps
-          // the row owners' work on tile k. Tile k uses buffer c = k % 3 at TMEM column
-          // 0, 128 or 384. K_k is at ring position base + 2k, V_k at base + 2k + 1.
+          // Output pass: this warp issues only the S tiles; tile k uses buffer c = k % 3
+          // at TMEM column 0, 128 or 384, which is free once O and Ot of tile k-3 are done.
+          // K_k is at ring position base + 2k, V_k at base + 2k + 1.
           int n = 0;
 #pragma unroll
           for (int w = 0; w < kMaskWords; ++w) n += __popc(list[w]);
           const uint32_t base = seq;
-          auto issue_s = [&](int k) {
+          for (int k = 0; k < n; ++k) {
             const int c = k % kOBufs;
-            if (k >= kOBufs) mbar_wait(&sh.pv_done[c], ((k - kOBufs) / kOBufs) & 1, status, abrt);   // buffer free
+            if (k >= kOBufs) mbar_wait(&sh.pv_done[c], ((k - kOBufs) / kOBufs) & 1, status, abrt);
             mma_s(base + 2 * k, c == 0 ? 0u : (c == 1 ? 128u : 384u));
             mma_commit(&sh.o_full[c]);
-          };
-          if (n > 0) issue_s(0);
-          for (int k = 0; k < n; ++k) {
-            if (k + 1 < n) issue_s(k + 1);
-            const int c = k % kOBufs;
-            const uint32_t pa = c == 0 ? 0u : (c == 1 ? 128u : 384u);
-            const uint32_t vpos = base + 2 * k + 1;
-            const int vslot = vpos % kSlots;
-            mbar_wait(&sh.full[vslot], (vpos / kSlots) & 1, status, abrt);
-            mbar_wait(&sh.o_ready[c], (k / kOBufs) & 1, status, abrt);   // A and g of tile k written
-            tc_fence_after();
-            const uint32_t vb = smem_u32(ring + vslot * kTileBytes);
-#pragma unroll
-            for (int t = 0; t < 8; ++t) {
-              // keys 16t..16t+15: half t/4, pair columns 8(t%4) within the half's A block
-              const uint32_t col = pa + (t >> 2) * 64 + (t & 3) * 8;
-              mma_ts(T + 256, T + col, sdesc_sw128(vb + t * 2048, 8192, 1024), idO, (k > 0 || t > 0) ? 1u : 0u);
-            }
-            mma_commit(&sh.empty[vslot]);
-            mma_commit(&sh.pv_done[c]);
           }
           seq = base + 2 * n;
         }
@@ -372,6 +355,45 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           for (int t = 0; t < 8; ++t) {
             const uint32_t col = pa + (t >> 2) * 64 + (t & 3) * 8 + 32;   // g block of the half
             mma_ts(T + 320, T + col, sdesc_sw128(vb + t * 2048, 8192, 1024), idO, (k > 0 || t > 0) ? 1u : 0u);
+          }
+          mma_commit(&sh.empty[vslot]);
+          mma_commit(&sh.pv_done[c]);
+        }
+      }
+      __syncwarp();
+      if (kind != kKindSweep) break;
+    }
+  } else if (warp == kMma3Warp) {
+    // ------------------------------------------------- third MMA issuer (output pass)
+    const uint32_t idO = idesc_f16(128, 64, 0, 1);
+    uint32_t seq = 0;   // ring positions, tracked exactly like the producer's
+    for_each_bit(act, kMaskWords, [&](int) { ++seq; });
+    while (true) {
+      named_bar(1, kThreads);
+      const int kind = sh.ctl_kind;
+      uint32_t list[kMaskWords];
+#pragma unroll
+      for (int w = 0; w < kMaskWords; ++w) list[w] = sh.lists[sh.ctl_buf][w];
+      int n = 0;
+#pragma unroll
+      for (int w = 0; w < kMaskWords; ++w) n += __popc(list[w]);
+      if (kind == kKindSweep) {
+        seq += n;
+      } else if (lane == 0) {
+        const uint32_t base = seq;
+        for (int k = 0; k < n; ++k) {
+          const int c = k % kOBufs;
+          const uint32_t pa = c == 0 ? 0u : (c == 1 ? 128u : 384u);
+          const uint32_t vpos = base + 2 * k + 1;
+          const int vslot = vpos % kSlots;
+          mbar_wait(&sh.full[vslot], (vpos / kSlots) & 1, status, abrt);
+          mbar_wait(&sh.o_ready[c], (k / kOBufs) & 1, status, abrt);
+          tc_fence_after();
+          const uint32_t vb = smem_u32(ring + vslot * kTileBytes);
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            const uint32_t col = pa + (t >> 2) * 64 + (t & 3) * 8;   // A block of the half
+            mma_ts(T + 256, T + col, sdesc_sw128(vb + t * 2048, 8192, 1024), idO, (k > 0 || t > 0) ? 1u : 0u);
           }
           mma_commit(&sh.empty[vslot]);
           mma_commit(&sh.pv_done[c]);
