@@ -24,7 +24,9 @@
 // fp16 copies of dO and V (exact conversions of the bf16 inputs). The row owners copy
 // dQ_i from TMEM into a swizzled fp32 staging tile in shared memory, and one thread adds
 // it to global dQ with a TMA reduce-add (cp.reduce.async.bulk.tensor .add), one query
-// tile behind the MMAs. Warp 8 issues the TMA loads, warp 9 the MMAs.
+// tile behind the MMAs. Warp 8 issues the TMA loads. Warp 9 issues S, dA and the dQ chain,
+// warp 10 the dV and dK chains: one thread issues an N=64 MMA only every ~54 cycles, so
+// the 40 MMAs of a tile's gradient products are split between two issuers.
 // TMEM: [0,128) S, [128,256) dA, [256,320) dV, [320,384) dK, [384,512) dQ x2.
 #include "common.cuh"
 #include "kernels.h"
@@ -33,9 +35,10 @@ namespace entmax {
 
 namespace {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;
 constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
+constexpr int kMmaWarp = 9;    // S, dA and the dQ chain
+constexpr int kMma2Warp = 10;  // the dV and dK chains
 constexpr int kStages = 2;
 constexpr int kPairBytes = 2 * kTileBytes;   // Q_i and dO_i
 
@@ -84,13 +87,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&sh.full[s], 1);
-      mbar_init(&sh.empty[s], 1);
+      mbar_init(&sh.empty[s], 2);   // one commit per MMA warp reading the stage
     }
     mbar_init(&sh.bar_kv, 1);
     mbar_init(&sh.s_full, 1);
     mbar_init(&sh.sda_free, 8);
     mbar_init(&sh.p_ready, 8);
-    mbar_init(&sh.mma2_done, 1);
+    mbar_init(&sh.mma2_done, 2);  // dQ chain and dV/dK chains
     sh.abort_flag = 0;
     fence_mbar_init();
   }
@@ -132,15 +135,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     }
     __syncwarp();
   } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------------- MMA issuer
+    // -------------------------------------------- MMA issuer: S, dA and the dQ chain
     if (lane == 0 && nq > 0) {
       const uint32_t idS = idesc_bf16(128, 128, 0, 0);    // S = Q K^T
       const uint32_t idA = idesc_f16(128, 128, 0, 0);     // dA = dO V^T (fp16 copies)
-      const uint32_t idV = idesc_f16(128, 64, 1, 1);      // dV += A^T dO: A MN-major (sA), B MN-major
-      const uint32_t idK = idesc_bf16(128, 64, 1, 1);     // dK += dS^T Q: A MN-major (sdS), B MN-major
       const uint32_t idQ = idesc_bf16(128, 64, 0, 1);     // dQ = dS K: A K-major (sdS), B MN-major (K_j)
       const uint32_t kA = smem_u32(sK), vA = smem_u32(sV);
-      const uint32_t aH = smem_u32(sA), dH = smem_u32(sdS), dL = smem_u32(sdSl);
+      const uint32_t dH = smem_u32(sdS), dL = smem_u32(sdSl);
       mbar_wait(&sh.bar_kv, 0, status, abrt);
       // S = Q_s K^T and dA = dO_s V^T into TMEM [0,256).
       auto issue_sda = [&](int s) {
@@ -159,11 +160,34 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       issue_sda(0);
       for (int s = 0; s < nq; ++s) {
         if (s + 1 < nq) issue_sda(s + 1);   // overlaps the row owners' work on tile s
-        const int st = s % kStages;
-        const uint32_t qA = smem_u32(ring + st * kPairBytes), oA = qA + kTileBytes;
         mbar_wait(&sh.p_ready, s & 1, status, abrt);   // A and dS of tile s in shared memory
         tc_fence_after();
         const uint32_t dq = T + 384 + (s & 1) * 64;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          // dQ_s = dS K_j: K = keys (16 per step; panel t/4), M = queries.
+          const uint32_t koff = (t >> 2) * kTileBytes + (t & 3) * 32;
+          const uint64_t bK = sdesc_sw128(kA + t * 2048, 8192, 1024);
+          mma_ss(dq, sdesc_sw128(dH + koff, 16, 1024), bK, idQ, t > 0 ? 1u : 0u);
+          mma_ss(dq, sdesc_sw128(dL + koff, 16, 1024), bK, idQ, 1u);
+        }
+        mma_commit(&sh.empty[s % kStages]);   // S and dA of tile s were this warp's last reads
+        mma_commit(&sh.mma2_done);
+      }
+    }
+    __syncwarp();
+  } else if (warp == kMma2Warp) {
+    // --------------------------------------------- second MMA issuer: dV and dK chains
+    if (lane == 0 && nq > 0) {
+      const uint32_t idV = idesc_f16(128, 64, 1, 1);      // dV += A^T dO: A MN-major (sA), B MN-major
+      const uint32_t idK = idesc_bf16(128, 64, 1, 1);     // dK += dS^T Q: A MN-major (sdS), B MN-major
+      const uint32_t aH = smem_u32(sA), dH = smem_u32(sdS), dL = smem_u32(sdSl);
+      for (int s = 0; s < nq; ++s) {
+        const int st = s % kStages;
+        const uint32_t qA = smem_u32(ring + st * kPairBytes), oA = qA + kTileBytes;
+        mbar_wait(&sh.full[st], (s / kStages) & 1, status, abrt);   // Q_s and dO_s landed
+        mbar_wait(&sh.p_ready, s & 1, status, abrt);                // A and dS of tile s written
+        tc_fence_after();
 #pragma unroll
         for (int t = 0; t < 8; ++t) {
           // dV += A^T dO_s and dK += dS^T Q_s: K = queries (16 per step), M = keys.
@@ -172,11 +196,6 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
           mma_ss(T + 256, sdesc_sw128(aH + t * 2048, 16384, 1024), bO, idV, acc);
           mma_ss(T + 320, sdesc_sw128(dH + t * 2048, 16384, 1024), bQ, idK, acc);
           mma_ss(T + 320, sdesc_sw128(dL + t * 2048, 16384, 1024), bQ, idK, 1u);
-          // dQ_s = dS K_j: K = keys (16 per step; panel t/4), M = queries.
-          const uint32_t koff = (t >> 2) * kTileBytes + (t & 3) * 32;
-          const uint64_t bK = sdesc_sw128(kA + t * 2048, 8192, 1024);
-          mma_ss(dq, sdesc_sw128(dH + koff, 16, 1024), bK, idQ, t > 0 ? 1u : 0u);
-          mma_ss(dq, sdesc_sw128(dL + koff, 16, 1024), bK, idQ, 1u);
         }
         mma_commit(&sh.empty[st]);
         mma_commit(&sh.mma2_done);

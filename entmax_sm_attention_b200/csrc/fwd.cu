@@ -267,7 +267,6 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     uint32_t sfree_par = 0;      // per sweep S buffer: parity of its uses so far (bit b)
     uint32_t sbuf = 0;           // next sweep S buffer
     const uint32_t idS = idesc_bf16(128, 128, 0, 0);
-    const uint32_t idO = idesc_f16(128, 64, 0, 1);   // A (TMEM) and V copy, both fp16
     const uint32_t sQa = smem_u32(sQ);
     // S = Q K^T from ring position `pos` into TMEM columns [dcol, dcol+128).
     auto mma_s = [&](uint32_t pos, uint32_t dcol) {
