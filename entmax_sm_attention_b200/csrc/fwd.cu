@@ -104,13 +104,33 @@ __device__ __forceinline__ void ld64(uint32_t taddr, float (&s)[64]) {
   }
 }
 
+// Adds one candidate at u = z - t to the sums of the current support (u > 0), without
+// a branch: the lanes of a warp follow one path whatever their candidates.
 __device__ __forceinline__ void accumulate(float u, float& S1, float& S2, float& C, float& umin) {
-  if (u > 0.f) {
-    S1 += u;
-    S2 = fmaf(u, u, S2);
-    C += 1.f;
-    umin = fminf(umin, u);
+  const bool in = u > 0.f;
+  const float v = in ? u : 0.f;
+  S1 += v;
+  S2 = fmaf(v, v, S2);
+  C += in ? 1.f : 0.f;
+  umin = fminf(umin, in ? u : INFINITY);
+}
+
+// Support sums of list[k*stride], k < n, at t: four independent partial sums, so the
+// adds do not form one serial chain.
+__device__ __forceinline__ void sum_list(const float* list, int n, int stride, float cz, float t, float& S1,
+                                         float& S2, float& C, float& umin) {
+  float a1[4] = {0.f, 0.f, 0.f, 0.f}, a2[4] = {0.f, 0.f, 0.f, 0.f}, ac[4] = {0.f, 0.f, 0.f, 0.f};
+  float am[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
+  int k = 0;
+  for (; k + 4 <= n; k += 4) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) accumulate(fmaf(list[(k + q) * stride], cz, -t), a1[q], a2[q], ac[q], am[q]);
   }
+  for (; k < n; ++k) accumulate(fmaf(list[k * stride], cz, -t), a1[0], a2[0], ac[0], am[0]);
+  S1 += (a1[0] + a1[1]) + (a1[2] + a1[3]);
+  S2 += (a2[0] + a2[1]) + (a2[2] + a2[3]);
+  C += (ac[0] + ac[1]) + (ac[2] + ac[3]);
+  umin = fminf(umin, fminf(fminf(am[0], am[1]), fminf(am[2], am[3])));
 }
 
 // Safeguarded solve of Eq. 4 for one row over raw scores vals0[k*stride] (k < n0) and
@@ -122,8 +142,8 @@ __device__ bool solve_list(const float* vals0, int n0, const float* vals1, int n
                            float lo, float hi, float& t_out) {
   for (int it = 0; it < 48; ++it) {
     float S1 = 0.f, S2 = 0.f, C = 0.f, umin = INFINITY;
-    for (int k = 0; k < n0; ++k) accumulate(fmaf(vals0[k * stride], cz, -t), S1, S2, C, umin);
-    for (int k = 0; k < n1; ++k) accumulate(fmaf(vals1[k * stride], cz, -t), S1, S2, C, umin);
+    sum_list(vals0, n0, stride, cz, t, S1, S2, C, umin);
+    sum_list(vals1, n1, stride, cz, t, S1, S2, C, umin);
     const float f = (AK == kAlpha15) ? S2 - 1.f : S1 - 1.f;
     const float fp = (AK == kAlpha15) ? 2.f * S1 : C;   // |f'(t)|
     if (C > 0.f) {
@@ -453,15 +473,23 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     bool done = !valid;
     if (valid) {
       // Only tile maxima above lo = m - 1 can be in the support of the maxima problem.
-      // Gather up to 32 of them into this thread's candidate area (unused until the
-      // first sweep). Entmax on any subset of the scores has a threshold <= tau*, so
-      // keeping only the first 32 still gives a lower bound.
+      // Gather up to kCandPerThread of them into this thread's candidate area (unused
+      // until the first sweep). Entmax on any subset of the scores has a threshold
+      // <= tau*, so keeping only the first ones still gives a lower bound. Tiles that
+      // are not active hold -inf. Eight independent loads per step.
       float* mylist = cand + hf * kCandPerThread * kTile + row;
       int nl = 0;
-      for_each_bit(act, kMaskWords, [&](int jt) {
-        const float v = ord2f(tmax[jt * kTile + row]);
-        if (nl < kCandPerThread && fmaf(v, cz, -lo) > 0.f) mylist[nl++ * kTile] = v;
-      });
+      for (int jb = 0; jb < p.Tc; jb += 8) {
+        float v[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) v[q] = jb + q < p.Tc ? ord2f(tmax[(jb + q) * kTile + row]) : -INFINITY;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const bool take = fmaf(v[q], cz, -lo) > 0.f && nl < kCandPerThread;
+          if (take) mylist[nl * kTile] = v[q];
+          nl += take ? 1 : 0;
+        }
+      }
       float t = lo;
       solve_list<AK>(mylist, nl, mylist, 0, kTile, cz, lo, lo, hi, t);
       tau = fminf(fmaxf(t, lo), hi);
@@ -477,13 +505,26 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       const bool need = !done && sweeps < p.max_sweeps;
       const bool final_mask = !rows_any(need, sh.votes, r, lane, kMathThreads);
       if (hf == 0) {
-        // Tiles that some row still needs (refinement) or that hold a nonzero (mask).
-        for_each_bit(act, kMaskWords, [&](int jt) {
-          const bool take = final_mask ? valid : !done;
-          const bool hit = take && fmaf(ord2f(tmax[jt * kTile + row]), cz, -tau) > 0.f;
-          const uint32_t bal = __ballot_sync(0xffffffffu, hit);
-          if (lane == 0 && bal) atomicOr(&sh.lists[buf][jt >> 5], 1u << (jt & 31));
-        });
+        // Tiles that some row still needs (refinement) or that hold a nonzero (mask): each
+        // warp builds a word of 32 tile bits from eight independent loads and votes per
+        // step, and ORs it into the list once.
+        const bool take = final_mask ? valid : !done;
+        for (int w = 0; w < kMaskWords; ++w) {
+          if (act[w] == 0) continue;
+          uint32_t word = 0;
+          for (int b0 = 0; b0 < 32 && w * 32 + b0 < p.Tc; b0 += 8) {
+            const int jb = w * 32 + b0;
+            float v[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) v[q] = jb + q < p.Tc ? ord2f(tmax[(jb + q) * kTile + row]) : -INFINITY;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const uint32_t bal = __ballot_sync(0xffffffffu, take && fmaf(v[q], cz, -tau) > 0.f);
+              word |= (bal != 0u ? 1u : 0u) << (b0 + q);
+            }
+          }
+          if (lane == 0 && word) atomicOr(&sh.lists[buf][w], word & act[w]);
+        }
       }
       named_bar(2, kMathThreads);
       if (tid == 0) {
