@@ -656,8 +656,10 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           s1[a] = make_float2(0.f, 0.f);
           s2[a] = make_float2(0.f, 0.f);
         }
-        // Groups of 8 scores: u+ summed per group (feeds S1); only a group with a
-        // positive sum (rare: a support candidate) is scanned element by element.
+        // Groups of 8 scores: u+ summed per group (feeds S1), straight-line for all eight
+        // groups; then only the groups with a positive sum (rare: a support candidate) are
+        // scanned element by element.
+        uint32_t gmask = 0;
 #pragma unroll
         for (int g = 0; g < 8; ++g) {
           float2 v[4];
@@ -670,12 +672,18 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           }
           const float2 gs = __fadd2_rn(__fadd2_rn(v[0], v[1]), __fadd2_rn(v[2], v[3]));
           s1[g & 3] = __fadd2_rn(s1[g & 3], gs);
-          if (gs.x + gs.y > 0.f) {
+          gmask |= (gs.x + gs.y > 0.f ? 1u : 0u) << g;
+        }
+        if (gmask) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              if (fmaf(s[8 * g + e], cz, -tau) > 0.f) {
-                if (nc < kCandPerThread) mycand[nc * kTile] = s[8 * g + e];
-                ++nc;
+          for (int g = 0; g < 8; ++g) {
+            if ((gmask >> g) & 1u) {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                if (fmaf(s[8 * g + e], cz, -tau) > 0.f) {
+                  if (nc < kCandPerThread) mycand[nc * kTile] = s[8 * g + e];
+                  ++nc;
+                }
               }
             }
           }
