@@ -5,10 +5,11 @@
 //   Phase 1 (maximum): stream the structurally active key tiles; S = Q K^T on the
 //     tensor cores (tcgen05, accumulator in TMEM). Each row keeps its max in every key
 //     tile, in shared memory.
-//   Initial threshold: the row's tau restricted to its key-tile maxima. Entmax on a
-//     subset of the scores has a smaller threshold than on all of them (fewer
-//     nonnegative terms in Eq. 4), so this is a lower bound tau_T <= tau*. It plays the
-//     role the paper gives its on-chip histogram (Phase 2), without an extra pass over K.
+//   Initial threshold: each thread keeps the four largest of its half-tile maxima in
+//     registers; the row's tau restricted to those eight scores is a lower bound
+//     tau_T <= tau* (entmax on a subset of the scores has fewer nonnegative terms in
+//     Eq. 4). It plays the role the paper gives its on-chip histogram (Phase 2), without
+//     an extra pass over K.
 //   Phase 3 (refinement): a sweep at tau accumulates S1 = sum u, S2 = sum u^2 and the
 //     count (u = [z - tau]_+) and copies every score with u > 0 into shared memory
 //     (64 per row and column half). While tau <= tau* (f(tau) >= 0, true at tau_T) those
@@ -170,6 +171,38 @@ __device__ bool solve_list(const float* vals0, int n0, const float* vals1, int n
   }
   t_out = t;
   return false;
+}
+
+// Threshold of Eq. 4 restricted to eight raw scores v (some may be -inf), in registers:
+// safeguarded Newton from lo inside [lo, hi], finished by the exact root of the current
+// support's piece once no value leaves the support. A subset of the row's scores has a
+// threshold at or below the row's tau*, so the result is a lower bound on tau*.
+template <int AK>
+__device__ __forceinline__ float solve8(const float (&v)[8], float cz, float lo, float hi) {
+  float t = lo;
+  for (int it = 0; it < 24; ++it) {
+    float S1 = 0.f, S2 = 0.f, C = 0.f, umin = INFINITY;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) accumulate(fmaf(v[q], cz, -t), S1, S2, C, umin);
+    const float f = (AK == kAlpha15) ? S2 - 1.f : S1 - 1.f;
+    const float fp = (AK == kAlpha15) ? 2.f * S1 : C;
+    if (C > 0.f) {
+      float d = -1.f;
+      if (AK == kAlpha15) {
+        const float disc = S1 * S1 - C * (S2 - 1.f);
+        if (disc >= 0.f) d = (S2 - 1.f) / (S1 + sqrtf(disc));
+      } else {
+        d = (S1 - 1.f) / C;
+      }
+      if (d >= 0.f && d < umin) return t + d;
+    }
+    if (fabsf(f) <= 1e-7f && fp > 0.f) return t + f / fp;
+    if (f > 0.f) lo = t; else hi = t;
+    float tn = t + f / fp;
+    if (!(tn > lo && tn <= hi && tn != t)) tn = 0.5f * (lo + hi);
+    t = tn;
+  }
+  return lo;   // not settled: lo is still a lower bound
 }
 
 }  // namespace
@@ -431,6 +464,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     const float cz = p.cz;
     uint32_t sfull_par = 0, sbuf = 0;
     float m = -INFINITY;
+    float top[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 
     // Phase 1: per-key-tile row maxima over this thread's column half (combined in smem).
     for_each_bit(act, kMaskWords, [&](int jt) {
@@ -456,13 +490,26 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       const float tm = fmaxf(fmaxf(fmaxf(t8[0], t8[1]), fmaxf(t8[2], t8[3])),
                              fmaxf(fmaxf(t8[4], t8[5]), fmaxf(t8[6], t8[7])));
       atomicMax(&tmax[jt * kTile + row], f2ord(tm));
-      m = fmaxf(m, tm);
+      // Keep the four largest half-tile maxima, sorted (compare-exchange, no branch).
+      float x = tm;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float big = fmaxf(top[k], x);
+        x = fminf(top[k], x);
+        top[k] = big;
+      }
       sbuf = (sbuf + 1) & (kSBufs - 1);
     });
-    // Row max over both column halves.
-    part[hf * 4 * kTile + row] = m;
+    // Both column halves' four largest half-tile maxima: the row max and the values of
+    // the initial threshold.
+#pragma unroll
+    for (int k = 0; k < 4; ++k) part[(hf * 4 + k) * kTile + row] = top[k];
     named_bar(3, kMathThreads);
-    m = fmaxf(part[row], part[4 * kTile + row]);
+    float v8[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) v8[k] = part[k * kTile + row];
+    named_bar(3, kMathThreads);   // read before anyone rewrites the partials
+    m = fmaxf(v8[0], v8[4]);
 
     // Bracket (§2.4) and the tile-maxima lower bound (identical in both threads of a row).
     const int n_act = valid ? pat.count(i) : 1;
@@ -472,26 +519,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     float tau = INFINITY;
     bool done = !valid;
     if (valid) {
-      // Only tile maxima above lo = m - 1 can be in the support of the maxima problem.
-      // Gather up to kCandPerThread of them into this thread's candidate area (unused
-      // until the first sweep). Entmax on any subset of the scores has a threshold
-      // <= tau*, so keeping only the first ones still gives a lower bound. Tiles that
-      // are not active hold -inf. Eight independent loads per step.
-      float* mylist = cand + hf * kCandPerThread * kTile + row;
-      int nl = 0;
-      for (int jb = 0; jb < p.Tc; jb += 8) {
-        float v[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) v[q] = jb + q < p.Tc ? ord2f(tmax[(jb + q) * kTile + row]) : -INFINITY;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const bool take = fmaf(v[q], cz, -lo) > 0.f && nl < kCandPerThread;
-          if (take) mylist[nl * kTile] = v[q];
-          nl += take ? 1 : 0;
-        }
-      }
-      float t = lo;
-      solve_list<AK>(mylist, nl, mylist, 0, kTile, cz, lo, lo, hi, t);
+      // The eight largest half-tile maxima of the row are a subset of its scores, so the
+      // threshold of entmax on them is a lower bound tau_T <= tau*.
+      const float t = solve8<AK>(v8, cz, lo, hi);
       tau = fminf(fmaxf(t, lo), hi);
     }
     float2 sg2 = make_float2(0.f, 0.f);   // sum_j g_ij, two chains
