@@ -79,11 +79,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* s
   }
 }
 
-// Warp-wide variant for code that all 32 lanes execute: lane 0 polls the barrier (the
-// other lanes do not spin on shared memory), then __syncwarp reconverges the warp before
-// the .sync.aligned tcgen05 instructions and bar.sync that follow, and makes the
-// barrier's completion (and the memory it guards) visible to every lane.
+// Warp-wide variant for code that all 32 lanes execute. Fast path: every lane probes the
+// phase once (acquiring it) and the warp votes; the lanes read the same barrier word, so
+// the vote is uniform. An mbarrier probe costs ~200 cycles even when the phase has
+// completed, and this saves a lane-0 round trip and a shuffle. Slow path: lane 0 polls
+// with the bounded wait (the other lanes do not spin on shared memory), then __syncwarp
+// reconverges the warp before the .sync.aligned tcgen05 instructions and bar.sync that
+// follow, and makes the barrier's completion (and the memory it guards) visible to every
+// lane.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, int* status, volatile int* abort) {
+  if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
   int ok = 1;
   if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, status, abort) ? 1 : 0;
   __syncwarp();
