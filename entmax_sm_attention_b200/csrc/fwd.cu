@@ -321,10 +321,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     uint32_t sbuf = 0;           // next sweep S buffer
     const uint32_t idS = idesc_bf16(128, 128, 0, 0);
     const uint32_t sQa = smem_u32(sQ);
-    // S = Q K^T from ring position `pos` into TMEM columns [dcol, dcol+128).
+    // S = Q K^T from ring position `pos` (already landed) into TMEM columns [dcol, dcol+128).
     auto mma_s = [&](uint32_t pos, uint32_t dcol) {
       const int slot = pos % kSlots;
-      mbar_wait(&sh.full[slot], (pos / kSlots) & 1, status, abrt);
       tc_fence_after();
       const uint32_t kb = smem_u32(ring + slot * kTileBytes);
 #pragma unroll
@@ -335,9 +334,12 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     };
     auto sweep_tile = [&]() {
       const uint32_t bf = sbuf;
-      mbar_wait(&sh.s_free[bf], ((sfree_par >> bf) & 1) ^ 1, status, abrt);   // buffer consumed
+      const uint32_t pos = seq++;
+      // S buffer consumed by the row owners, and K tile landed.
+      mbar_wait2(&sh.s_free[bf], ((sfree_par >> bf) & 1) ^ 1, &sh.full[pos % kSlots], (pos / kSlots) & 1, status,
+                 abrt);
       sfree_par ^= 1u << bf;
-      mma_s(seq++, bf * 128);
+      mma_s(pos, bf * 128);
       mma_commit(&sh.s_full[bf]);
       sbuf = (sbuf + 1) & (kSBufs - 1);
     };
@@ -366,8 +368,13 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           const uint32_t base = seq;
           for (int k = 0; k < n; ++k) {
             const int c = k % kOBufs;
-            if (k >= kOBufs) mbar_wait(&sh.pv_done[c], ((k - kOBufs) / kOBufs) & 1, status, abrt);
-            mma_s(base + 2 * k, c == 0 ? 0u : (c == 1 ? 128u : 384u));
+            const uint32_t pos = base + 2 * k;
+            if (k >= kOBufs)
+              mbar_wait2(&sh.pv_done[c], ((k - kOBufs) / kOBufs) & 1, &sh.full[pos % kSlots], (pos / kSlots) & 1,
+                         status, abrt);
+            else
+              mbar_wait(&sh.full[pos % kSlots], (pos / kSlots) & 1, status, abrt);
+            mma_s(pos, c == 0 ? 0u : (c == 1 ? 128u : 384u));
             mma_commit(&sh.o_full[c]);
           }
           seq = base + 2 * n;
@@ -399,8 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           const uint32_t pa = c == 0 ? 0u : (c == 1 ? 128u : 384u);
           const uint32_t vpos = base + 2 * k + 1;
           const int vslot = vpos % kSlots;
-          mbar_wait(&sh.full[vslot], (vpos / kSlots) & 1, status, abrt);
-          mbar_wait(&sh.o_ready[c], (k / kOBufs) & 1, status, abrt);
+          mbar_wait2(&sh.full[vslot], (vpos / kSlots) & 1, &sh.o_ready[c], (k / kOBufs) & 1, status, abrt);
           tc_fence_after();
           const uint32_t vb = smem_u32(ring + vslot * kTileBytes);
 #pragma unroll
@@ -438,8 +444,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           const uint32_t pa = c == 0 ? 0u : (c == 1 ? 128u : 384u);
           const uint32_t vpos = base + 2 * k + 1;
           const int vslot = vpos % kSlots;
-          mbar_wait(&sh.full[vslot], (vpos / kSlots) & 1, status, abrt);
-          mbar_wait(&sh.o_ready[c], (k / kOBufs) & 1, status, abrt);
+          mbar_wait2(&sh.full[vslot], (vpos / kSlots) & 1, &sh.o_ready[c], (k / kOBufs) & 1, status, abrt);
           tc_fence_after();
           const uint32_t vb = smem_u32(ring + vslot * kTileBytes);
 #pragma unroll

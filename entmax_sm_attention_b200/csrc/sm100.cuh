@@ -79,6 +79,31 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* s
   }
 }
 
+// Non-blocking probe of a phase (mbarrier.test_wait): the thread is never suspended, so
+// probes of different barriers issued back to back overlap their latencies.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Waits for phase p1 of b1 and phase p2 of b2: both are probed back to back first; the
+// bounded waits run only if a phase is still open.
+__device__ __forceinline__ bool mbar_wait2(uint64_t* b1, uint32_t p1, uint64_t* b2, uint32_t p2, int* status,
+                                           volatile int* abort) {
+  const bool r1 = mbar_test_wait(b1, p1);
+  const bool r2 = mbar_test_wait(b2, p2);
+  if (r1 && r2) return true;
+  const bool w1 = mbar_wait(b1, p1, status, abort);
+  const bool w2 = mbar_wait(b2, p2, status, abort);
+  return w1 && w2;
+}
+
 // Warp-wide variant for code that all 32 lanes execute. Fast path: every lane probes the
 // phase once (acquiring it) and the warp votes; the lanes read the same barrier word, so
 // the vote is uniform. An mbarrier probe costs ~200 cycles even when the phase has
