@@ -140,20 +140,22 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       const uint32_t idS = idesc_bf16(128, 128, 0, 0);    // S = Q K^T
       const uint32_t idA = idesc_f16(128, 128, 0, 0);     // dA = dO V^T (fp16 copies)
       const uint32_t idQ = idesc_bf16(128, 64, 0, 1);     // dQ = dS K: A K-major (sdS), B MN-major (K_j)
-      const uint32_t kA = smem_u32(sK), vA = smem_u32(sV);
-      const uint32_t dH = smem_u32(sdS), dL = smem_u32(sdSl);
+      const uint64_t kK = sdesc_sw128(smem_u32(sK), 16, 1024), vK = sdesc_sw128(smem_u32(sV), 16, 1024);
+      const uint64_t kM = sdesc_sw128(smem_u32(sK), 8192, 1024);    // K_j as MN-major B (dQ)
+      const uint64_t rK = sdesc_sw128(smem_u32(ring), 16, 1024);    // ring stage 0, K-major
+      const uint64_t dHd = sdesc_sw128(smem_u32(sdS), 16, 1024), dLd = sdesc_sw128(smem_u32(sdSl), 16, 1024);
       mbar_wait(&sh.bar_kv, 0, status, abrt);
       // S = Q_s K^T and dA = dO_s V^T into TMEM [0,256).
       auto issue_sda = [&](int s) {
         const int st = s % kStages;
-        const uint32_t qA = smem_u32(ring + st * kPairBytes), oA = qA + kTileBytes;
+        const uint64_t qd = sdesc_add(rK, st * kPairBytes), od = sdesc_add(qd, kTileBytes);
         mbar_wait(&sh.full[st], (s / kStages) & 1, status, abrt);
         if (s > 0) mbar_wait(&sh.sda_free, (s - 1) & 1, status, abrt);   // S, dA of s-1 are in registers
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          mma_ss(T, sdesc_sw128(qA + k * 32, 16, 1024), sdesc_sw128(kA + k * 32, 16, 1024), idS, k > 0);
-          mma_ss(T + 128, sdesc_sw128(oA + k * 32, 16, 1024), sdesc_sw128(vA + k * 32, 16, 1024), idA, k > 0);
+          mma_ss(T, sdesc_add(qd, k * 32), sdesc_add(kK, k * 32), idS, k > 0);
+          mma_ss(T + 128, sdesc_add(od, k * 32), sdesc_add(vK, k * 32), idA, k > 0);
         }
         mma_commit(&sh.s_full);
       };
@@ -167,9 +169,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
         for (int t = 0; t < 8; ++t) {
           // dQ_s = dS K_j: K = keys (16 per step; panel t/4), M = queries.
           const uint32_t koff = (t >> 2) * kTileBytes + (t & 3) * 32;
-          const uint64_t bK = sdesc_sw128(kA + t * 2048, 8192, 1024);
-          mma_ss(dq, sdesc_sw128(dH + koff, 16, 1024), bK, idQ, t > 0 ? 1u : 0u);
-          mma_ss(dq, sdesc_sw128(dL + koff, 16, 1024), bK, idQ, 1u);
+          const uint64_t bK = sdesc_add(kM, t * 2048);
+          mma_ss(dq, sdesc_add(dHd, koff), bK, idQ, t > 0 ? 1u : 0u);
+          mma_ss(dq, sdesc_add(dLd, koff), bK, idQ, 1u);
         }
         mma_commit(&sh.empty[s % kStages]);   // S and dA of tile s were this warp's last reads
         mma_commit(&sh.mma2_done);
@@ -181,10 +183,12 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     if (lane == 0 && nq > 0) {
       const uint32_t idV = idesc_f16(128, 64, 1, 1);      // dV += A^T dO: A MN-major (sA), B MN-major
       const uint32_t idK = idesc_bf16(128, 64, 1, 1);     // dK += dS^T Q: A MN-major (sdS), B MN-major
-      const uint32_t aH = smem_u32(sA), dH = smem_u32(sdS), dL = smem_u32(sdSl);
+      const uint64_t aM = sdesc_sw128(smem_u32(sA), 16384, 1024);      // A, MN-major (dV)
+      const uint64_t dHM = sdesc_sw128(smem_u32(sdS), 16384, 1024), dLM = sdesc_sw128(smem_u32(sdSl), 16384, 1024);
+      const uint64_t rM = sdesc_sw128(smem_u32(ring), 8192, 1024);     // ring stage 0, MN-major
       for (int s = 0; s < nq; ++s) {
         const int st = s % kStages;
-        const uint32_t qA = smem_u32(ring + st * kPairBytes), oA = qA + kTileBytes;
+        const uint64_t qM = sdesc_add(rM, st * kPairBytes), oM = sdesc_add(qM, kTileBytes);
         mbar_wait(&sh.full[st], (s / kStages) & 1, status, abrt);   // Q_s and dO_s landed
         mbar_wait(&sh.p_ready, s & 1, status, abrt);                // A and dS of tile s written
         tc_fence_after();
@@ -192,10 +196,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
         for (int t = 0; t < 8; ++t) {
           // dV += A^T dO_s and dK += dS^T Q_s: K = queries (16 per step), M = keys.
           const uint32_t acc = (s > 0 || t > 0) ? 1u : 0u;
-          const uint64_t bO = sdesc_sw128(oA + t * 2048, 8192, 1024), bQ = sdesc_sw128(qA + t * 2048, 8192, 1024);
-          mma_ss(T + 256, sdesc_sw128(aH + t * 2048, 16384, 1024), bO, idV, acc);
-          mma_ss(T + 320, sdesc_sw128(dH + t * 2048, 16384, 1024), bQ, idK, acc);
-          mma_ss(T + 320, sdesc_sw128(dL + t * 2048, 16384, 1024), bQ, idK, 1u);
+          const uint64_t bO = sdesc_add(oM, t * 2048), bQ = sdesc_add(qM, t * 2048);
+          mma_ss(T + 256, sdesc_add(aM, t * 2048), bO, idV, acc);
+          mma_ss(T + 320, sdesc_add(dHM, t * 2048), bQ, idK, acc);
+          mma_ss(T + 320, sdesc_add(dLM, t * 2048), bQ, idK, 1u);
         }
         mma_commit(&sh.empty[st]);
         mma_commit(&sh.mma2_done);

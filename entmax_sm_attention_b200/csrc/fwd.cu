@@ -320,15 +320,15 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     uint32_t sfree_par = 0;      // per sweep S buffer: parity of its uses so far (bit b)
     uint32_t sbuf = 0;           // next sweep S buffer
     const uint32_t idS = idesc_bf16(128, 128, 0, 0);
-    const uint32_t sQa = smem_u32(sQ);
+    const uint64_t qd0 = sdesc_sw128(smem_u32(sQ), 16, 1024);      // Q tile, K-major
+    const uint64_t kd0 = sdesc_sw128(smem_u32(ring), 16, 1024);    // ring slot 0, K-major
     // S = Q K^T from ring position `pos` (already landed) into TMEM columns [dcol, dcol+128).
     auto mma_s = [&](uint32_t pos, uint32_t dcol) {
       const int slot = pos % kSlots;
       tc_fence_after();
-      const uint32_t kb = smem_u32(ring + slot * kTileBytes);
+      const uint64_t kd = sdesc_add(kd0, slot * kTileBytes);
 #pragma unroll
-      for (int k = 0; k < 4; ++k)
-        mma_ss(T + dcol, sdesc_sw128(sQa + k * 32, 16, 1024), sdesc_sw128(kb + k * 32, 16, 1024), idS, k > 0);
+      for (int k = 0; k < 4; ++k) mma_ss(T + dcol, sdesc_add(qd0, k * 32), sdesc_add(kd, k * 32), idS, k > 0);
       mma_commit(&sh.empty[slot]);   // a K slot is read by this issuer only: both arrivals here
       mma_commit(&sh.empty[slot]);
     };
@@ -386,6 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
   } else if (warp == kMma2Warp) {
     // ------------------------------------------------ second MMA issuer (output pass)
     const uint32_t idO = idesc_f16(128, 64, 0, 1);
+    const uint64_t vd0 = sdesc_sw128(smem_u32(ring), 8192, 1024);   // ring slot 0, MN-major
     uint32_t seq = 0;   // ring positions, tracked exactly like the producer's
     for_each_bit(act, kMaskWords, [&](int) { ++seq; });
     while (true) {
@@ -408,11 +409,11 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           const int vslot = vpos % kSlots;
           mbar_wait2(&sh.full[vslot], (vpos / kSlots) & 1, &sh.o_ready[c], (k / kOBufs) & 1, status, abrt);
           tc_fence_after();
-          const uint32_t vb = smem_u32(ring + vslot * kTileBytes);
+          const uint64_t vd = sdesc_add(vd0, vslot * kTileBytes);
 #pragma unroll
           for (int t = 0; t < 8; ++t) {
             const uint32_t col = pa + (t >> 2) * 64 + (t & 3) * 8 + 32;   // g block of the half
-            mma_ts(T + 320, T + col, sdesc_sw128(vb + t * 2048, 8192, 1024), idO, (k > 0 || t > 0) ? 1u : 0u);
+            mma_ts(T + 320, T + col, sdesc_add(vd, t * 2048), idO, (k > 0 || t > 0) ? 1u : 0u);
           }
           mma_commit(&sh.empty[vslot]);
           mma_commit(&sh.pv_done[c]);
@@ -424,6 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
   } else if (warp == kMma3Warp) {
     // ------------------------------------------------- third MMA issuer (output pass)
     const uint32_t idO = idesc_f16(128, 64, 0, 1);
+    const uint64_t vd0 = sdesc_sw128(smem_u32(ring), 8192, 1024);   // ring slot 0, MN-major
     uint32_t seq = 0;   // ring positions, tracked exactly like the producer's
     for_each_bit(act, kMaskWords, [&](int) { ++seq; });
     while (true) {
@@ -446,11 +448,11 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           const int vslot = vpos % kSlots;
           mbar_wait2(&sh.full[vslot], (vpos / kSlots) & 1, &sh.o_ready[c], (k / kOBufs) & 1, status, abrt);
           tc_fence_after();
-          const uint32_t vb = smem_u32(ring + vslot * kTileBytes);
+          const uint64_t vd = sdesc_add(vd0, vslot * kTileBytes);
 #pragma unroll
           for (int t = 0; t < 8; ++t) {
             const uint32_t col = pa + (t >> 2) * 64 + (t & 3) * 8;   // A block of the half
-            mma_ts(T + 256, T + col, sdesc_sw128(vb + t * 2048, 8192, 1024), idO, (k > 0 || t > 0) ? 1u : 0u);
+            mma_ts(T + 256, T + col, sdesc_add(vd, t * 2048), idO, (k > 0 || t > 0) ? 1u : 0u);
           }
           mma_commit(&sh.empty[vslot]);
           mma_commit(&sh.pv_done[c]);

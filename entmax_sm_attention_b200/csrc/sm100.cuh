@@ -186,6 +186,11 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
 }
 
 // Shared-memory matrix descriptor for a 128-byte-swizzled operand (version 1, sm_100).
+// Moves a shared-memory descriptor `bytes` forward (a multiple of 16). The start address
+// field holds (address >> 4) in 14 bits and every shared address is below 256 KB, so the
+// add never carries into the next field; this replaces rebuilding the descriptor.
+__device__ __forceinline__ uint64_t sdesc_add(uint64_t d, uint32_t bytes) { return d + (uint64_t)(bytes >> 4); }
+
 __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
   uint64_t d = 0;
   d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
