@@ -190,3 +190,12 @@ def test_planted_block_structure(alpha):
     st = g["stats"].reshape(-1, 4)
     sparsity = 1.0 - st[:, 2].sum() / st[:, 3].sum()
     assert sparsity > 0.5, sparsity
+
+
+def test_long_head_L12288():
+    """One long head (L = 12288, 96 key tiles; 48 KB of per-tile maxima in shared
+    memory), causal, alpha = 1.5, checked element by element."""
+    w = small_case("long_L12288", B=1, H=1, L=12288, causal=True, sigma_q=3.0)
+    rep = {}
+    compare(w, 1.5, backward=True, report=rep)
+    print(w.name, {k: (float(v) if not isinstance(v, int) else v) for k, v in rep.items()})
