@@ -12,8 +12,9 @@
 // One CTA per (batch*head, 128-key tile). K_j and V_j stay in shared memory; the
 // flagged query tiles stream through a 2-stage ring of (Q_i, dO_i). Per query tile the
 // tensor cores compute S = Q_i K_j^T and dA = dO_i V_j^T into TMEM (M = queries).
-// Warps 0-7 are row owners: warp w reads TMEM lanes 32(w%4)..+31 (one query row per
-// lane) and the columns of keys [64(w/4), 64(w/4)+64). Once a warp holds its S and dA
+// Warps 0-15 are row owners: warp w reads TMEM lanes 32(w%4)..+31 (one query row per
+// lane) and the columns of keys [32(w/4), 32(w/4)+32), so four threads share a row and
+// four warps share each SM sub-partition, which hides the latency of forming A and dS. Once a warp holds its S and dA
 // values in registers it releases them, so the MMA warp computes S and dA of the next
 // query tile while the row owners form A and dS. Both go to swizzled shared-memory
 // buffers: A in fp16 (with the fp16 copy of dO; 2^-11 rounding), dS as a two-term
@@ -24,8 +25,8 @@
 // fp16 copies of dO and V (exact conversions of the bf16 inputs). The row owners copy
 // dQ_i from TMEM into a swizzled fp32 staging tile in shared memory, and one thread adds
 // it to global dQ with a TMA reduce-add (cp.reduce.async.bulk.tensor .add), one query
-// tile behind the MMAs. Warp 8 issues the TMA loads. Warp 9 issues S, dA and the dQ chain,
-// warp 10 the dV and dK chains: one thread issues an N=64 MMA only every ~54 cycles, so
+// tile behind the MMAs. Warp 16 issues the TMA loads. Warp 17 issues S, dA and the dQ chain,
+// warp 18 the dV and dK chains: one thread issues an N=64 MMA only every ~54 cycles, so
 // the 40 MMAs of a tile's gradient products are split between two issuers.
 // TMEM: [0,128) S, [128,256) dA, [256,320) dV, [320,384) dK, [384,512) dQ x2.
 #include "common.cuh"
@@ -35,10 +36,11 @@ namespace entmax {
 
 namespace {
 
-constexpr int kThreads = 352;
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;    // S, dA and the dQ chain
-constexpr int kMma2Warp = 10;  // the dV and dK chains
+constexpr int kMathWarps = 16;   // row owners: 4 per TMEM lane quadrant, 32 keys each
+constexpr int kThreads = (kMathWarps + 3) * 32;
+constexpr int kProducerWarp = kMathWarps;
+constexpr int kMmaWarp = kMathWarps + 1;    // S, dA and the dQ chain
+constexpr int kMma2Warp = kMathWarps + 2;   // the dV and dK chains
 constexpr int kStages = 2;
 constexpr int kPairBytes = 2 * kTileBytes;   // Q_i and dO_i
 
@@ -77,7 +79,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bh = blockIdx.x % p.BH;
   const int kt = blockIdx.x / p.BH;          // key tile (low key tiles have the most query tiles)
-  const int kMathThreads = 256;
+  constexpr int kMathThreads = kMathWarps * 32;
   const int b = bh / p.H;
   const Pattern pat{p.L, p.kv_len ? min(max(p.kv_len[b], 1), p.L) : p.L, p.causal, p.window};
   const int j0 = kt * kTile;
@@ -91,8 +93,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     }
     mbar_init(&sh.bar_kv, 1);
     mbar_init(&sh.s_full, 1);
-    mbar_init(&sh.sda_free, 8);
-    mbar_init(&sh.p_ready, 8);
+    mbar_init(&sh.sda_free, kMathWarps);
+    mbar_init(&sh.p_ready, kMathWarps);
     mbar_init(&sh.mma2_done, 2);  // dQ chain and dV/dK chains
     sh.abort_flag = 0;
     fence_mbar_init();
@@ -208,7 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- row owners
-    const int quad = warp & 3, hf = warp >> 2;   // TMEM lane quadrant, key half
+    const int quad = warp & 3, qc = warp >> 2;   // TMEM lane quadrant, key quarter
     const int row = quad * 32 + lane;
     const uint32_t tl = T + ((uint32_t)(quad * 32) << 16);
     const float cz = p.cz;
@@ -216,23 +218,25 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     int prev_it = -1;
     // Adds dQ of the query tile `it` handled at step `s` (TMEM buffer s % 2) to global
     // memory. The caller has already waited for that step's MMAs. Each thread stages its
-    // 32 columns (scaled) in the swizzled box of its column half; then thread 0 issues
+    // 16 columns (scaled) in the swizzled box of its column half; then thread 0 issues
     // one TMA reduce-add per box. The staging buffer is reused only after the previous
     // reduce-adds have read it.
     auto flush_dq = [&](uint32_t s, int it) {
       if (tid == 0) bulk_wait_read_all();
       named_bar(1, kMathThreads);
       tc_fence_after();
-      uint32_t a[32];
-      tmem_ld32(tl + 384 + (s & 1) * 64 + hf * 32, a);
+      uint32_t a[16];
+      tmem_ld16(tl + 384 + (s & 1) * 64 + qc * 16, a);
       tmem_wait_ld();
-      uint8_t* box = sStage + hf * kTileBytes + row * 128;
+      uint8_t* box = sStage + (qc >> 1) * kTileBytes + row * 128;
       const float sc = p.scale;
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<float4*>(box + ((c ^ (row & 7)) << 4)) =
+      for (int c = 0; c < 4; ++c) {
+        const int ch = (qc & 1) * 4 + c;
+        *reinterpret_cast<float4*>(box + ((ch ^ (row & 7)) << 4)) =
             make_float4(sc * __uint_as_float(a[4 * c]), sc * __uint_as_float(a[4 * c + 1]),
                         sc * __uint_as_float(a[4 * c + 2]), sc * __uint_as_float(a[4 * c + 3]));
+      }
       fence_proxy_async_smem();
       named_bar(1, kMathThreads);
       if (tid == 0) {
@@ -249,27 +253,25 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       const bool full = pat.block_full(it * kTile, min(p.L, it * kTile + kTile), j0, j0 + kTile);
       warp_wait(&sh.s_full, seq & 1, status, abrt);
       tc_fence_after();
-      uint32_t sr[64], ar[64];
-      tmem_ld32(tl + hf * 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-      tmem_ld32(tl + hf * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-      tmem_ld32(tl + 128 + hf * 64, *reinterpret_cast<uint32_t(*)[32]>(&ar[0]));
-      tmem_ld32(tl + 128 + hf * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&ar[32]));
+      uint32_t sr[32], ar[32];
+      tmem_ld32(tl + qc * 32, sr);
+      tmem_ld32(tl + 128 + qc * 32, ar);
       tmem_wait_ld();
       tc_fence_before();
       warp_arrive(&sh.sda_free);
       // The previous tile's dV/dK/dQ MMAs must be done reading sA / sdS.
       if (seq > 0) warp_wait(&sh.mma2_done, (seq - 1) & 1, status, abrt);
-      // Keys [64 hf, 64 hf + 64) of row `row`: panel hf, 16-byte chunks 0..7.
-      const int pan = hf * kTileBytes;
+      // Keys [32 qc, 32 qc + 32) of row `row`: panel qc/2, 16-byte chunks 4(qc%2)..+3.
+      const int pan = (qc >> 1) * kTileBytes;
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
+      for (int cc = 0; cc < 4; ++cc) {
         uint32_t ah[4], dh[4], dl2[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int c = ch * 8 + 2 * e;
+          const int c = cc * 8 + 2 * e;
           float s0 = __uint_as_float(sr[c]), s1 = __uint_as_float(sr[c + 1]);
           if (!full) {
-            const int jj = j0 + hf * 64 + c;
+            const int jj = j0 + qc * 32 + c;
             if (!pat.active(i, jj)) s0 = -INFINITY;
             if (!pat.active(i, jj + 1)) s1 = -INFINITY;
           }
@@ -286,7 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
             split_bf16x2(u.x > 0.f ? d0 : 0.f, u.y > 0.f ? d1 : 0.f, dh[e], dl2[e]);
           }
         }
-        const uint32_t off = pan + sw128_offset(row, ch * 8);
+        const uint32_t off = pan + sw128_offset(row, ((qc & 1) * 4 + cc) * 8);
         *reinterpret_cast<uint4*>(sA + off) = make_uint4(ah[0], ah[1], ah[2], ah[3]);
         *reinterpret_cast<uint4*>(sdS + off) = make_uint4(dh[0], dh[1], dh[2], dh[3]);
         *reinterpret_cast<uint4*>(sdSl + off) = make_uint4(dl2[0], dl2[1], dl2[2], dl2[3]);
@@ -302,27 +304,27 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       flush_dq(seq - 1, prev_it);
     }
     if (tid == 0) bulk_wait_all();   // the last reduce-adds complete before the CTA retires
-    // dK and dV of this key tile (TMEM lane = key); each thread writes 32 of the 64
-    // columns. Every lane executes the TMEM loads (.sync.aligned); only the global stores
-    // depend on the key being inside L.
+    // dK and dV of this key tile (TMEM lane = key); each thread writes 16 of the 64
+    // columns of each. Every lane executes the TMEM loads (.sync.aligned); only the global
+    // stores depend on the key being inside L.
     const int j = j0 + row;
     const bool jvalid = j < p.L;
-    float* dk = p.dK + ((size_t)bh * p.L + (jvalid ? j : 0)) * kD + hf * 32;
-    float* dv = p.dV + ((size_t)bh * p.L + (jvalid ? j : 0)) * kD + hf * 32;
+    float* dk = p.dK + ((size_t)bh * p.L + (jvalid ? j : 0)) * kD + qc * 16;
+    float* dv = p.dV + ((size_t)bh * p.L + (jvalid ? j : 0)) * kD + qc * 16;
     const float sc = p.scale;
-    uint32_t a[32], c[32];
+    uint32_t a[16], c[16];
     if (seq > 0) {
       tc_fence_after();
-      tmem_ld32(tl + 256 + hf * 32, a);
-      tmem_ld32(tl + 320 + hf * 32, c);
+      tmem_ld16(tl + 256 + qc * 16, a);
+      tmem_ld16(tl + 320 + qc * 16, c);
       tmem_wait_ld();
     } else {
 #pragma unroll
-      for (int k = 0; k < 32; ++k) a[k] = c[k] = 0u;
+      for (int k = 0; k < 16; ++k) a[k] = c[k] = 0u;
     }
     if (jvalid) {
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
+      for (int k = 0; k < 4; ++k) {
         reinterpret_cast<float4*>(dv)[k] = make_float4(__uint_as_float(a[4 * k]), __uint_as_float(a[4 * k + 1]),
                                                        __uint_as_float(a[4 * k + 2]), __uint_as_float(a[4 * k + 3]));
         reinterpret_cast<float4*>(dk)[k] =
