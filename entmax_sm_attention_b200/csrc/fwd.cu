@@ -31,19 +31,20 @@
 //     tolerances once g reaches dK through delta. sum_j g_ij is kept per row for the
 //     backward.
 //
-// Roles (384 threads): warps 0-7 are row owners. Warp w reads TMEM lanes 32(w%4)..+31
-// (one query row per lane) and columns [64(w/4), 64(w/4)+64) of every S tile, so two
-// threads share a row and combine partial sums in shared memory. Warp 8 issues TMA
-// loads into a 4-slot ring of 16 KB K/V tiles. Warp 9 owns TMEM and issues the S = Q K^T
-// MMAs of every phase; in the output pass warp 11 issues the O = A V chain and warp 10
+// Roles (640 threads): warps 0-15 are row owners. Warp w reads TMEM lanes 32(w%4)..+31
+// (one query row per lane) and columns [32(w/4), 32(w/4)+32) of every S tile, so four
+// threads share a row and combine partial sums in shared memory; four warps per SM
+// sub-partition hide the latency of the per-score work. Warp 16 issues TMA
+// loads into a 4-slot ring of 16 KB K/V tiles. Warp 17 owns TMEM and issues the S = Q K^T
+// MMAs of every phase; in the output pass warp 19 issues the O = A V chain and warp 18
 // the Ot = g V chain. One thread issues an N=64 MMA only every ~54 cycles and each
 // mbarrier wait costs ~200 cycles even when the phase is complete, so one issuer per
 // chain keeps each below the tile's tensor time.
 // TMEM (512 columns): during the sweeps, four S buffers at 0/128/256/384, so the MMA
 // warp runs up to three tiles ahead. During the output pass:
-//   - three S buffers at 0, 128 and 384 (tile k in buffer k % 3). The thread owning key
-//     half h overwrites its 64 S columns [64h, 64h+64) with A (fp16 pairs) at 64h and
-//     g at 64h + 32;
+//   - three S buffers at 0, 128 and 384 (tile k in buffer k % 3). The row owner of keys
+//     [32q, 32q+32) writes their A (fp16 pairs) into columns [32q, 32q+16) and g into
+//     [32q+16, 32q+32): only over S columns it has read itself;
 //   - O at [256,320) and Ot at [320,384).
 #include "common.cuh"
 #include "kernels.h"
@@ -52,16 +53,20 @@ namespace entmax {
 
 namespace {
 
-constexpr int kThreads = 384;
-constexpr int kMathThreads = 256;
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
-constexpr int kMma2Warp = 10;   // second MMA issuer: the Ot = g V chain of the output pass
-constexpr int kMma3Warp = 11;   // third MMA issuer: the O = A V chain of the output pass
+constexpr int kMathWarps = 16;                // row owners: kParts per TMEM lane quadrant
+constexpr int kParts = kMathWarps / 4;        // threads per query row
+constexpr int kCols = kTile / kParts;         // key columns per thread
+constexpr int kOCols = kD / kParts;           // output columns per thread in the epilogue
+constexpr int kThreads = (kMathWarps + 4) * 32;
+constexpr int kMathThreads = kMathWarps * 32;
+constexpr int kProducerWarp = kMathWarps;
+constexpr int kMmaWarp = kMathWarps + 1;
+constexpr int kMma2Warp = kMathWarps + 2;     // second MMA issuer: the Ot = g V chain of the output pass
+constexpr int kMma3Warp = kMathWarps + 3;     // third MMA issuer: the O = A V chain of the output pass
 constexpr int kOBufs = 3;       // S/A buffers in the output pass (TMEM columns 0, 128, 384)
 constexpr int kSlots = 4;
 constexpr int kSBufs = 4;
-constexpr int kCandPerThread = 64;     // candidates per (row, column half); 128 per row
+constexpr int kCandPerThread = kTile / kParts;   // candidates per (row, column part); 128 per row
 constexpr float kTolF = 3e-5f;         // |f(tau)| = |sum p - 1| small enough to stop sweeping
 constexpr int kMaxVotes = 72;
 
@@ -92,8 +97,12 @@ __device__ __forceinline__ int f2ord(float f) {
 }
 __device__ __forceinline__ float ord2f(int i) { return __int_as_float(i >= 0 ? i : i ^ 0x7fffffff); }
 
+// Load kCols consecutive fp32 TMEM columns of this thread's lane.
+template <int N>
+__device__ __forceinline__ void ldc(uint32_t taddr, float (&s)[N]);
+
 // Load 64 consecutive fp32 TMEM columns of this thread's lane.
-__device__ __forceinline__ void ld64(uint32_t taddr, float (&s)[64]) {
+[[maybe_unused]] __device__ __forceinline__ void ld64(uint32_t taddr, float (&s)[64]) {
   uint32_t a[32], b[32];
   tmem_ld32(taddr, a);
   tmem_ld32(taddr + 32, b);
@@ -103,6 +112,32 @@ __device__ __forceinline__ void ld64(uint32_t taddr, float (&s)[64]) {
     s[c] = __uint_as_float(a[c]);
     s[32 + c] = __uint_as_float(b[c]);
   }
+}
+
+template <int N>
+__device__ __forceinline__ void ldc(uint32_t taddr, float (&s)[N]) {
+  if constexpr (N == 64) {
+    ld64(taddr, s);
+  } else {
+    static_assert(N == 32, "32 or 64 columns per thread");
+    uint32_t a[32];
+    tmem_ld32(taddr, a);
+    tmem_wait_ld();
+#pragma unroll
+    for (int c = 0; c < 32; ++c) s[c] = __uint_as_float(a[c]);
+  }
+}
+
+// Loads kOCols fp32 TMEM columns (16 or 32) as raw words.
+template <int N>
+__device__ __forceinline__ void ldw(uint32_t taddr, uint32_t (&o)[N]) {
+  if constexpr (N == 32) {
+    tmem_ld32(taddr, o);
+  } else {
+    static_assert(N == 16, "16 or 32 columns per thread");
+    tmem_ld16(taddr, o);
+  }
+  tmem_wait_ld();
 }
 
 // Adds one candidate at u = z - t to the sums of the current support (u > 0), without
@@ -134,17 +169,17 @@ __device__ __forceinline__ void sum_list(const float* list, int n, int stride, f
   umin = fminf(umin, fminf(fminf(am[0], am[1]), fminf(am[2], am[3])));
 }
 
-// Safeguarded solve of Eq. 4 for one row over raw scores vals0[k*stride] (k < n0) and
-// vals1[k*stride] (k < n1), which must hold every score that can be in the support.
+// Safeguarded solve of Eq. 4 for one row over raw scores vals[q*list_stride + k*stride]
+// (q < kParts, k < n[q]), which must hold every score that can be in the support.
 // u = fma(s, cz, -t). Starts at t (a lower bound) inside [lo, hi]; on success returns
 // true with the exact root up to fp32 rounding.
 template <int AK>
-__device__ bool solve_list(const float* vals0, int n0, const float* vals1, int n1, int stride, float cz, float t,
-                           float lo, float hi, float& t_out) {
+__device__ bool solve_list(const float* vals, const int (&n)[kParts], int list_stride, int stride, float cz,
+                           float t, float lo, float hi, float& t_out) {
   for (int it = 0; it < 48; ++it) {
     float S1 = 0.f, S2 = 0.f, C = 0.f, umin = INFINITY;
-    sum_list(vals0, n0, stride, cz, t, S1, S2, C, umin);
-    sum_list(vals1, n1, stride, cz, t, S1, S2, C, umin);
+#pragma unroll
+    for (int q = 0; q < kParts; ++q) sum_list(vals + q * list_stride, n[q], stride, cz, t, S1, S2, C, umin);
     const float f = (AK == kAlpha15) ? S2 - 1.f : S1 - 1.f;
     const float fp = (AK == kAlpha15) ? 2.f * S1 : C;   // |f'(t)|
     if (C > 0.f) {
@@ -173,17 +208,17 @@ __device__ bool solve_list(const float* vals0, int n0, const float* vals1, int n
   return false;
 }
 
-// Threshold of Eq. 4 restricted to eight raw scores v (some may be -inf), in registers:
+// Threshold of Eq. 4 restricted to N raw scores v (some may be -inf), in registers:
 // safeguarded Newton from lo inside [lo, hi], finished by the exact root of the current
 // support's piece once no value leaves the support. A subset of the row's scores has a
 // threshold at or below the row's tau*, so the result is a lower bound on tau*.
-template <int AK>
-__device__ __forceinline__ float solve8(const float (&v)[8], float cz, float lo, float hi) {
+template <int AK, int N>
+__device__ __forceinline__ float solveN(const float (&v)[N], float cz, float lo, float hi) {
   float t = lo;
   for (int it = 0; it < 24; ++it) {
     float S1 = 0.f, S2 = 0.f, C = 0.f, umin = INFINITY;
 #pragma unroll
-    for (int q = 0; q < 8; ++q) accumulate(fmaf(v[q], cz, -t), S1, S2, C, umin);
+    for (int q = 0; q < N; ++q) accumulate(fmaf(v[q], cz, -t), S1, S2, C, umin);
     const float f = (AK == kAlpha15) ? S2 - 1.f : S1 - 1.f;
     const float fp = (AK == kAlpha15) ? 2.f * S1 : C;
     if (C > 0.f) {
@@ -215,8 +250,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
   uint8_t* sQ = dsm;
   uint8_t* ring = dsm + kTileBytes;
   int* tmax = reinterpret_cast<int*>(dsm + kTileBytes * (1 + kSlots));   // [Tc][128], f2ord
-  float* cand = reinterpret_cast<float*>(tmax + p.Tc * kTile);           // [2 halves][32][128]
-  float* part = cand + 2 * kCandPerThread * kTile;                       // [2 halves][4][128]
+  float* cand = reinterpret_cast<float*>(tmax + p.Tc * kTile);   // [kParts][kCandPerThread][128]
+  float* part = cand + kParts * kCandPerThread * kTile;          // [kParts][4][128]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bh = blockIdx.x % p.BH;
@@ -235,11 +270,11 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     mbar_init(&sh.bar_q, 1);
     for (int s = 0; s < kSBufs; ++s) {
       mbar_init(&sh.s_full[s], 1);
-      mbar_init(&sh.s_free[s], 8);
+      mbar_init(&sh.s_free[s], kMathWarps);
     }
     for (int s = 0; s < kOBufs; ++s) {
       mbar_init(&sh.o_full[s], 1);
-      mbar_init(&sh.o_ready[s], 8);
+      mbar_init(&sh.o_ready[s], kMathWarps);
       mbar_init(&sh.pv_done[s], 2);   // O chain and Ot chain
     }
     sh.abort_flag = 0;
@@ -412,7 +447,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           const uint64_t vd = sdesc_add(vd0, vslot * kTileBytes);
 #pragma unroll
           for (int t = 0; t < 8; ++t) {
-            const uint32_t col = pa + (t >> 2) * 64 + (t & 3) * 8 + 32;   // g block of the half
+            // keys 16t..16t+15: part 16t / kCols, pair columns ((16t) % kCols) / 2 of its A block
+            const uint32_t col = pa + (16 * t / kCols) * kCols + ((16 * t) % kCols) / 2 + kCols / 2;   // g block
             mma_ts(T + 320, T + col, sdesc_add(vd, t * 2048), idO, (k > 0 || t > 0) ? 1u : 0u);
           }
           mma_commit(&sh.empty[vslot]);
@@ -451,7 +487,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           const uint64_t vd = sdesc_add(vd0, vslot * kTileBytes);
 #pragma unroll
           for (int t = 0; t < 8; ++t) {
-            const uint32_t col = pa + (t >> 2) * 64 + (t & 3) * 8;   // A block of the half
+            // keys 16t..16t+15: part 16t / kCols, pair columns ((16t) % kCols) / 2 of its A block
+            const uint32_t col = pa + (16 * t / kCols) * kCols + ((16 * t) % kCols) / 2;   // A block
             mma_ts(T + 256, T + col, sdesc_add(vd, t * 2048), idO, (k > 0 || t > 0) ? 1u : 0u);
           }
           mma_commit(&sh.empty[vslot]);
@@ -463,7 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     }
   } else {
     // ---------------------------------------------------------------- row owners
-    const int quad = warp & 3, hf = warp >> 2;   // TMEM lane quadrant, column half
+    const int quad = warp & 3, qp = warp >> 2;   // TMEM lane quadrant, column part
     const int row = quad * 32 + lane;
     const int i = i0 + row;
     const bool valid = i < p.L;
@@ -479,25 +516,25 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       warp_wait(&sh.s_full[bf], (sfull_par >> bf) & 1, status, abrt);
       sfull_par ^= 1u << bf;
       tc_fence_after();
-      const int j0 = jt * kTile + hf * 64;
-      float s[64];
-      ld64(tl + bf * 128 + hf * 64, s);
+      const int j0 = jt * kTile + qp * kCols;
+      float s[kCols];
+      ldc(tl + bf * 128 + qp * kCols, s);
       tc_fence_before();
       warp_arrive(&sh.s_free[bf]);
       if (!pat.block_full(i0, i1, jt * kTile, jt * kTile + kTile)) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c)
+        for (int c = 0; c < kCols; ++c)
           if (!pat.active(i, j0 + c)) s[c] = -INFINITY;
       }
       float t8[8];   // eight independent max chains
 #pragma unroll
       for (int c = 0; c < 8; ++c) t8[c] = s[c];
 #pragma unroll
-      for (int c = 8; c < 64; ++c) t8[c & 7] = fmaxf(t8[c & 7], s[c]);
+      for (int c = 8; c < kCols; ++c) t8[c & 7] = fmaxf(t8[c & 7], s[c]);
       const float tm = fmaxf(fmaxf(fmaxf(t8[0], t8[1]), fmaxf(t8[2], t8[3])),
                              fmaxf(fmaxf(t8[4], t8[5]), fmaxf(t8[6], t8[7])));
       atomicMax(&tmax[jt * kTile + row], f2ord(tm));
-      // Keep the four largest half-tile maxima, sorted (compare-exchange, no branch).
+      // Keep the four largest part-tile maxima, sorted (compare-exchange, no branch).
       float x = tm;
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
@@ -507,18 +544,19 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       }
       sbuf = (sbuf + 1) & (kSBufs - 1);
     });
-    // Both column halves' four largest half-tile maxima: the row max and the values of
-    // the initial threshold.
+    // All column parts' four largest part-tile maxima: the row max and the values of the
+    // initial threshold.
 #pragma unroll
-    for (int k = 0; k < 4; ++k) part[(hf * 4 + k) * kTile + row] = top[k];
+    for (int k = 0; k < 4; ++k) part[(qp * 4 + k) * kTile + row] = top[k];
     named_bar(3, kMathThreads);
-    float v8[8];
+    float vt[4 * kParts];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) v8[k] = part[k * kTile + row];
+    for (int k = 0; k < 4 * kParts; ++k) vt[k] = part[k * kTile + row];
     named_bar(3, kMathThreads);   // read before anyone rewrites the partials
-    m = fmaxf(v8[0], v8[4]);
+#pragma unroll
+    for (int q = 0; q < kParts; ++q) m = fmaxf(m, vt[4 * q]);
 
-    // Bracket (§2.4) and the tile-maxima lower bound (identical in both threads of a row).
+    // Bracket (§2.4) and the tile-maxima lower bound (identical in all threads of a row).
     const int n_act = valid ? pat.count(i) : 1;
     const float mz = m * cz;
     float lo = mz - 1.f;
@@ -526,9 +564,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     float tau = INFINITY;
     bool done = !valid;
     if (valid) {
-      // The eight largest half-tile maxima of the row are a subset of its scores, so the
-      // threshold of entmax on them is a lower bound tau_T <= tau*.
-      const float t = solve8<AK>(v8, cz, lo, hi);
+      // The row's largest part-tile maxima are a subset of its scores, so the threshold
+      // of entmax on them is a lower bound tau_T <= tau*.
+      const float t = solveN<AK, 4 * kParts>(vt, cz, lo, hi);
       tau = fminf(fmaxf(t, lo), hi);
     }
     float2 sg2 = make_float2(0.f, 0.f);   // sum_j g_ij, two chains
@@ -541,7 +579,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       const int buf = r & 1;
       const bool need = !done && sweeps < p.max_sweeps;
       const bool final_mask = !rows_any(need, sh.votes, r, lane, kMathThreads);
-      if (hf == 0) {
+      if (qp == 0) {
         // Tiles that some row still needs (refinement) or that hold a nonzero (mask): each
         // warp builds a word of 32 tile bits from eight independent loads and votes per
         // step, and ORs it into the list once.
@@ -575,7 +613,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       named_bar(1, kThreads);
 
       if (final_mask) {
-        if (!done && hf == 0) atomicOr(status, kStatusNoConverge);   // cap reached; tau stays bracketed
+        if (!done && qp == 0) atomicOr(status, kStatusNoConverge);   // cap reached; tau stays bracketed
         // Block mask row of this query tile and the transposed bits (Appendix C.4).
         if (tid < p.Wc) p.M[((size_t)bh * p.Tr + qt) * p.Wc + tid] = list[tid];
         if (tid == 0) {
@@ -590,17 +628,17 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           const uint32_t pa = c == 0 ? 0u : (c == 1 ? 128u : 384u);
           warp_wait(&sh.o_full[c], (k / kOBufs) & 1, status, abrt);
           tc_fence_after();
-          const int j0 = jt * kTile + hf * 64;
-          float s[64];
-          ld64(tl + pa + hf * 64, s);
+          const int j0 = jt * kTile + qp * kCols;
+          float s[kCols];
+          ldc(tl + pa + qp * kCols, s);
           if (!pat.block_full(i0, i1, jt * kTile, jt * kTile + kTile)) {
 #pragma unroll
-            for (int cc = 0; cc < 64; ++cc)
+            for (int cc = 0; cc < kCols; ++cc)
               if (!pat.active(i, j0 + cc)) s[cc] = -INFINITY;
           }
-          uint32_t aw[32], gw[32];
+          uint32_t aw[kCols / 2], gw[kCols / 2];
 #pragma unroll
-          for (int cc = 0; cc < 32; ++cc) {
+          for (int cc = 0; cc < kCols / 2; ++cc) {
             const float2 u = __ffma2_rn(make_float2(s[2 * cc], s[2 * cc + 1]), make_float2(cz, cz),
                                         make_float2(-tau, -tau));
             const float v0 = fmaxf(u.x, 0.f), v1 = fmaxf(u.y, 0.f);
@@ -616,11 +654,15 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
               sg2 = __fadd2_rn(sg2, make_float2(g0, g1));
             }
           }
-          const uint32_t col = pa + hf * 64;
-          tmem_st16(tl + col, *reinterpret_cast<uint32_t(*)[16]>(&aw[0]));
-          tmem_st16(tl + col + 16, *reinterpret_cast<uint32_t(*)[16]>(&aw[16]));
-          tmem_st16(tl + col + 32, *reinterpret_cast<uint32_t(*)[16]>(&gw[0]));
-          tmem_st16(tl + col + 48, *reinterpret_cast<uint32_t(*)[16]>(&gw[16]));
+          // This part's keys qp*kCols.. go back into its own S columns [qp*kCols, +kCols):
+          // A (fp16 pairs) in the first half, g in the second. Writing only into columns this
+          // thread has read keeps the row's other parts from seeing overwritten S values.
+          const uint32_t col = pa + qp * kCols;
+#pragma unroll
+          for (int h = 0; h < kCols / 32; ++h) {
+            tmem_st16(tl + col + 16 * h, *reinterpret_cast<uint32_t(*)[16]>(&aw[16 * h]));
+            tmem_st16(tl + col + kCols / 2 + 16 * h, *reinterpret_cast<uint32_t(*)[16]>(&gw[16 * h]));
+          }
           tmem_wait_st();
           tc_fence_before();
           warp_arrive(&sh.o_ready[c]);
@@ -628,34 +670,35 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           ++n_s;
         });
         const int n_out = k;
-        // Epilogue: O and Ot from TMEM (each thread of a row writes 32 of the 64 columns).
+        // Epilogue: O and Ot from TMEM (each thread of a row writes kOCols of the 64 columns).
         warp_wait(&sh.pv_done[(n_out - 1) % kOBufs], ((n_out - 1) / kOBufs) & 1, status, abrt);
         tc_fence_after();
-        part[(hf * 4 + 1) * kTile + row] = sg2.x + sg2.y;
-        uint32_t o[32];
-        tmem_ld32(tl + 256 + hf * 32, o);
-        tmem_wait_ld();
+        part[(qp * 4 + 1) * kTile + row] = sg2.x + sg2.y;
+        uint32_t o[kOCols];
+        ldw(tl + 256 + qp * kOCols, o);
         if (valid) {
-          float4* dst = reinterpret_cast<float4*>(p.O + ((size_t)bh * p.L + i) * kD + hf * 32);
+          float4* dst = reinterpret_cast<float4*>(p.O + ((size_t)bh * p.L + i) * kD + qp * kOCols);
 #pragma unroll
-          for (int cc = 0; cc < 8; ++cc)
+          for (int cc = 0; cc < kOCols / 4; ++cc)
             dst[cc] = make_float4(__uint_as_float(o[4 * cc]), __uint_as_float(o[4 * cc + 1]),
                                   __uint_as_float(o[4 * cc + 2]), __uint_as_float(o[4 * cc + 3]));
         }
         __syncwarp();
-        tmem_ld32(tl + 320 + hf * 32, o);
-        tmem_wait_ld();
+        ldw(tl + 320 + qp * kOCols, o);
         if (valid) {
-          float4* dst = reinterpret_cast<float4*>(p.Ot + ((size_t)bh * p.L + i) * kD + hf * 32);
+          float4* dst = reinterpret_cast<float4*>(p.Ot + ((size_t)bh * p.L + i) * kD + qp * kOCols);
 #pragma unroll
-          for (int cc = 0; cc < 8; ++cc)
+          for (int cc = 0; cc < kOCols / 4; ++cc)
             dst[cc] = make_float4(__uint_as_float(o[4 * cc]), __uint_as_float(o[4 * cc + 1]),
                                   __uint_as_float(o[4 * cc + 2]), __uint_as_float(o[4 * cc + 3]));
         }
         named_bar(3, kMathThreads);
-        if (valid && hf == 0) {
+        if (valid && qp == 0) {
+          float sg = 0.f;
+#pragma unroll
+          for (int q = 0; q < kParts; ++q) sg += part[(q * 4 + 1) * kTile + row];
           p.tau[(size_t)bh * p.L + i] = tau;
-          p.sumg[(size_t)bh * p.L + i] = part[1 * kTile + row] + part[5 * kTile + row];
+          p.sumg[(size_t)bh * p.L + i] = sg;
         }
         if (tid == 0) {
           int na = 0;
@@ -670,21 +713,21 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       // thread's candidates u > 0: when tau <= tau* (f >= 0) they hold the whole support.
       float S1 = 0.f, S2 = 0.f;
       int nc = 0;
-      float* mycand = cand + hf * kCandPerThread * kTile + row;
+      float* mycand = cand + qp * kCandPerThread * kTile + row;
       sbuf = 0;
       for_each_bit(list, kMaskWords, [&](int jt) {
         const uint32_t bf = sbuf;
         warp_wait(&sh.s_full[bf], (sfull_par >> bf) & 1, status, abrt);
         sfull_par ^= 1u << bf;
         tc_fence_after();
-        const int j0 = jt * kTile + hf * 64;
-        float s[64];
-        ld64(tl + bf * 128 + hf * 64, s);
+        const int j0 = jt * kTile + qp * kCols;
+        float s[kCols];
+        ldc(tl + bf * 128 + qp * kCols, s);
         tc_fence_before();
         warp_arrive(&sh.s_free[bf]);
         if (!pat.block_full(i0, i1, jt * kTile, jt * kTile + kTile)) {
 #pragma unroll
-          for (int cc = 0; cc < 64; ++cc)
+          for (int cc = 0; cc < kCols; ++cc)
             if (!pat.active(i, j0 + cc)) s[cc] = -INFINITY;
         }
         float2 s1[4], s2[4];
@@ -693,12 +736,12 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           s1[a] = make_float2(0.f, 0.f);
           s2[a] = make_float2(0.f, 0.f);
         }
-        // Groups of 8 scores: u+ summed per group (feeds S1), straight-line for all eight
-        // groups; then only the groups with a positive sum (rare: a support candidate) are
-        // scanned element by element.
+        // Groups of 8 scores: u+ summed per group (feeds S1), straight-line for all groups;
+        // then only the groups with a positive sum (rare: a support candidate) are scanned
+        // element by element.
         uint32_t gmask = 0;
 #pragma unroll
-        for (int g = 0; g < 8; ++g) {
+        for (int g = 0; g < kCols / 8; ++g) {
           float2 v[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -713,7 +756,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         }
         if (gmask) {
 #pragma unroll
-          for (int g = 0; g < 8; ++g) {
+          for (int g = 0; g < kCols / 8; ++g) {
             if ((gmask >> g) & 1u) {
 #pragma unroll
               for (int e = 0; e < 8; ++e) {
@@ -732,30 +775,38 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         ++n_s;
         sbuf = (sbuf + 1) & (kSBufs - 1);
       });
-      // Combine the two column halves of each row.
-      float* mp = part + hf * 4 * kTile + row;
+      // Combine the column parts of each row.
+      float* mp = part + qp * 4 * kTile + row;
       mp[0] = S1;
       mp[kTile] = S2;
       mp[2 * kTile] = (float)nc;
       named_bar(3, kMathThreads);
-      const float* p0 = part + row;
-      const float* p1 = part + 4 * kTile + row;
-      S1 = p0[0] + p1[0];
-      S2 = p0[kTile] + p1[kTile];
-      const int nc0 = (int)p0[2 * kTile], nc1 = (int)p1[2 * kTile];
-      const float C = (float)(nc0 + nc1);   // support size at tau (alpha = 2: |f'(tau)|)
+      S1 = 0.f;
+      S2 = 0.f;
+      int ncs[kParts];
+      int ntot = 0;
+      bool fits = true;
+#pragma unroll
+      for (int q = 0; q < kParts; ++q) {
+        const float* pq = part + q * 4 * kTile + row;
+        S1 += pq[0];
+        S2 += pq[kTile];
+        ncs[q] = (int)pq[2 * kTile];
+        ntot += ncs[q];
+        fits = fits && ncs[q] <= kCandPerThread;
+      }
+      const float C = (float)ntot;   // support size at tau (alpha = 2: |f'(tau)|)
       named_bar(3, kMathThreads);   // partials consumed before anyone rewrites them
       ++sweeps;
       if (!done) {
         const float f = (AK == kAlpha15) ? S2 - 1.f : S1 - 1.f;
         const float fp = (AK == kAlpha15) ? 2.f * S1 : C;   // |f'(tau)|
         if (f > 0.f) lo = fmaxf(lo, tau); else hi = fminf(hi, tau);
-        if (f >= 0.f && nc0 <= kCandPerThread && nc1 <= kCandPerThread) {
-          // tau <= tau*, so every score of the support is in the two candidate lists: the
+        if (f >= 0.f && fits) {
+          // tau <= tau*, so every score of the support is in the candidate lists: the
           // exact solve on chip ends the refinement.
           float t;
-          if (solve_list<AK>(cand + row, nc0, cand + kCandPerThread * kTile + row, nc1, kTile, cz, tau, lo, hi,
-                             t)) {
+          if (solve_list<AK>(cand + row, ncs, kCandPerThread * kTile, kTile, cz, tau, lo, hi, t)) {
             tau = t;
             done = true;
           }
@@ -782,7 +833,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
 }
 
 int fwd_smem_bytes(int Tc) {
-  return 1024 + kTileBytes * (1 + kSlots) + Tc * kTile * 4 + 2 * kCandPerThread * kTile * 4 + 8 * kTile * 4;
+  return 1024 + kTileBytes * (1 + kSlots) + Tc * kTile * 4 + kParts * kCandPerThread * kTile * 4 + kParts * 4 * kTile * 4;
 }
 
 cudaError_t launch_fwd(bool alpha15, const FwdParams& p, int grid, cudaStream_t s) {
