@@ -283,24 +283,55 @@ def run_ours(args):
     tokens_per_step = w.B * w.L
     value = job_throughput(world, tokens_per_step, args.steps, total_ms)
 
-    # ---- end to end through the public API: pinned host -> device, fwd+bwd, device -> host
-    out_host = {k: torch.empty(shp, dtype=torch.float32).pin_memory() for k in ("O", "dQ", "dK", "dV")}
+    # ---- end to end through the public API: pinned host -> device, fwd+bwd, device -> host.
+    # Every step copies its inputs in and its results out. The copies run on their own
+    # streams with two buffer sets, so step k's kernels overlap step k+1's upload and step
+    # k-1's download (as a training loop would pipeline them); events order each buffer
+    # set's reuse. The time runs from the first upload to the last download.
+    out_host = [{k: torch.empty(shp, dtype=torch.float32).pin_memory() for k in ("O", "dQ", "dK", "dV")}
+                for _ in range(2)]
     h2d = sum(v.numel() * v.element_size() for v in pinned.values())
-    d2h = sum(v.numel() * v.element_size() for v in out_host.values())
+    d2h = sum(v.numel() * v.element_size() for v in out_host[0].values())
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    din = [d, {k: torch.empty_like(v) for k, v in d.items()}]
+    dout = [{"O": O, "dQ": dQ, "dK": dK, "dV": dV},
+            {k: torch.empty(shp, dtype=torch.float32, device=dev) for k in ("O", "dQ", "dK", "dV")}]
+    tau2 = [tau, torch.empty_like(tau)]
+    ws2 = [ws, eb.alloc_workspace(desc, dev)]
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    in_ready, computed, out_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize(dev)
-    e0.record(stream)
-    for _ in range(args.steps):
-        for k in ("Q", "K", "V", "dO"):
-            d[k].copy_(pinned[k], non_blocking=True)
-        step(d)
-        for k, src in (("O", O), ("dQ", dQ), ("dK", dK), ("dV", dV)):
-            out_host[k].copy_(src, non_blocking=True)
-    e1.record(stream)
+    e0.record(s_in)
+    for k in range(args.steps):
+        b = k % 2
+        if k >= 2:
+            s_in.wait_event(computed[b])         # the kernels of step k-2 are done with din[b]
+        with torch.cuda.stream(s_in):
+            for n in ("Q", "K", "V", "dO"):
+                din[b][n].copy_(pinned[n], non_blocking=True)
+        in_ready[b].record(s_in)
+        stream.wait_event(in_ready[b])
+        if k >= 2:
+            stream.wait_event(out_done[b])       # step k-2's results have left dout[b]
+        src, dst = din[b], dout[b]
+        eb.entmax_attn_fwd(desc, src["Q"], src["K"], src["V"], dst["O"], tau2[b], ws2[b], stream)
+        eb.entmax_attn_bwd(desc, src["Q"], src["K"], src["V"], src["dO"], tau2[b], ws2[b], dst["dQ"], dst["dK"],
+                           dst["dV"], stream)
+        computed[b].record(stream)
+        s_out.wait_event(computed[b])
+        with torch.cuda.stream(s_out):
+            for n in ("O", "dQ", "dK", "dV"):
+                out_host[b][n].copy_(dst[n], non_blocking=True)
+        out_done[b].record(s_out)
+    e1.record(s_out)
     torch.cuda.synchronize(dev)
     e2e_value = job_throughput(world, tokens_per_step, args.steps,
                                max_over_ranks(e0.elapsed_time(e1), world, dev))
+    code2, _ = eb.entmax_last_device_status(desc, ws2[1], stream)
+    if code2 != eb.ENTMAX_OK:
+        raise SystemExit(f"device status {eb.STATUS_NAMES[code2]} in the end-to-end run")
 
     # ---- work actually done (per-tile counters written by the forward)
     M, st = eb.block_mask((desc, ws))
@@ -409,6 +440,7 @@ def sparsity_sweeps(w, alpha, dev, steps: int = 10):
         return {"block_sparsity_128": 1.0 - float(st[..., 2].sum()) / max(1, int(st[..., 3].sum())),
                 "refine_sweeps_mean": float(st[..., 0].float().mean()),
                 "s_tiles_per_active": float(st[..., 1].sum()) / max(1, int(st[..., 3].sum())),
+                "s_tiles": int(st[..., 1].sum()), "flagged_tiles": int(st[..., 2].sum()),
                 "fwd_ms": statistics.mean(fwd), "bwd_ms": statistics.mean(bwd),
                 "ms": statistics.mean(fwd) + statistics.mean(bwd)}
 
@@ -422,8 +454,29 @@ def sparsity_sweeps(w, alpha, dev, steps: int = 10):
         r = point(make_inputs(w.with_(sigma_q=sq), seed=7))
         r["sigma_q"] = sq
         sigma.append(r)
-    return {"planted_rho": planted, "iid_sigma_q": sigma,
+    return {"planted_rho": planted, "iid_sigma_q": sigma, "marginal": marginal_throughput(planted),
             "note": "same shape as the timed workload; planted inputs are a builder-added family"}
+
+
+def marginal_throughput(points) -> dict:
+    """Throughput on non-skipped blocks: a least-squares line of time against algorithmic
+    tile products over the planted points (block sparsity 0.06 .. 0.93). The slope is the
+    cost of the work that grows with the flagged blocks (the intercept holds the fixed and
+    the max-pass costs), so 1 / slope is the rate at which flagged blocks are processed."""
+    def fit(xs, ys):
+        n = len(xs)
+        mx, my = sum(xs) / n, sum(ys) / n
+        sxx = sum((x - mx) ** 2 for x in xs)
+        b = sum((x - mx) * (y - my) for x, y in zip(xs, ys)) / sxx
+        return b, my - b * mx
+    out = {}
+    fl = [UNIT_FLOP * (p["s_tiles"] + 2 * p["flagged_tiles"]) for p in points]
+    bl = [UNIT_FLOP * 5 * p["flagged_tiles"] for p in points]
+    for name, xs, ys in (("fwd", fl, [p["fwd_ms"] for p in points]), ("bwd", bl, [p["bwd_ms"] for p in points]),
+                         ("fwd+bwd", [a + b for a, b in zip(fl, bl)], [p["ms"] for p in points])):
+        b, a = fit(xs, ys)
+        out[name] = {"tflops_on_flagged_blocks": 1e-9 / b if b > 0 else None, "intercept_ms": a}
+    return out
 
 
 def act_pairs(w) -> int:
