@@ -199,3 +199,12 @@ def test_long_head_L12288():
     rep = {}
     compare(w, 1.5, backward=True, report=rep)
     print(w.name, {k: (float(v) if not isinstance(v, int) else v) for k, v in rep.items()})
+
+
+def test_max_length_head():
+    """L = ENTMAX_MAX_L = 16384 (128 key tiles: every bit of the four mask words), one head,
+    causal, alpha = 1.5, checked element by element. Shared memory: 217 KB of 227."""
+    w = small_case("max_L16384", B=1, H=1, L=16384, causal=True, sigma_q=3.0)
+    rep = {}
+    compare(w, 1.5, backward=True, report=rep)
+    print(w.name, {k: (float(v) if not isinstance(v, int) else v) for k, v in rep.items()})
