@@ -218,7 +218,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     int prev_it = -1;
     // Adds dQ of the query tile `it` handled at step `s` (TMEM buffer s % 2) to global
     // memory. The caller has already waited for that step's MMAs. Each thread stages its
-    // 16 columns (scaled) in the swizzled box of its column half; then thread 0 issues
+    // 16 columns (scaled) in the swizzled box that holds them (one box per 32 of dQ's 64
+    // columns); then thread 0 issues
     // one TMA reduce-add per box. The staging buffer is reused only after the previous
     // reduce-adds have read it.
     auto flush_dq = [&](uint32_t s, int it) {

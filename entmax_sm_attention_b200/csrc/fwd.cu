@@ -5,14 +5,15 @@
 //   Phase 1 (maximum): stream the structurally active key tiles; S = Q K^T on the
 //     tensor cores (tcgen05, accumulator in TMEM). Each row keeps its max in every key
 //     tile, in shared memory.
-//   Initial threshold: each thread keeps the four largest of its half-tile maxima in
-//     registers; the row's tau restricted to those eight scores is a lower bound
+//   Initial threshold: each thread keeps the four largest of its part-tile maxima (the
+//     maxima over its 32 columns of each key tile) in registers; the row's tau
+//     restricted to those 16 scores (four threads per row) is a lower bound
 //     tau_T <= tau* (entmax on a subset of the scores has fewer nonnegative terms in
 //     Eq. 4). It plays the role the paper gives its on-chip histogram (Phase 2), without
 //     an extra pass over K.
 //   Phase 3 (refinement): a sweep at tau accumulates S1 = sum u, S2 = sum u^2 and the
 //     count (u = [z - tau]_+) and copies every score with u > 0 into shared memory
-//     (64 per row and column half). While tau <= tau* (f(tau) >= 0, true at tau_T) those
+//     (32 per row and column part, 128 per row). While tau <= tau* (f(tau) >= 0, true at tau_T) those
 //     copies hold the whole support, so a row whose copies fit is solved exactly on
 //     chip: safeguarded Newton on Eq. 4 (§3.2), finished by the exact root of the
 //     current support's piece (alpha = 2: (S1-1)/C; alpha = 1.5: the smaller root of
@@ -510,7 +511,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     float m = -INFINITY;
     float top[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 
-    // Phase 1: per-key-tile row maxima over this thread's column half (combined in smem).
+    // Phase 1: per-key-tile row maxima over this thread's column part (combined in smem).
     for_each_bit(act, kMaskWords, [&](int jt) {
       const uint32_t bf = sbuf;
       warp_wait(&sh.s_full[bf], (sfull_par >> bf) & 1, status, abrt);
