@@ -162,6 +162,7 @@ def cpu_oracle_sample(w, alpha: float, seed: int, target_s: float):
 
     inp = make_inputs(w.with_(B=1, H=1), seed)
     heads, t_total = 0, 0.0
+    sparsity = None
     g = __import__("torch").Generator().manual_seed(seed)
     while heads < w.B * w.H and (heads == 0 or t_total < target_s):
         if heads > 0:   # a fresh head of the same distribution per iteration
@@ -173,12 +174,30 @@ def cpu_oracle_sample(w, alpha: float, seed: int, target_s: float):
         r = pr.rows(backward=True)
         pr.cols(r["tau"], r["delta"])
         t_total += time.perf_counter() - t0
+        if heads == 0:
+            sparsity = oracle_block_sparsity(pr, r["tau"], w)
         heads += 1
     del g
     tokens = w.B * w.L * heads / (w.B * w.H)
     return tokens / t_total, oracle.max_threads(), (
         f"{heads} of {w.B * w.H} heads (b,h) of {w.name}, full fwd+bwd per head in fp64; "
-        f"tokens/s = heads/(B*H) * B*L / seconds")
+        f"tokens/s = heads/(B*H) * B*L / seconds"), sparsity
+
+
+def oracle_block_sparsity(pr, tau, w) -> dict:
+    """Block sparsity of one head from the fp64 oracle, at the kernel's 128 x 128 blocks and
+    at the 64 x 64 blocks of AdaSplash-2 Fig. 7: the share of structurally active blocks
+    with no nonzero weight (causal workloads without padding or window)."""
+    import numpy as np
+
+    out = {}
+    for blk in (128, 64):
+        M, _, _ = pr.block_mask(tau, blk, blk)
+        flagged = int(np.unpackbits(M.view(np.uint8)).sum())
+        T = -(-w.L // blk)
+        active = T * (T + 1) // 2 if w.causal else T * T
+        out[f"{blk}x{blk}"] = 1.0 - flagged / active
+    return out
 
 
 def run_reference(args):
@@ -193,7 +212,7 @@ def run_reference(args):
 
     times = []
     for k in range(args.warmup + args.steps):
-        v, cores, _ = cpu_oracle_sample(w, args.alpha, args.seed + 100 * k, 0.0)   # one head per step
+        v, cores, _, _ = cpu_oracle_sample(w, args.alpha, args.seed + 100 * k, 0.0)   # one head per step
         if k >= args.warmup:
             times.append(v)
     value = statistics.mean(times)
@@ -392,8 +411,10 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_sweeps:
         result["detail"]["sparsity_sweeps"] = sparsity_sweeps(w, alpha, dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, cores, sample = cpu_oracle_sample(w, alpha, args.seed, args.cpu_seconds)
+        v, cores, sample, osp = cpu_oracle_sample(w, alpha, args.seed, args.cpu_seconds)
         result["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
+        if osp is not None and w.window < 0 and w.kv_len is None:
+            result["detail"]["block_sparsity_oracle_head0"] = osp
     if rank == 0:
         print(json.dumps(result), flush=True)
     if world > 1:
