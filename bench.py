@@ -153,21 +153,23 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------------ CPU oracle
-def cpu_oracle_sample(w, alpha: float, seed: int, target_s: float):
-    """Times the fp64 oracle (as it stands) on whole heads of the workload: forward and
-    backward of head 0, 1, ... until target_s has passed. Returns tokens/s scaled to the
-    full batch (heads done / H of B*L tokens), the thread count and a description."""
+def cpu_oracle_sample(w, alpha: float, seed: int, target_s: float, inp=None):
+    """Times the fp64 oracle (as it stands) on whole heads of the workload, drawn with the
+    GPU arm's seed (the same bytes the GPU arm computes on): forward and backward of head
+    (0, 0), (0, 1), ... until target_s has passed. Returns tokens/s scaled to the full
+    batch (heads done / (B*H) of B*L tokens), the thread count, a description, the oracle
+    block sparsity of the first head, and the seconds per head."""
     import oracle
     from entmax_sm_attention_b200.workloads import make_inputs
 
-    inp = make_inputs(w.with_(B=1, H=1), seed)
+    if inp is None:
+        inp = make_inputs(w, seed)
     heads, t_total = 0, 0.0
     sparsity = None
-    g = __import__("torch").Generator().manual_seed(seed)
     while heads < w.B * w.H and (heads == 0 or t_total < target_s):
-        if heads > 0:   # a fresh head of the same distribution per iteration
-            inp = make_inputs(w.with_(B=1, H=1), seed + heads)
-        pr = oracle.Problem(inp["Q"], inp["K"], inp["V"], inp["dO"], alpha=alpha, scale=w.scale,
+        b, h = divmod(heads, w.H)
+        one = {k: v[b:b + 1, h:h + 1] for k, v in inp.items()}
+        pr = oracle.Problem(one["Q"], one["K"], one["V"], one["dO"], alpha=alpha, scale=w.scale,
                             causal=w.causal, window=w.window,
                             kv_len=None if w.kv_len is None else [w.kv_len])
         t0 = time.perf_counter()
@@ -177,11 +179,10 @@ def cpu_oracle_sample(w, alpha: float, seed: int, target_s: float):
         if heads == 0:
             sparsity = oracle_block_sparsity(pr, r["tau"], w)
         heads += 1
-    del g
     tokens = w.B * w.L * heads / (w.B * w.H)
     return tokens / t_total, oracle.max_threads(), (
-        f"{heads} of {w.B * w.H} heads (b,h) of {w.name}, full fwd+bwd per head in fp64; "
-        f"tokens/s = heads/(B*H) * B*L / seconds"), sparsity
+        f"{heads} of {w.B * w.H} heads (b,h) of {w.name} (seed {seed}, the GPU arm's inputs), full fwd+bwd "
+        f"per head in fp64; tokens/s = heads/(B*H) * B*L / seconds"), sparsity, t_total / heads
 
 
 def oracle_block_sparsity(pr, tau, w) -> dict:
@@ -200,30 +201,48 @@ def oracle_block_sparsity(pr, tau, w) -> dict:
     return out
 
 
+def bench_config(w, alpha: float, seed: int, world: int) -> dict:
+    """The `config` object of both arms' JSON lines (the same workload, same keys)."""
+    return {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "d": w.d, "alpha": alpha,
+            "causal": w.causal, "window": w.window, "kv_len": w.kv_len, "sigma_q": w.sigma_q,
+            "seed": seed, "l2": "flushed (256 MB write) before every timed GPU step",
+            "parallelism": f"replica x{world} (independent batches)"}
+
+
 def run_reference(args):
-    """--impl reference: the oracle on the host cores, one head per step."""
+    """--impl reference: the oracle on the host cores. Step k computes forward + backward
+    of head k mod (B*H) of the GPU arm's own inputs (same seed); ms_per_step is the measured
+    mean time of one such step, and value is the workload's tokens/s at that rate."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    from entmax_sm_attention_b200.workloads import WORKLOADS
+    from entmax_sm_attention_b200.workloads import WORKLOADS, make_inputs
 
     w = WORKLOADS[args.workload]
+    inp = make_inputs(w, args.seed)
     import oracle
 
-    times = []
+    secs = []
     for k in range(args.warmup + args.steps):
-        v, cores, _, _ = cpu_oracle_sample(w, args.alpha, args.seed + 100 * k, 0.0)   # one head per step
+        b, h = divmod(k % (w.B * w.H), w.H)
+        one = {n: v[b:b + 1, h:h + 1] for n, v in inp.items()}
+        pr = oracle.Problem(one["Q"], one["K"], one["V"], one["dO"], alpha=args.alpha, scale=w.scale,
+                            causal=w.causal, window=w.window, kv_len=None if w.kv_len is None else [w.kv_len])
+        t0 = time.perf_counter()
+        r = pr.rows(backward=True)
+        pr.cols(r["tau"], r["delta"])
         if k >= args.warmup:
-            times.append(v)
-    value = statistics.mean(times)
-    sample = (f"each step = full fwd+bwd of one (b,h) head of {w.name} (of {w.B * w.H}); "
-              f"tokens/s scaled by heads/(B*H)")
-    ms = w.B * w.L / value * 1e3
+            secs.append(time.perf_counter() - t0)
+    ms_per_step = statistics.mean(secs) * 1e3
+    tokens_per_step = w.B * w.L / (w.B * w.H)      # one head's share of the batch
+    value = tokens_per_step / (ms_per_step * 1e-3)
+    cores = oracle.max_threads()
+    sample = (f"each step = full fwd+bwd in fp64 of one (b,h) head of {w.name} (head k mod {w.B * w.H}, "
+              f"seed {args.seed}: the GPU arm's inputs); tokens/s = (B*L/(B*H)) / seconds per step")
     out = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
-           "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+           "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-           "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "d": w.d, "alpha": args.alpha,
-                      "causal": w.causal, "sigma_q": w.sigma_q},
+           "config": bench_config(w, args.alpha, args.seed, args.gpus),
            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
@@ -352,27 +371,41 @@ def run_ours(args):
     if code2 != eb.ENTMAX_OK:
         raise SystemExit(f"device status {eb.STATUS_NAMES[code2]} in the end-to-end run")
 
-    # ---- work actually done (per-tile counters written by the forward)
+    # ---- work actually done (per-tile counters written by the forward and the backward)
     M, st = eb.block_mask((desc, ws))
+    bst = eb.bwd_counters((desc, ws)).cpu().long()
     st = st.cpu().long()
     n_sweeps, n_s, n_out, n_act = (st[..., c] for c in range(4))
     s_tiles, out_tiles, act_tiles = int(n_s.sum()), int(n_out.sum()), int(n_act.sum())
-    # Algorithmic tensor work at tile granularity: forward = every S tile computed (max
-    # pass + refinement passes + output pass) + the A V and g V products on flagged
-    # tiles; backward = S, dA, dV, dK, dQ on every flagged tile pair.
-    fwd_flops = UNIT_FLOP * (s_tiles + 2 * out_tiles)
-    bwd_flops = UNIT_FLOP * 5 * out_tiles
-    # Issued tensor work: the backward feeds dS as two bf16 terms (hi + lo) to dK and dQ.
-    fwd_issued = UNIT_FLOP * (s_tiles + 2 * out_tiles)
+    work = pair_work(w, M.cpu(), st)
+    # Algorithmic tensor work (the scope table's per-pair figures): forward
+    # (1+R) 2d |A_i| + 3 2d |F_i| summed over rows (max pass and R refinement passes over
+    # the active keys; S, A V and g V over the keys of flagged tiles), backward 5 2d |F_i|
+    # (S, dA, dV, dK, dQ). R is each query tile's measured refinement count.
+    fwd_flops = work["fwd_flops"]
+    bwd_flops = work["bwd_flops"]
+    # The same at tile granularity (every 128x128 block counted whole, diagonal blocks
+    # included), and the work the tensor cores are issued (dS enters dK and dQ as two
+    # bf16 terms, hi + lo).
+    fwd_tile_flops = UNIT_FLOP * (s_tiles + 2 * out_tiles)
+    bwd_tile_flops = UNIT_FLOP * 5 * out_tiles
+    fwd_issued = fwd_tile_flops
     bwd_issued = UNIT_FLOP * 7 * out_tiles
     fwd_avg, bwd_avg = statistics.mean(fwd_ms), statistics.mean(bwd_ms)
     peaks = load_peaks()
-    peak = peaks["bf16_tflops_sustained"]
+    # Each kernel runs for about half a millisecond inside a ~1 ms step: the burst peak
+    # (cuBLAS timed alone) is its denominator, not the seconds-long sustained figure.
+    peak = peaks["bf16_tflops"]
     dom = "bwd" if bwd_avg >= fwd_avg else "fwd"
     dom_ms = bwd_avg if dom == "bwd" else fwd_avg
     dom_flops = bwd_flops if dom == "bwd" else fwd_flops
     achieved = dom_flops / (dom_ms * 1e-3) / 1e12
     total_tflops = (fwd_flops + bwd_flops) / (ms_per_step * 1e-3) / 1e12
+    phases = phase_shares(st, bst)
+    # The threshold and mask passes (max pass, refinement, decision) read Q and K once per
+    # head from HBM (2 B per element) and write tau (4 B per row) and the two masks.
+    tm_bytes = 2 * 2 * w.B * w.H * w.L * w.d + 4 * w.B * w.H * w.L + 2 * M.numel() * 4
+    tm_ms = fwd_avg * (phases["fwd"]["max_pass"] + phases["fwd"]["refine_and_mask"])
     # Softmax-equivalent work over structurally active pairs (4d fwd, 10d bwd per pair).
     pairs = act_pairs(w)
     sm_eq = (4 + 10) * w.d * pairs / (ms_per_step * 1e-3) / 1e12
@@ -381,13 +414,11 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "d": w.d, "alpha": alpha,
-                   "causal": w.causal, "window": w.window, "kv_len": w.kv_len, "sigma_q": w.sigma_q,
-                   "seed": args.seed, "l2": "flushed (256 MB write) before every timed step",
-                   "parallelism": f"replica x{world} (independent batches)"},
-        "roofline": {"bound": "tensor", "kernel": f"entmax {dom} (algorithmic bf16 tile products)",
+        "config": bench_config(w, alpha, args.seed, world),
+        "roofline": {"bound": "tensor",
+                     "kernel": f"entmax {dom} (algorithmic bf16 work over active / flagged pairs)",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                     "peak_source": f"{peaks['source']} bf16 sustained (cuBLAS loop under the power cap)",
+                     "peak_source": f"{peaks['source']} bf16 burst (cuBLAS timed alone; of measured)",
                      "traffic": ncu_traffic(dom, w.name, alpha),
                      "traffic_unit": "bytes per launch (ncu dram read+write; null if the kernel changed)"},
         "clocks": clk,
@@ -399,8 +430,19 @@ def run_ours(args):
             "tflops_total_algorithmic": total_tflops,
             "tflops_fwd_algorithmic": fwd_flops / (fwd_avg * 1e-3) / 1e12,
             "tflops_bwd_algorithmic": bwd_flops / (bwd_avg * 1e-3) / 1e12,
+            "fwd_flops_pairs": fwd_flops, "bwd_flops_pairs": bwd_flops,
+            "fwd_flops_tiles": fwd_tile_flops, "bwd_flops_tiles": bwd_tile_flops,
+            "tflops_fwd_tiles": fwd_tile_flops / (fwd_avg * 1e-3) / 1e12,
+            "tflops_bwd_tiles": bwd_tile_flops / (bwd_avg * 1e-3) / 1e12,
+            "frac_fwd_of_burst": fwd_flops / (fwd_avg * 1e-3) / 1e12 / peaks["bf16_tflops"],
+            "frac_bwd_of_burst": bwd_flops / (bwd_avg * 1e-3) / 1e12 / peaks["bf16_tflops"],
             "tflops_fwd_issued": fwd_issued / (fwd_avg * 1e-3) / 1e12,
             "tflops_bwd_issued": bwd_issued / (bwd_avg * 1e-3) / 1e12,
+            "active_pairs": work["active_pairs"], "flagged_pairs": work["flagged_pairs"],
+            "phase_cycle_shares": phases,
+            "tau_mask_passes": {"ms_equiv": tm_ms, "algorithmic_bytes": tm_bytes,
+                                "hbm_gbs": tm_bytes / (tm_ms * 1e-3) / 1e9 if tm_ms > 0 else None,
+                                "note": "time = forward time x the max-pass and refinement cycle shares"},
             "softmax_equiv_tflops": sm_eq,
             "block_sparsity_128": 1.0 - out_tiles / max(1, act_tiles),
             "refine_sweeps_mean": float(n_sweeps.float().mean()), "refine_sweeps_max": int(n_sweeps.max()),
@@ -411,7 +453,7 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_sweeps:
         result["detail"]["sparsity_sweeps"] = sparsity_sweeps(w, alpha, dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, cores, sample, osp = cpu_oracle_sample(w, alpha, args.seed, args.cpu_seconds)
+        v, cores, sample, osp, _ = cpu_oracle_sample(w, alpha, args.seed, args.cpu_seconds, inp=host)
         result["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
         if osp is not None and w.window < 0 and w.kv_len is None:
             result["detail"]["block_sparsity_oracle_head0"] = osp
@@ -498,6 +540,67 @@ def marginal_throughput(points) -> dict:
         b, a = fit(xs, ys)
         out[name] = {"tflops_on_flagged_blocks": 1e-9 / b if b > 0 else None, "intercept_ms": a}
     return out
+
+
+def block_pair_counts(w):
+    """Structurally active (query, key) pairs in every 128 x 128 block, per batch entry:
+    int64 [B, T, T] (the same for every head)."""
+    import numpy as np
+
+    L, T = w.L, -(-w.L // TILE)
+    out = np.zeros((w.B, T, T), np.int64)
+    i = np.arange(L)[:, None]
+    j = np.arange(L)[None, :]
+    for b in range(w.B):
+        kv = L if w.kv_len is None else min(max(w.kv_len, 1), L)
+        act = np.broadcast_to(j < kv, (L, L))
+        if w.window >= 0:
+            act = act & (j <= i) & ((j == 0) | (i - j <= w.window))
+        elif w.causal:
+            act = act & (j <= i)
+        pad = np.zeros((T * TILE, T * TILE), np.int64)
+        pad[:L, :L] = act
+        out[b] = pad.reshape(T, TILE, T, TILE).sum((1, 3))
+    return out
+
+
+def pair_work(w, M, st) -> dict:
+    """Algorithmic tensor work at pair granularity from the block mask M (int32 bit
+    patterns [B, H, T, words]) and the forward counters st ([B, H, T, 8]): forward
+    sum_i (1+R_i) 2d |A_i| + 3 2d |F_i|, backward 5 2d |F_i|, where A_i are the active keys
+    of row i, F_i the active keys of row i inside flagged blocks, and R_i the refinement
+    passes of row i's query tile."""
+    import numpy as np
+
+    cnt = block_pair_counts(w)                                      # [B, T, T]
+    T = cnt.shape[1]
+    words = M.numpy().view(np.uint32).astype(np.int64)              # [B, H, T, W]
+    bits = np.zeros(words.shape[:3] + (T,), bool)
+    for jt in range(T):
+        bits[..., jt] = (words[..., jt // 32] >> (jt % 32)) & 1 == 1
+    flagged = (bits * cnt[:, None]).sum(-1)                         # [B, H, T] pairs in flagged blocks
+    active = np.broadcast_to(cnt.sum(-1)[:, None], flagged.shape)   # [B, H, T] active pairs per query tile
+    R = st[..., 0].numpy().astype(np.int64)
+    two_d = 2 * w.d
+    fwd = int(((1 + R) * active).sum() * two_d + 3 * flagged.sum() * two_d)
+    bwd = int(5 * flagged.sum() * two_d)
+    return {"fwd_flops": fwd, "bwd_flops": bwd, "active_pairs": int(active.sum()),
+            "flagged_pairs": int(flagged.sum())}
+
+
+def phase_shares(st, bst) -> dict:
+    """Cycle shares of the phases, summed over CTAs, from the kernels' clock64 counters:
+    forward max pass / refinement + mask decision / output pass; backward (first
+    row-owner warp) waiting for S and dA / waiting for the previous tile's MMAs / forming
+    A and dS / staging dQ."""
+    f = st[..., 4:8].double().sum((0, 1, 2))
+    b = bst[..., 1:6].double().sum((0, 1, 2))
+    ft = float(f[3]) or 1.0
+    bt = float(b[0]) or 1.0
+    return {"fwd": {"max_pass": float(f[0]) / ft, "refine_and_mask": float(f[1]) / ft,
+                    "output_pass": float(f[2]) / ft, "cta_cycles": float(f[3])},
+            "bwd": {"wait_s_dA": float(b[1]) / bt, "wait_prev_mma": float(b[2]) / bt,
+                    "form_A_dS": float(b[3]) / bt, "stage_dQ": float(b[4]) / bt, "cta_cycles": float(b[0])}}
 
 
 def act_pairs(w) -> int:

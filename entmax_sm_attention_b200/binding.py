@@ -25,6 +25,9 @@ ENTMAX_TILE = 128
 EXPORTS = ("entmax_attn_workspace_bytes", "entmax_attn_fwd", "entmax_attn_bwd", "entmax_rows",
            "entmax_last_device_status", "entmax_attn_block_mask", "entmax_attn_fwd_noalloc")
 ENTMAX_NOALLOC_SCRATCH_BYTES = 16 << 20
+ENTMAX_SELFTEST_STALL = 1
+FWD_STATS = 8     # int32 counters per query tile (forward)
+BWD_STATS = 8     # int32 counters per key tile (backward)
 
 
 class EntmaxError(RuntimeError):
@@ -40,6 +43,7 @@ class AttnDesc(ctypes.Structure):
         ("alpha", ctypes.c_float), ("scale", ctypes.c_float),
         ("causal", ctypes.c_int), ("window", ctypes.c_int),
         ("kv_len", ctypes.c_void_p), ("dtype", ctypes.c_int), ("max_sweeps", ctypes.c_int),
+        ("wait_limit_us", ctypes.c_int), ("selftest", ctypes.c_int),
     ]
 
 
@@ -62,11 +66,11 @@ def load_library(path: str = LIB_PATH):
     lib.entmax_attn_fwd.restype = i
     lib.entmax_attn_bwd.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.entmax_attn_bwd.restype = i
-    lib.entmax_rows.argtypes = [vp, i, i, i, f, vp, vp, vp]
+    lib.entmax_rows.argtypes = [vp, i, i, i, f, vp, vp, vp, vp]
     lib.entmax_rows.restype = i
     lib.entmax_last_device_status.argtypes = [dp, vp, ctypes.POINTER(i), vp]
     lib.entmax_last_device_status.restype = i
-    lib.entmax_attn_block_mask.argtypes = [dp, vp, vp, vp, vp]
+    lib.entmax_attn_block_mask.argtypes = [dp, vp, vp, vp, vp, vp]
     lib.entmax_attn_block_mask.restype = i
     lib.entmax_attn_fwd_noalloc.argtypes = [dp, vp, vp, vp, vp, vp, vp]
     lib.entmax_attn_fwd_noalloc.restype = i
@@ -111,12 +115,14 @@ class Options:
 
 def make_desc(B: int, H: int, L: int, d: int = 64, *, alpha: float = 1.5, scale: float | None = None,
               causal: bool = False, window: int = -1, kv_len: torch.Tensor | None = None,
-              dtype: int = ENTMAX_BF16, max_sweeps: int = 0) -> AttnDesc:
+              dtype: int = ENTMAX_BF16, max_sweeps: int = 0, wait_limit_us: int = 0,
+              selftest: int = 0) -> AttnDesc:
     """Fill an entmax_attn_desc. kv_len, if given, is a device int32 tensor [B]."""
     if kv_len is not None and (kv_len.dtype != torch.int32 or not kv_len.is_cuda):
         raise ValueError("kv_len must be a CUDA int32 tensor")
     return AttnDesc(B, H, L, d, float(alpha), float(scale if scale is not None else d ** -0.5),
-                    int(bool(causal) or window >= 0), int(window), _ptr(kv_len), int(dtype), int(max_sweeps))
+                    int(bool(causal) or window >= 0), int(window), _ptr(kv_len), int(dtype), int(max_sweeps),
+                    int(wait_limit_us), int(selftest))
 
 
 def entmax_attn_workspace_bytes(desc: AttnDesc) -> int:
@@ -134,13 +140,14 @@ def entmax_attn_bwd(desc: AttnDesc, Q, K, V, dO, tau, workspace, dQ, dK, dV, str
         _ptr(dQ), _ptr(dK), _ptr(dV), _stream(stream)))
 
 
-def entmax_rows(S, rows: int, n: int, ld: int, alpha: float, P, tau, stream=None) -> int:
+def entmax_rows(S, rows: int, n: int, ld: int, alpha: float, P, tau, status=None, stream=None) -> int:
     return _check("entmax_rows", load_library().entmax_rows(
-        _ptr(S), int(rows), int(n), int(ld), float(alpha), _ptr(P), _ptr(tau), _stream(stream)))
+        _ptr(S), int(rows), int(n), int(ld), float(alpha), _ptr(P), _ptr(tau), _ptr(status), _stream(stream)))
 
 
 def entmax_last_device_status(desc: AttnDesc, workspace, stream=None) -> tuple[int, int]:
-    """Returns (status code, raw status word); synchronises the stream."""
+    """Returns (status code, raw status word); synchronises the stream. workspace=None reads
+    the no-allocation forward's scratch on the current device."""
     word = ctypes.c_int(0)
     code = load_library().entmax_last_device_status(ctypes.byref(desc), _ptr(workspace), ctypes.byref(word),
                                                      _stream(stream))
@@ -148,9 +155,9 @@ def entmax_last_device_status(desc: AttnDesc, workspace, stream=None) -> tuple[i
     return code, word.value
 
 
-def entmax_attn_block_mask(desc: AttnDesc, workspace, M=None, stats=None, stream=None) -> int:
+def entmax_attn_block_mask(desc: AttnDesc, workspace, M=None, stats=None, bwd_stats=None, stream=None) -> int:
     return _check("entmax_attn_block_mask", load_library().entmax_attn_block_mask(
-        ctypes.byref(desc), _ptr(workspace), _ptr(M), _ptr(stats), _stream(stream)))
+        ctypes.byref(desc), _ptr(workspace), _ptr(M), _ptr(stats), _ptr(bwd_stats), _stream(stream)))
 
 
 def entmax_attn_fwd_noalloc(desc: AttnDesc, Q, K, V, O, tau, stream=None) -> int:
@@ -175,12 +182,13 @@ def mask_shape(desc: AttnDesc) -> tuple:
 
 
 def forward(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, *, alpha: float = 1.5, scale=None,
-            causal: bool = False, window: int = -1, kv_len=None, max_sweeps: int = 0):
+            causal: bool = False, window: int = -1, kv_len=None, max_sweeps: int = 0, wait_limit_us: int = 0,
+            selftest: int = 0):
     """O, tau and the (desc, workspace) context of one forward call on [B, H, L, 64] tensors."""
     B, H, L, d = Q.shape
     dtype = ENTMAX_BF16 if Q.dtype == torch.bfloat16 else ENTMAX_FP32
     desc = make_desc(B, H, L, d, alpha=alpha, scale=scale, causal=causal, window=window, kv_len=kv_len,
-                     dtype=dtype, max_sweeps=max_sweeps)
+                     dtype=dtype, max_sweeps=max_sweeps, wait_limit_us=wait_limit_us, selftest=selftest)
     ws = alloc_workspace(desc, Q.device)
     O = torch.empty((B, H, L, d), dtype=torch.float32, device=Q.device)
     tau = torch.empty((B, H, L), dtype=torch.float32, device=Q.device)
@@ -197,19 +205,34 @@ def backward(ctx, Q, K, V, dO, tau):
 
 
 def block_mask(ctx):
-    """(M as int32 bit patterns [B, H, Tr, ceil(Tc/32)], stats int32 [B, H, Tr, 4]) of a
-    forward; stats = (refinement passes, S tiles computed, flagged tiles, active tiles)."""
+    """(M as int32 bit patterns [B, H, Tr, ceil(Tc/32)], stats int32 [B, H, Tr, 8]) of a
+    forward; stats = (refinement passes, S tiles computed, flagged tiles, active tiles,
+    then cycles of the max pass, of refinement + mask decision, of the output pass, total)."""
     desc, ws = ctx
     Mv = torch.empty(mask_shape(desc), dtype=torch.int32, device=ws.device)
-    st = torch.empty(mask_shape(desc)[:3] + (4,), dtype=torch.int32, device=ws.device)
+    st = torch.empty(mask_shape(desc)[:3] + (FWD_STATS,), dtype=torch.int32, device=ws.device)
     entmax_attn_block_mask(desc, ws, Mv, st)
     return Mv, st
 
 
-def rows(S: torch.Tensor, alpha: float = 1.5):
-    """P, tau = alpha-entmax of the rows of a CUDA fp32 matrix S [rows, n] (n % 4 == 0 or padded)."""
+def bwd_counters(ctx):
+    """int32 [B, H, Tc, 8] counters of the last backward per key tile: flagged query tiles
+    visited, total cycles, and the first row-owner warp's cycles waiting for S/dA, waiting
+    for the previous tile's MMAs, forming A/dS, staging dQ (then two zeros)."""
+    desc, ws = ctx
+    st = torch.empty(mask_shape(desc)[:3] + (BWD_STATS,), dtype=torch.int32, device=ws.device)
+    entmax_attn_block_mask(desc, ws, None, None, st)
+    return st
+
+
+def rows(S: torch.Tensor, alpha: float = 1.5, return_status: bool = False):
+    """P, tau = alpha-entmax of the rows of a CUDA fp32 matrix S [rows, n] (n % 4 == 0 or padded).
+    With return_status, also the device status word (1 = a row reached the iteration cap)."""
     r, n = S.shape
     P = torch.empty_like(S)
     tau = torch.empty(r, dtype=torch.float32, device=S.device)
-    entmax_rows(S, r, n, S.stride(0), alpha, P, tau)
+    status = torch.zeros(1, dtype=torch.int32, device=S.device)
+    entmax_rows(S, r, n, S.stride(0), alpha, P, tau, status)
+    if return_status:
+        return P, tau, int(status.item())
     return P, tau

@@ -20,10 +20,13 @@ constexpr int kMaxSweeps = 64;
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Workspace layout. Everything the forward writes comes first (up to fwd_total); the
+// backward-only parts follow.
 struct Layout {
   int BH, Tr, Tc, Wc, Wr;
-  size_t off_status, off_M, off_MT, off_sumg, off_Ot, off_delta, off_stats, off_v16, off_do16, total;
-  size_t bytes_M, bytes_MT, bytes_stats;
+  size_t off_status, off_M, off_MT, off_sumg, off_Ot, off_stats, off_v16, fwd_total;
+  size_t off_delta, off_bstats, off_do16, total;
+  size_t bytes_M, bytes_MT, bytes_stats, bytes_bstats;
 };
 
 bool layout_of(const entmax_attn_desc* d, Layout* l) {
@@ -46,13 +49,17 @@ bool layout_of(const entmax_attn_desc* d, Layout* l) {
   off += align256(rows * 4);
   l->off_Ot = off;
   off += align256(rows * kD * 4);
-  l->off_delta = off;
-  off += align256(rows * 4);
   l->off_stats = off;
-  l->bytes_stats = (size_t)l->BH * l->Tr * 16;
+  l->bytes_stats = (size_t)l->BH * l->Tr * kFwdStats * 4;
   off += align256(l->bytes_stats);
   l->off_v16 = off;
   off += align256(rows * kD * 2);
+  l->fwd_total = off;
+  l->off_delta = off;
+  off += align256(rows * 4);
+  l->off_bstats = off;
+  l->bytes_bstats = (size_t)l->BH * l->Tc * kBwdStats * 4;
+  off += align256(l->bytes_bstats);
   l->off_do16 = off;
   off += align256(rows * kD * 2);
   l->total = off;
@@ -67,6 +74,8 @@ entmax_status check_desc(const entmax_attn_desc* d) {
   if (d->causal != 0 && d->causal != 1) return ENTMAX_EINVAL;
   if (d->max_sweeps < 0 || d->max_sweeps > kMaxSweeps) return ENTMAX_EINVAL;
   if (d->dtype != ENTMAX_BF16 && d->dtype != ENTMAX_FP32) return ENTMAX_EINVAL;
+  if (d->wait_limit_us < 0) return ENTMAX_EINVAL;
+  if (d->selftest != 0 && d->selftest != ENTMAX_SELFTEST_STALL) return ENTMAX_EINVAL;
   if (d->d != kD) return ENTMAX_EUNSUPPORTED;
   if (d->L > ENTMAX_MAX_L) return ENTMAX_EUNSUPPORTED;
   if (d->alpha != 1.5f && d->alpha != 2.0f) return ENTMAX_EUNSUPPORTED;
@@ -74,6 +83,10 @@ entmax_status check_desc(const entmax_attn_desc* d) {
 }
 
 bool aligned(const void* p, size_t a) { return p && (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+unsigned long long wait_limit_ns(const entmax_attn_desc* d) {
+  return d->wait_limit_us == 0 ? kWaitLimitNs : (unsigned long long)d->wait_limit_us * 1000ull;
+}
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -122,6 +135,15 @@ extern "C" size_t entmax_attn_workspace_bytes(const entmax_attn_desc* d) {
   layout_of(d, &l);
   return l.total;
 }
+
+namespace entmax {
+size_t fwd_workspace_bytes(const entmax_attn_desc* d) {
+  if (check_desc(d) != ENTMAX_OK) return 0;
+  Layout l;
+  layout_of(d, &l);
+  return l.fwd_total;
+}
+}  // namespace entmax
 
 extern "C" entmax_status entmax_attn_fwd(const entmax_attn_desc* d, const void* Q, const void* K, const void* V,
                                          float* O, float* tau, void* ws, void* stream) {
@@ -189,6 +211,8 @@ extern "C" entmax_status entmax_attn_fwd(const entmax_attn_desc* d, const void* 
   p.causal = d->causal || d->window >= 0;
   p.window = d->window < 0 ? -1 : d->window;
   p.max_sweeps = d->max_sweeps == 0 ? kDefaultSweeps : d->max_sweeps;
+  p.wait_limit_ns = wait_limit_ns(d);
+  p.selftest = d->selftest;
   return launch_fwd(d->alpha == 1.5f, p, l.BH * l.Tr, s) == cudaSuccess ? ENTMAX_OK : ENTMAX_ECUDA;
 }
 
@@ -221,6 +245,7 @@ extern "C" entmax_status entmax_attn_bwd(const entmax_attn_desc* d, const void* 
   p.dK = dK;
   p.dV = dV;
   p.status = reinterpret_cast<int*>(w + l.off_status);
+  p.stats = reinterpret_cast<int*>(w + l.off_bstats);
   p.kv_len = d->kv_len;
   p.H = d->H;
   p.L = d->L;
@@ -232,6 +257,8 @@ extern "C" entmax_status entmax_attn_bwd(const entmax_attn_desc* d, const void* 
   p.scale = d->scale;
   p.causal = d->causal || d->window >= 0;
   p.window = d->window < 0 ? -1 : d->window;
+  p.wait_limit_ns = wait_limit_ns(d);
+  p.selftest = d->selftest;
   const long rows = (long)l.BH * d->L;
   if (cudaMemsetAsync(dQ, 0, (size_t)rows * kD * 4, s) != cudaSuccess) return ENTMAX_ECUDA;
   if (launch_bf16_to_f16(dO, do16, rows * kD, reinterpret_cast<int*>(w + l.off_status), s) != cudaSuccess)
@@ -243,18 +270,24 @@ extern "C" entmax_status entmax_attn_bwd(const entmax_attn_desc* d, const void* 
 }
 
 extern "C" entmax_status entmax_rows(const float* S, int rows, int n, int ld, float alpha, float* P, float* tau,
-                                     void* stream) {
+                                     int* status, void* stream) {
   if (rows < 0 || n < 1 || ld < n || (ld % 4) != 0) return ENTMAX_EINVAL;
   if (alpha != 1.5f && alpha != 2.0f) return ENTMAX_EUNSUPPORTED;
   if (rows == 0) return ENTMAX_OK;
   if (!aligned(S, 16) || !aligned(P, 16) || !aligned(tau, 4)) return ENTMAX_EINVAL;
+  if (status && !aligned(status, 4)) return ENTMAX_EINVAL;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return launch_rows(alpha == 1.5f, S, rows, n, ld, P, tau, s) == cudaSuccess ? ENTMAX_OK : ENTMAX_ECUDA;
+  return launch_rows(alpha == 1.5f, S, rows, n, ld, P, tau, status, s) == cudaSuccess ? ENTMAX_OK : ENTMAX_ECUDA;
 }
 
 extern "C" entmax_status entmax_last_device_status(const entmax_attn_desc* d, const void* ws, int* status_out,
                                                    void* stream) {
-  if (check_desc(d) != ENTMAX_OK || !aligned(ws, 256) || !status_out) return ENTMAX_EINVAL;
+  if (check_desc(d) != ENTMAX_OK || !status_out) return ENTMAX_EINVAL;
+  if (!ws) {
+    ws = noalloc_scratch();   // the no-allocation forward's scratch on the current device
+    if (!ws) return ENTMAX_ECUDA;
+  }
+  if (!aligned(ws, 256)) return ENTMAX_EINVAL;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(s) != cudaSuccess) return ENTMAX_ECUDA;
   int word = 0;
@@ -267,7 +300,7 @@ extern "C" entmax_status entmax_last_device_status(const entmax_attn_desc* d, co
 }
 
 extern "C" entmax_status entmax_attn_block_mask(const entmax_attn_desc* d, const void* ws, uint32_t* M,
-                                                int* stats, void* stream) {
+                                                int* stats, int* bwd_stats, void* stream) {
   if (check_desc(d) != ENTMAX_OK || !aligned(ws, 256)) return ENTMAX_EINVAL;
   Layout l;
   layout_of(d, &l);
@@ -276,6 +309,9 @@ extern "C" entmax_status entmax_attn_block_mask(const entmax_attn_desc* d, const
   if (M && cudaMemcpyAsync(M, w + l.off_M, l.bytes_M, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
     return ENTMAX_ECUDA;
   if (stats && cudaMemcpyAsync(stats, w + l.off_stats, l.bytes_stats, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    return ENTMAX_ECUDA;
+  if (bwd_stats &&
+      cudaMemcpyAsync(bwd_stats, w + l.off_bstats, l.bytes_bstats, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
     return ENTMAX_ECUDA;
   return ENTMAX_OK;
 }

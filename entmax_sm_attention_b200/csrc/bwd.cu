@@ -47,6 +47,8 @@ constexpr int kPairBytes = 2 * kTileBytes;   // Q_i and dO_i
 struct Shared {
   uint64_t full[kStages], empty[kStages];
   uint64_t bar_kv, s_full, sda_free, p_ready, mma2_done;
+  uint64_t mma_drain;   // end of kernel: both issuers' MMAs complete
+  uint64_t never;       // self-test: a barrier nothing completes
   uint32_t tmem_base;
   int abort_flag;
   uint32_t qlist[kMaskWords];
@@ -84,7 +86,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
   const Pattern pat{p.L, p.kv_len ? min(max(p.kv_len[b], 1), p.L) : p.L, p.causal, p.window};
   const int j0 = kt * kTile;
   int* status = p.status;
-  volatile int* abrt = &sh.abort_flag;
+  const WaitCtx wc{status, &sh.abort_flag, p.wait_limit_ns};
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -96,6 +98,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     mbar_init(&sh.sda_free, kMathWarps);
     mbar_init(&sh.p_ready, kMathWarps);
     mbar_init(&sh.mma2_done, 2);  // dQ chain and dV/dK chains
+    mbar_init(&sh.mma_drain, 2);
+    mbar_init(&sh.never, 1);
     sh.abort_flag = 0;
     fence_mbar_init();
   }
@@ -106,6 +110,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
   }
   __syncthreads();
   tc_fence_after();
+  const long long clk0 = clock64();
   const uint32_t T = sh.tmem_base;
   uint32_t qlist[kMaskWords];
 #pragma unroll
@@ -122,18 +127,22 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       mbar_expect_tx(&sh.bar_kv, 2 * kTileBytes);
       tma_load_3d(sK, &p.tK, &sh.bar_kv, 0, j0, bh);
       tma_load_3d(sV, &p.tV, &sh.bar_kv, 0, j0, bh);
+      // After a failed wait (abort) no further copy is issued: at most kStages copies,
+      // one per stage, are in flight, and the drain below sees each stage's last one.
       uint32_t seq = 0;
+      bool live = true;
       for_each_bit(qlist, kMaskWords, [&](int it) {
         const int st = seq % kStages;
-        mbar_wait(&sh.empty[st], ((seq / kStages) & 1) ^ 1, status, abrt);
+        live = live && mbar_wait(&sh.empty[st], ((seq / kStages) & 1) ^ 1, wc);
+        if (!live) return;
         mbar_expect_tx(&sh.full[st], kPairBytes);
         tma_load_3d(ring + st * kPairBytes, &p.tQ, &sh.full[st], 0, it * kTile, bh);
         tma_load_3d(ring + st * kPairBytes + kTileBytes, &p.tdO, &sh.full[st], 0, it * kTile, bh);
         ++seq;
       });
-      volatile int no_abort = 0;
+      mbar_drain(&sh.bar_kv, 0, status);
       for (uint32_t k = (seq > kStages ? seq - kStages : 0); k < seq; ++k)
-        mbar_wait(&sh.full[k % kStages], (k / kStages) & 1, status, &no_abort);
+        mbar_drain(&sh.full[k % kStages], (k / kStages) & 1, status);
     }
     __syncwarp();
   } else if (warp == kMmaWarp) {
@@ -146,13 +155,16 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       const uint64_t kM = sdesc_sw128(smem_u32(sK), 8192, 1024);    // K_j as MN-major B (dQ)
       const uint64_t rK = sdesc_sw128(smem_u32(ring), 16, 1024);    // ring stage 0, K-major
       const uint64_t dHd = sdesc_sw128(smem_u32(sdS), 16, 1024), dLd = sdesc_sw128(smem_u32(sdSl), 16, 1024);
-      mbar_wait(&sh.bar_kv, 0, status, abrt);
+      bool live = true;   // false after a failed wait: no further MMA is issued
+      if (p.selftest & kSelftestStall) live = mbar_wait(&sh.never, 0, wc);   // expires: nothing completes it
+      live = live && mbar_wait(&sh.bar_kv, 0, wc);
       // S = Q_s K^T and dA = dO_s V^T into TMEM [0,256).
       auto issue_sda = [&](int s) {
         const int st = s % kStages;
         const uint64_t qd = sdesc_add(rK, st * kPairBytes), od = sdesc_add(qd, kTileBytes);
-        mbar_wait(&sh.full[st], (s / kStages) & 1, status, abrt);
-        if (s > 0) mbar_wait(&sh.sda_free, (s - 1) & 1, status, abrt);   // S, dA of s-1 are in registers
+        live = live && mbar_wait(&sh.full[st], (s / kStages) & 1, wc);
+        if (s > 0) live = live && mbar_wait(&sh.sda_free, (s - 1) & 1, wc);   // S, dA of s-1 are in registers
+        if (!live) return;
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -164,7 +176,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       issue_sda(0);
       for (int s = 0; s < nq; ++s) {
         if (s + 1 < nq) issue_sda(s + 1);   // overlaps the row owners' work on tile s
-        mbar_wait(&sh.p_ready, s & 1, status, abrt);   // A and dS of tile s in shared memory
+        live = live && mbar_wait(&sh.p_ready, s & 1, wc);   // A and dS of tile s in shared memory
+        if (!live) break;
         tc_fence_after();
         const uint32_t dq = T + 384 + (s & 1) * 64;
 #pragma unroll
@@ -191,8 +204,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       for (int s = 0; s < nq; ++s) {
         const int st = s % kStages;
         const uint64_t qM = sdesc_add(rM, st * kPairBytes), oM = sdesc_add(qM, kTileBytes);
-        mbar_wait(&sh.full[st], (s / kStages) & 1, status, abrt);   // Q_s and dO_s landed
-        mbar_wait(&sh.p_ready, s & 1, status, abrt);                // A and dS of tile s written
+        if (!mbar_wait(&sh.full[st], (s / kStages) & 1, wc)) break;   // Q_s and dO_s landed
+        if (!mbar_wait(&sh.p_ready, s & 1, wc)) break;                // A and dS of tile s written
         tc_fence_after();
 #pragma unroll
         for (int t = 0; t < 8; ++t) {
@@ -216,6 +229,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     const float cz = p.cz;
     uint32_t seq = 0;
     int prev_it = -1;
+    long long cyc_s = 0, cyc_mma = 0, cyc_form = 0, cyc_flush = 0;   // first row-owner warp's breakdown
     // Adds dQ of the query tile `it` handled at step `s` (TMEM buffer s % 2) to global
     // memory. The caller has already waited for that step's MMAs. Each thread stages its
     // 16 columns (scaled) in the swizzled box that holds them (one box per 32 of dQ's 64
@@ -252,7 +266,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       const float tau = valid ? p.tau[(size_t)bh * p.L + i] : INFINITY;
       const float dl = valid ? p.delta[(size_t)bh * p.L + i] : 0.f;
       const bool full = pat.block_full(it * kTile, min(p.L, it * kTile + kTile), j0, j0 + kTile);
-      warp_wait(&sh.s_full, seq & 1, status, abrt);
+      const long long c0 = clock64();
+      warp_wait(&sh.s_full, seq & 1, wc);
+      const long long c1 = clock64();
       tc_fence_after();
       uint32_t sr[32], ar[32];
       tmem_ld32(tl + qc * 32, sr);
@@ -261,7 +277,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       tc_fence_before();
       warp_arrive(&sh.sda_free);
       // The previous tile's dV/dK/dQ MMAs must be done reading sA / sdS.
-      if (seq > 0) warp_wait(&sh.mma2_done, (seq - 1) & 1, status, abrt);
+      const long long c2 = clock64();
+      if (seq > 0) warp_wait(&sh.mma2_done, (seq - 1) & 1, wc);
+      const long long c3 = clock64();
       // Keys [32 qc, 32 qc + 32) of row `row`: panel qc/2, 16-byte chunks 4(qc%2)..+3.
       const int pan = (qc >> 1) * kTileBytes;
 #pragma unroll
@@ -296,13 +314,23 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       }
       fence_proxy_async_smem();
       warp_arrive(&sh.p_ready);
+      const long long c4 = clock64();
       if (seq > 0) flush_dq(seq - 1, prev_it);   // its MMAs were waited for above
+      const long long c5 = clock64();
+      cyc_s += c1 - c0;
+      cyc_mma += c3 - c2;
+      cyc_form += (c2 - c1) + (c4 - c3);
+      cyc_flush += c5 - c4;
       prev_it = it;
       ++seq;
     });
     if (seq > 0) {
-      warp_wait(&sh.mma2_done, (seq - 1) & 1, status, abrt);
+      const long long c0 = clock64();
+      warp_wait(&sh.mma2_done, (seq - 1) & 1, wc);
+      const long long c1 = clock64();
       flush_dq(seq - 1, prev_it);
+      cyc_mma += c1 - c0;
+      cyc_flush += clock64() - c1;
     }
     if (tid == 0) bulk_wait_all();   // the last reduce-adds complete before the CTA retires
     // dK and dV of this key tile (TMEM lane = key); each thread writes 16 of the 64
@@ -333,9 +361,21 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
                         sc * __uint_as_float(c[4 * k + 2]), sc * __uint_as_float(c[4 * k + 3]));
       }
     }
+    if (tid == 0) {
+      int4* st = reinterpret_cast<int4*>(p.stats + ((size_t)bh * p.Tc + kt) * kBwdStats);
+      st[0] = make_int4(nq, (int)(clock64() - clk0), (int)cyc_s, (int)cyc_mma);
+      st[1] = make_int4((int)cyc_form, (int)cyc_flush, 0, 0);
+    }
     __syncwarp();
   }
 
+  // No MMA may still write tensor memory when it is freed: both issuers commit once more
+  // and wait for both commits (a drain, bounded and independent of the abort flag).
+  if ((warp == kMmaWarp || warp == kMma2Warp) && lane == 0) {
+    mma_commit(&sh.mma_drain);
+    mbar_drain(&sh.mma_drain, 0, status);
+  }
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == kMmaWarp) tmem_dealloc(T, 512);

@@ -4,8 +4,11 @@
 // shows up in O and, through delta, in dK at the size of the gradient tolerance). The
 // tensor cores need both factors in the same type, so V (for O = A V, Ot = g V) and dO
 // (for dV = A^T dO, dA = dO V^T) get fp16 copies. A bf16 value converts to fp16
-// exactly when |x| <= 65504 and x is not below fp16's subnormal range (2^-24); values
-// outside that range set the status bit kStatusRange.
+// exactly when 2^-14 <= |x| <= 65504 (or x = 0). Only the overflow side is flagged:
+// |x| > 65504 sets the status bit kStatusRange. Below 2^-14 the value lands on fp16's
+// subnormal grid (spacing 2^-24) and below 2^-25 it rounds to zero; either way the
+// absolute error is at most 2^-25, far inside the output and gradient tolerances, so it
+// is not reported.
 #include "common.cuh"
 #include "kernels.h"
 

@@ -79,6 +79,8 @@ struct Shared {
   uint64_t bar_q;
   uint64_t s_full[kSBufs], s_free[kSBufs];     // sweeps: MMA -> rows, rows -> MMA
   uint64_t o_full[kOBufs], o_ready[kOBufs], pv_done[kOBufs];  // output pass, buffer c = k % 3
+  uint64_t mma_drain;                          // end of kernel: every issuer's MMAs complete
+  uint64_t never;                              // self-test: a barrier nothing completes
   uint32_t tmem_base;
   int abort_flag;
   int ctl_kind, ctl_buf;
@@ -261,7 +263,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
   const Pattern pat{p.L, p.kv_len ? min(max(p.kv_len[b], 1), p.L) : p.L, p.causal, p.window};
   const int i0 = qt * kTile, i1 = min(p.L, i0 + kTile);
   int* status = p.status;
-  volatile int* abrt = &sh.abort_flag;
+  const WaitCtx wc{status, &sh.abort_flag, p.wait_limit_ns};
 
   if (tid == 0) {
     for (int s = 0; s < kSlots; ++s) {
@@ -278,6 +280,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       mbar_init(&sh.o_ready[s], kMathWarps);
       mbar_init(&sh.pv_done[s], 2);   // O chain and Ot chain
     }
+    mbar_init(&sh.mma_drain, 3);   // one commit per MMA issuer
+    mbar_init(&sh.never, 1);
     sh.abort_flag = 0;
     fence_mbar_init();
   }
@@ -298,6 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       atomicOr(&sh.act[jt >> 5], 1u << (jt & 31));
   __syncthreads();
   tc_fence_after();
+  const long long clk0 = clock64();
   const uint32_t T = sh.tmem_base;
   uint32_t act[kMaskWords];
 #pragma unroll
@@ -307,10 +312,17 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     // ------------------------------------------------------------------ TMA producer
     // Ring positions are taken in program order: every tile of phase 1 and of each
     // sweep is one K load; the output pass loads K_k, V_k, K_{k+1}, V_{k+1}, ...
+    // After a failed wait (abort) no further copy is issued, so at most kSlots copies,
+    // one per slot, are ever in flight, and the drain below sees each slot's last one.
     uint32_t seq = 0;
+    bool live = true;
     auto load = [&](const CUtensorMap* map, int jt) {
+      if (!live) return;
       const int slot = seq % kSlots;
-      mbar_wait(&sh.empty[slot], ((seq / kSlots) & 1) ^ 1, status, abrt);
+      if (!mbar_wait(&sh.empty[slot], ((seq / kSlots) & 1) ^ 1, wc)) {
+        live = false;
+        return;
+      }
       mbar_expect_tx(&sh.full[slot], kTileBytes);
       tma_load_3d(ring + slot * kTileBytes, map, &sh.full[slot], 0, jt * kTile, bh);
       ++seq;
@@ -345,9 +357,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     }
     // Make sure no copy is still in flight when the CTA retires.
     if (lane == 0) {
-      volatile int no_abort = 0;
+      mbar_drain(&sh.bar_q, 0, status);
       for (uint32_t k = (seq > kSlots ? seq - kSlots : 0); k < seq; ++k)
-        mbar_wait(&sh.full[k % kSlots], (k / kSlots) & 1, status, &no_abort);
+        mbar_drain(&sh.full[k % kSlots], (k / kSlots) & 1, status);
     }
     __syncwarp();
   } else if (warp == kMmaWarp) {
@@ -355,6 +367,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     uint32_t seq = 0;            // next ring position (sweeps consume in order)
     uint32_t sfree_par = 0;      // per sweep S buffer: parity of its uses so far (bit b)
     uint32_t sbuf = 0;           // next sweep S buffer
+    bool live = true;            // false after a failed wait: no further MMA is issued
     const uint32_t idS = idesc_bf16(128, 128, 0, 0);
     const uint64_t qd0 = sdesc_sw128(smem_u32(sQ), 16, 1024);      // Q tile, K-major
     const uint64_t kd0 = sdesc_sw128(smem_u32(ring), 16, 1024);    // ring slot 0, K-major
@@ -372,15 +385,18 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       const uint32_t bf = sbuf;
       const uint32_t pos = seq++;
       // S buffer consumed by the row owners, and K tile landed.
-      mbar_wait2(&sh.s_free[bf], ((sfree_par >> bf) & 1) ^ 1, &sh.full[pos % kSlots], (pos / kSlots) & 1, status,
-                 abrt);
+      live = live && mbar_wait2(&sh.s_free[bf], ((sfree_par >> bf) & 1) ^ 1, &sh.full[pos % kSlots],
+                                (pos / kSlots) & 1, wc);
       sfree_par ^= 1u << bf;
-      mma_s(pos, bf * 128);
-      mma_commit(&sh.s_full[bf]);
+      if (live) {
+        mma_s(pos, bf * 128);
+        mma_commit(&sh.s_full[bf]);
+      }
       sbuf = (sbuf + 1) & (kSBufs - 1);
     };
     if (lane == 0) {
-      mbar_wait(&sh.bar_q, 0, status, abrt);
+      if (p.selftest & kSelftestStall) live = mbar_wait(&sh.never, 0, wc);   // expires: nothing completes it
+      live = live && mbar_wait(&sh.bar_q, 0, wc);
       for_each_bit(act, kMaskWords, [&](int) { sweep_tile(); });
     }
     __syncwarp();
@@ -406,10 +422,11 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
             const int c = k % kOBufs;
             const uint32_t pos = base + 2 * k;
             if (k >= kOBufs)
-              mbar_wait2(&sh.pv_done[c], ((k - kOBufs) / kOBufs) & 1, &sh.full[pos % kSlots], (pos / kSlots) & 1,
-                         status, abrt);
+              live = live && mbar_wait2(&sh.pv_done[c], ((k - kOBufs) / kOBufs) & 1, &sh.full[pos % kSlots],
+                                        (pos / kSlots) & 1, wc);
             else
-              mbar_wait(&sh.full[pos % kSlots], (pos / kSlots) & 1, status, abrt);
+              live = live && mbar_wait(&sh.full[pos % kSlots], (pos / kSlots) & 1, wc);
+            if (!live) break;
             mma_s(pos, c == 0 ? 0u : (c == 1 ? 128u : 384u));
             mma_commit(&sh.o_full[c]);
           }
@@ -443,7 +460,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           const uint32_t pa = c == 0 ? 0u : (c == 1 ? 128u : 384u);
           const uint32_t vpos = base + 2 * k + 1;
           const int vslot = vpos % kSlots;
-          mbar_wait2(&sh.full[vslot], (vpos / kSlots) & 1, &sh.o_ready[c], (k / kOBufs) & 1, status, abrt);
+          if (!mbar_wait2(&sh.full[vslot], (vpos / kSlots) & 1, &sh.o_ready[c], (k / kOBufs) & 1, wc)) break;
           tc_fence_after();
           const uint64_t vd = sdesc_add(vd0, vslot * kTileBytes);
 #pragma unroll
@@ -483,7 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           const uint32_t pa = c == 0 ? 0u : (c == 1 ? 128u : 384u);
           const uint32_t vpos = base + 2 * k + 1;
           const int vslot = vpos % kSlots;
-          mbar_wait2(&sh.full[vslot], (vpos / kSlots) & 1, &sh.o_ready[c], (k / kOBufs) & 1, status, abrt);
+          if (!mbar_wait2(&sh.full[vslot], (vpos / kSlots) & 1, &sh.o_ready[c], (k / kOBufs) & 1, wc)) break;
           tc_fence_after();
           const uint64_t vd = sdesc_add(vd0, vslot * kTileBytes);
 #pragma unroll
@@ -514,7 +531,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     // Phase 1: per-key-tile row maxima over this thread's column part (combined in smem).
     for_each_bit(act, kMaskWords, [&](int jt) {
       const uint32_t bf = sbuf;
-      warp_wait(&sh.s_full[bf], (sfull_par >> bf) & 1, status, abrt);
+      warp_wait(&sh.s_full[bf], (sfull_par >> bf) & 1, wc);
       sfull_par ^= 1u << bf;
       tc_fence_after();
       const int j0 = jt * kTile + qp * kCols;
@@ -554,6 +571,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
 #pragma unroll
     for (int k = 0; k < 4 * kParts; ++k) vt[k] = part[k * kTile + row];
     named_bar(3, kMathThreads);   // read before anyone rewrites the partials
+    const long long clk1 = clock64();
+    long long clk2 = clk1;
 #pragma unroll
     for (int q = 0; q < kParts; ++q) m = fmaxf(m, vt[4 * q]);
 
@@ -614,6 +633,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       named_bar(1, kThreads);
 
       if (final_mask) {
+        clk2 = clock64();
         if (!done && qp == 0) atomicOr(status, kStatusNoConverge);   // cap reached; tau stays bracketed
         // Block mask row of this query tile and the transposed bits (Appendix C.4).
         if (tid < p.Wc) p.M[((size_t)bh * p.Tr + qt) * p.Wc + tid] = list[tid];
@@ -627,7 +647,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         for_each_bit(list, kMaskWords, [&](int jt) {
           const int c = k % kOBufs;
           const uint32_t pa = c == 0 ? 0u : (c == 1 ? 128u : 384u);
-          warp_wait(&sh.o_full[c], (k / kOBufs) & 1, status, abrt);
+          warp_wait(&sh.o_full[c], (k / kOBufs) & 1, wc);
           tc_fence_after();
           const int j0 = jt * kTile + qp * kCols;
           float s[kCols];
@@ -672,7 +692,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         });
         const int n_out = k;
         // Epilogue: O and Ot from TMEM (each thread of a row writes kOCols of the 64 columns).
-        warp_wait(&sh.pv_done[(n_out - 1) % kOBufs], ((n_out - 1) / kOBufs) & 1, status, abrt);
+        if (n_out > 0) warp_wait(&sh.pv_done[(n_out - 1) % kOBufs], ((n_out - 1) / kOBufs) & 1, wc);
         tc_fence_after();
         part[(qp * 4 + 1) * kTile + row] = sg2.x + sg2.y;
         uint32_t o[kOCols];
@@ -704,8 +724,10 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         if (tid == 0) {
           int na = 0;
           for (int w = 0; w < kMaskWords; ++w) na += __popc(act[w]);
-          int4* st = reinterpret_cast<int4*>(p.stats) + (size_t)bh * p.Tr + qt;
-          *st = make_int4(sweeps, (int)n_s, n_out, na);
+          const long long clk3 = clock64();
+          int4* st = reinterpret_cast<int4*>(p.stats + ((size_t)bh * p.Tr + qt) * kFwdStats);
+          st[0] = make_int4(sweeps, (int)n_s, n_out, na);
+          st[1] = make_int4((int)(clk1 - clk0), (int)(clk2 - clk1), (int)(clk3 - clk2), (int)(clk3 - clk0));
         }
         break;
       }
@@ -718,7 +740,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       sbuf = 0;
       for_each_bit(list, kMaskWords, [&](int jt) {
         const uint32_t bf = sbuf;
-        warp_wait(&sh.s_full[bf], (sfull_par >> bf) & 1, status, abrt);
+        warp_wait(&sh.s_full[bf], (sfull_par >> bf) & 1, wc);
         sfull_par ^= 1u << bf;
         tc_fence_after();
         const int j0 = jt * kTile + qp * kCols;
@@ -828,6 +850,13 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     }
   }
 
+  // No MMA may still write tensor memory when it is freed: each issuer commits once more
+  // and waits for all three commits (a drain, bounded and independent of the abort flag).
+  if ((warp == kMmaWarp || warp == kMma2Warp || warp == kMma3Warp) && lane == 0) {
+    mma_commit(&sh.mma_drain);
+    mbar_drain(&sh.mma_drain, 0, status);
+  }
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == kMmaWarp) tmem_dealloc(T, 512);

@@ -261,7 +261,9 @@ __global__ void __launch_bounds__(kThreads32) fwd_f32_kernel(const FwdF32Params 
       na += __popc(a[w]);
       nflag += __popc(f[w]);
     }
-    reinterpret_cast<int4*>(p.stats)[(size_t)bh * p.Tr + qt] = make_int4(sweeps, 0, nflag, na);
+    int4* st = reinterpret_cast<int4*>(p.stats + ((size_t)bh * p.Tr + qt) * kFwdStats);
+    st[0] = make_int4(sweeps, 0, nflag, na);
+    st[1] = make_int4(0, 0, 0, 0);   // no phase timing on this path
   }
 }
 

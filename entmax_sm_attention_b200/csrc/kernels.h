@@ -6,6 +6,20 @@
 
 namespace entmax {
 
+// Per-query-tile counters written by the forward kernels (int32 each):
+//   0 refinement sweeps, 1 S = Q K^T tiles computed (all passes), 2 flagged key tiles
+//   (output pass), 3 structurally active key tiles, then SM clock cycles (clock64
+//   differences) of 4 the max pass, 5 threshold refinement and mask decision, 6 the output
+//   pass and epilogue, 7 the whole CTA.
+constexpr int kFwdStats = 8;
+// Per-key-tile counters of the backward kernel: 0 flagged query tiles visited, then cycles
+// of 1 the whole CTA, and, for the first row-owner warp, 2 waiting for S and dA, 3 waiting
+// for the previous tile's gradient MMAs, 4 forming A and dS, 5 staging dQ (reduce-add).
+constexpr int kBwdStats = 8;
+// Self-test switch: every CTA makes one bounded wait on an mbarrier that nothing
+// completes, so the wait expires and the abort path runs.
+constexpr int kSelftestStall = 1;
+
 struct FwdParams {
   CUtensorMap tQ, tK, tV;   // [B*H][L][64], box 64 x 128 x 1, 128-byte swizzle (Q, K bf16; V fp16)
   float* O;                 // [B*H][L][64]
@@ -14,12 +28,14 @@ struct FwdParams {
   float* Ot;                // [B*H][L][64]  sum_j g_ij V_j
   uint32_t* M;              // [B*H][Tr][Wc]
   uint32_t* MT;             // [B*H][Tc][Wr] (zeroed before the launch)
-  int* stats;               // [B*H][Tr][4]: sweeps, S tiles computed, flagged tiles, active tiles
+  int* stats;               // [B*H][Tr][kFwdStats] (layout above)
   int* status;
   const int* kv_len;        // [B] or nullptr
   int H, L, Tr, Tc, Wc, Wr, BH;
   float cz;                 // (alpha - 1) * scale
   int causal, window, max_sweeps;
+  unsigned long long wait_limit_ns;   // bound on every in-kernel wait
+  int selftest;             // kSelftestStall: one wait per CTA on a barrier nothing completes
 };
 
 struct BwdParams {
@@ -32,11 +48,14 @@ struct BwdParams {
   float* dK;
   float* dV;
   int* status;
+  int* stats;                    // [B*H][Tc][kBwdStats] (layout above)
   const int* kv_len;
   int H, L, Tr, Tc, Wr, BH;
   float cz;                      // (alpha - 1) * scale
   float scale;
   int causal, window;
+  unsigned long long wait_limit_ns;
+  int selftest;
 };
 
 struct FwdF32Params {
@@ -47,7 +66,7 @@ struct FwdF32Params {
   float* tau;
   uint32_t* M;
   uint32_t* MT;
-  int* stats;
+  int* stats;               // [B*H][Tr][kFwdStats]
   int* status;
   const int* kv_len;
   int H, L, Tr, Tc, Wc, Wr, BH;
@@ -65,7 +84,11 @@ cudaError_t launch_bwd(bool alpha15, const BwdParams& p, int grid, cudaStream_t 
 cudaError_t launch_bf16_to_f16(const void* src, void* dst, long elems, int* status, cudaStream_t s);
 cudaError_t launch_delta(const uint16_t* dO, const float* Ot, const float* sumg, float* delta, long rows,
                          cudaStream_t s);
-cudaError_t launch_rows(bool alpha15, const float* S, int rows, int n, long ld, float* P, float* tau,
+cudaError_t launch_rows(bool alpha15, const float* S, int rows, int n, long ld, float* P, float* tau, int* status,
                         cudaStream_t s);
+
+// Device address of the no-allocation forward's static scratch on the current device
+// (looked up on first use per device), or nullptr on failure.
+void* noalloc_scratch();
 
 }  // namespace entmax

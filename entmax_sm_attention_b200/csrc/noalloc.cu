@@ -13,6 +13,11 @@
 #include <mutex>
 
 #include "../../include/entmax_attn.h"
+#include "kernels.h"
+
+namespace entmax {
+size_t fwd_workspace_bytes(const entmax_attn_desc* d);   // abi.cu: the forward's part of the workspace
+}
 
 namespace {
 
@@ -44,9 +49,15 @@ void* scratch_for_current_device() {
 
 }  // namespace
 
+namespace entmax {
+void* noalloc_scratch() { return scratch_for_current_device(); }
+}  // namespace entmax
+
 extern "C" entmax_status entmax_attn_fwd_noalloc(const entmax_attn_desc* desc, const void* Q, const void* K,
                                                  const void* V, float* O, float* tau, void* stream) {
-  const size_t need = entmax_attn_workspace_bytes(desc);
+  // Only the forward's part of the workspace is needed (status, masks, counters, sum g,
+  // Ot and the fp16 copy of V); the backward-only parts come after it in the layout.
+  const size_t need = entmax::fwd_workspace_bytes(desc);
   if (need == 0) return ENTMAX_EINVAL;
   if (need > (size_t)ENTMAX_NOALLOC_SCRATCH_BYTES) return ENTMAX_EUNSUPPORTED;   // problem too large
   void* scratch = scratch_for_current_device();

@@ -14,6 +14,10 @@
 //     leaves the support, so it is tau* and the solve ends.
 //   - otherwise a Newton step on Eq. 4, clamped to the bracket, with bisection as the
 //     fallback.
+// Rows of up to kRowsSmem scores are staged once in shared memory, so the iterations
+// read them there; longer rows are re-read from global memory (L2) on each iteration.
+// A row that reaches the iteration cap keeps tau inside the bracket and sets bit 0 of the
+// optional status word.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -21,6 +25,8 @@ namespace entmax {
 
 namespace {
 constexpr int kRowThreads = 256;
+constexpr int kRowsSmem = 16384;   // longest row staged in shared memory (64 KB)
+constexpr int kRowIters = 100;
 
 struct Red {
   float s1, s2, c, umin;
@@ -49,9 +55,16 @@ __device__ Red block_reduce(Red v, Red* buf) {
 
 template <int AK>
 __global__ void __launch_bounds__(kRowThreads) rows_kernel(const float* __restrict__ S, int n, long ld,
-                                                            float* __restrict__ P, float* __restrict__ tau_out) {
+                                                            float* __restrict__ P, float* __restrict__ tau_out,
+                                                            int* status) {
   __shared__ Red buf[kRowThreads / 32];
+  extern __shared__ float srow[];
   const float* x = S + (long)blockIdx.x * ld;
+  if (n <= kRowsSmem) {
+    for (int j = threadIdx.x; j < n; j += kRowThreads) srow[j] = x[j];
+    __syncthreads();
+    x = srow;
+  }
   const float c = (AK == kAlpha15) ? 0.5f : 1.0f;   // alpha - 1
 
   // Row max (-inf entries are inactive) and active count.
@@ -83,7 +96,8 @@ __global__ void __launch_bounds__(kRowThreads) rows_kernel(const float* __restri
   float lo = mz - 1.f;
   float hi = mz - ((AK == kAlpha15) ? rsqrtf(n_act) : 1.f / n_act);
   float t = lo;
-  for (int it = 0; it < 100; ++it) {
+  bool settled = false;
+  for (int it = 0; it < kRowIters; ++it) {
     Red v{0.f, 0.f, 0.f, INFINITY};
     for (int j = threadIdx.x; j < n; j += kRowThreads) {
       const float u = fmaf(x[j], c, -t);
@@ -107,11 +121,13 @@ __global__ void __launch_bounds__(kRowThreads) rows_kernel(const float* __restri
       }
       if (d >= 0.f && d < r.umin) {   // support unchanged at t + d: exact root
         t += d;
+        settled = true;
         break;
       }
     }
     if (fabsf(f) <= 1e-7f && fp > 0.f) {
       t += f / fp;
+      settled = true;
       break;
     }
     if (f > 0.f) lo = t; else hi = t;
@@ -119,7 +135,10 @@ __global__ void __launch_bounds__(kRowThreads) rows_kernel(const float* __restri
     if (!(tn > lo && tn <= hi && tn != t)) tn = 0.5f * (lo + hi);   // the root may sit at hi (uniform scores); a stalled step bisects
     t = tn;
   }
-  if (threadIdx.x == 0) tau_out[blockIdx.x] = t;
+  if (threadIdx.x == 0) {
+    tau_out[blockIdx.x] = t;
+    if (!settled && status) atomicOr(status, kStatusNoConverge);
+  }
   float* out = P + (long)blockIdx.x * ld;
   for (int j = threadIdx.x; j < n; j += kRowThreads) {
     const float u = fmaxf(fmaf(x[j], c, -t), 0.f);
@@ -127,12 +146,13 @@ __global__ void __launch_bounds__(kRowThreads) rows_kernel(const float* __restri
   }
 }
 
-cudaError_t launch_rows(bool alpha15, const float* S, int rows, int n, long ld, float* P, float* tau,
+cudaError_t launch_rows(bool alpha15, const float* S, int rows, int n, long ld, float* P, float* tau, int* status,
                         cudaStream_t s) {
-  if (alpha15)
-    rows_kernel<kAlpha15><<<rows, kRowThreads, 0, s>>>(S, n, ld, P, tau);
-  else
-    rows_kernel<kAlpha2><<<rows, kRowThreads, 0, s>>>(S, n, ld, P, tau);
+  const int smem = n <= kRowsSmem ? n * 4 : 0;
+  auto kern = alpha15 ? rows_kernel<kAlpha15> : rows_kernel<kAlpha2>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kRowsSmem * 4);
+  if (e != cudaSuccess) return e;
+  kern<<<rows, kRowThreads, smem, s>>>(S, n, ld, P, tau, status);
   return cudaGetLastError();
 }
 

@@ -15,15 +15,27 @@
 
 namespace entmax {
 
-// Every mbarrier wait is bounded in wall time (kWaitLimitNs of %globaltimer; a healthy
-// wait finishes in microseconds). On expiry the wait sets bit 1 of the device status
-// word and raises the CTA's abort flag, so later waits return at once; callers keep
-// going through the kernel's control flow so that no thread is left at a CTA barrier
-// and tensor memory is still freed.
+// Every mbarrier wait is bounded in wall time. The bound comes with the launch (WaitCtx;
+// by default kWaitLimitNs of %globaltimer, while a healthy wait ends in microseconds). On
+// expiry the wait sets bit 1 of the device status word and raises the CTA's abort flag,
+// so later waits return at once. After an abort the TMA producer issues no further copy
+// and the MMA issuers no further MMA; every role still runs through the kernel's control
+// flow, so no thread is left at a CTA barrier, and tensor memory is freed at the end.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+// End-of-kernel drains (copies or MMAs already issued, which finish in microseconds) use
+// this bound and ignore the abort flag.
+constexpr unsigned long long kDrainLimitNs = 2000000000ull;
 constexpr int kStatusNoConverge = 1;
 constexpr int kStatusTimeout = 2;
 constexpr int kStatusRange = 4;   // a bf16 input outside the fp16 range (|x| > 65504)
+
+// Wait bookkeeping of one CTA: the device status word (may be null), the CTA's abort flag
+// in shared memory, and the wait bound of this launch.
+struct WaitCtx {
+  int* status;
+  volatile int* abort;
+  unsigned long long limit_ns;
+};
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -63,20 +75,28 @@ __device__ __forceinline__ unsigned long long globaltimer_ns() {
   return t;
 }
 // Wait for phase `parity` of `bar` to complete, bounded. Returns false, flags the status
-// word and sets *abort if the budget runs out; returns false at once if *abort is set.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status, volatile int* abort) {
+// word and sets the abort flag if the bound runs out; returns false at once if the abort
+// flag is set.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
   while (true) {
-    if (*abort) return false;
+    if (*w.abort) return false;
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
-      *abort = 1;
-      if (status) atomicOr(status, kStatusTimeout);
+    if (globaltimer_ns() - t0 > w.limit_ns) {
+      *w.abort = 1;
+      if (w.status) atomicOr(w.status, kStatusTimeout);
       return false;
     }
   }
+}
+// Wait for work already issued to finish (a drain at the end of a kernel): bounded by
+// kDrainLimitNs, and independent of the abort flag. Returns false if the bound ran out.
+__device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity, int* status) {
+  volatile int no_abort = 0;
+  const WaitCtx w{status, &no_abort, kDrainLimitNs};
+  return mbar_wait(bar, parity, w);
 }
 
 // Non-blocking probe of a phase (mbarrier.test_wait): the thread is never suspended, so
@@ -94,13 +114,13 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
 }
 // Waits for phase p1 of b1 and phase p2 of b2: both are probed back to back first; the
 // bounded waits run only if a phase is still open.
-__device__ __forceinline__ bool mbar_wait2(uint64_t* b1, uint32_t p1, uint64_t* b2, uint32_t p2, int* status,
-                                           volatile int* abort) {
+__device__ __forceinline__ bool mbar_wait2(uint64_t* b1, uint32_t p1, uint64_t* b2, uint32_t p2,
+                                           const WaitCtx& w) {
   const bool r1 = mbar_test_wait(b1, p1);
   const bool r2 = mbar_test_wait(b2, p2);
   if (r1 && r2) return true;
-  const bool w1 = mbar_wait(b1, p1, status, abort);
-  const bool w2 = mbar_wait(b2, p2, status, abort);
+  const bool w1 = mbar_wait(b1, p1, w);
+  const bool w2 = mbar_wait(b2, p2, w);
   return w1 && w2;
 }
 
@@ -112,10 +132,10 @@ __device__ __forceinline__ bool mbar_wait2(uint64_t* b1, uint32_t p1, uint64_t* 
 // reconverges the warp before the .sync.aligned tcgen05 instructions and bar.sync that
 // follow, and makes the barrier's completion (and the memory it guards) visible to every
 // lane.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, int* status, volatile int* abort) {
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
   if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
   int ok = 1;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, status, abort) ? 1 : 0;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, w) ? 1 : 0;
   __syncwarp();
   ok = __shfl_sync(0xffffffffu, ok, 0);
   return ok != 0;

@@ -28,8 +28,11 @@
  *   - Layout: Q, K, V, dO, O, dQ, dK, dV are contiguous row-major [B, H, L, d] (one
  *     64-element row per token); tau is [B, H, L]. All are device pointers.
  *   - Ownership: the caller allocates and frees all memory, the workspace included.
- *     The library never allocates, frees or keeps device memory, and holds no global
- *     state beyond cached kernel attributes.
+ *     The library never allocates or frees device memory. It keeps one piece of device
+ *     memory and global state: the ENTMAX_NOALLOC_SCRATCH_BYTES scratch array of
+ *     entmax_attn_fwd_noalloc, present on every GPU that loads the library until the
+ *     process exits (with its device address, cached per device), plus a cached driver
+ *     entry point.
  *   - Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream). All device work is enqueued on it. No call synchronises except
  *     entmax_last_device_status.
@@ -38,6 +41,11 @@
  *     ENTMAX_ECUDA. Conditions found on the device (solver cap reached, a bounded wait
  *     that expired) are recorded in the workspace status word and read back with
  *     entmax_last_device_status. Nothing throws across the ABI.
+ *   - Bounded waits: every wait inside a kernel (pipeline barriers between the copy,
+ *     tensor-core and row roles) gives up after desc->wait_limit_us (default 2 s). The
+ *     CTA then issues no further copy or MMA, finishes its control flow, frees its
+ *     tensor memory and records ENTMAX_ETIMEOUT; the results of that call are undefined,
+ *     and the CUDA context stays usable.
  *   - Non-finite inputs give undefined results. The probability-side products (O = A V,
  *     Ot = g V, dV = A^T dO, dA = dO V^T) run in fp16, so bf16 V and dO must lie within
  *     the fp16 range (|x| <= 65504); a value outside it sets ENTMAX_ERANGE.
@@ -77,7 +85,16 @@ typedef struct {
                              rows at or past kv_len.                                      */
     entmax_dtype dtype;   /* dtype of Q, K, V (and dO). ENTMAX_FP32 is forward-only.      */
     int max_sweeps;       /* cap on threshold-refinement passes; 0 = library default (12) */
+    int wait_limit_us;    /* bound on each in-kernel wait in microseconds; 0 = 2 s.
+                             Must be >= 0.                                                 */
+    int selftest;         /* 0 for normal use. ENTMAX_SELFTEST_STALL makes one thread of
+                             every CTA of the fwd/bwd kernels wait on a barrier that
+                             nothing completes, so that the wait expires after
+                             wait_limit_us and the call reports ENTMAX_ETIMEOUT: a test of
+                             the failure path that faults and hangs nothing.              */
 } entmax_attn_desc;
+
+#define ENTMAX_SELFTEST_STALL 1
 
 #define ENTMAX_MAX_L 16384   /* longest supported sequence (the per-row tile maxima live
                                 in shared memory, 4 bytes per key tile per row)           */
@@ -85,10 +102,10 @@ typedef struct {
 
 /* Bytes of device workspace needed by entmax_attn_fwd / entmax_attn_bwd for *desc.
  * The workspace holds the status word, the block mask M and its transpose M^T, the
- * per-row sum_j g_ij and Ot_i = sum_j g_ij V_j, delta_i, per-tile counters and fp16
- * copies of V and dO. Returns 0 for an invalid
- * descriptor. The base address must be 256-byte aligned; the fwd -> bwd pair must use
- * the same workspace, and the caller keeps it alive in between. */
+ * per-row sum_j g_ij and Ot_i = sum_j g_ij V_j, delta_i, per-tile counters of both
+ * passes and fp16 copies of V and dO. Returns 0 for an invalid descriptor. The base
+ * address must be 256-byte aligned; the fwd -> bwd pair must use the same workspace,
+ * and the caller keeps it alive in between. */
 size_t entmax_attn_workspace_bytes(const entmax_attn_desc *desc);
 
 /* Forward (AdaSplash-2 §3.3 Phases 1-4).
@@ -112,29 +129,40 @@ entmax_status entmax_attn_bwd(const entmax_attn_desc *desc, const void *Q, const
  * study works on such score vectors). Row r holds S[r*ld + j], j < n. Scores of -inf
  * are inactive; every row needs at least one finite score.
  * Out: P[r*ld + j] = [(alpha-1) S - tau_r]_+^{1/(alpha-1)} and tau[r] (Eq. 3 units).
+ * status: a device int32 or NULL. When a row reaches the solver's iteration cap (its tau
+ * then stays inside the §2.4 bracket) the kernel ORs 1 into it; the caller zeroes it
+ * beforehand and reads it after the stream has finished.
  * Constraints: rows >= 0, 1 <= n <= ld, 16-byte-aligned S and P, ld % 4 == 0,
  * alpha in {1.5, 2}. rows == 0 is a no-op. */
 entmax_status entmax_rows(const float *S, int rows, int n, int ld, float alpha, float *P,
-                          float *tau, void *stream);
+                          float *tau, int *status, void *stream);
 
 /* Synchronises `stream`, then reads the workspace status word left by the last
  * fwd/bwd: ENTMAX_OK, ENTMAX_ENOCONVERGE, ENTMAX_ETIMEOUT or ENTMAX_ERANGE. *status_out receives the
  * raw word: bit 0 = no convergence, bit 1 = wait timeout, bit 2 = a V or dO value outside
- * the fp16 range (ENTMAX_ERANGE; the results of that call are then undefined). */
+ * the fp16 range (ENTMAX_ERANGE; the results of that call are then undefined).
+ * workspace == NULL reads the status word of entmax_attn_fwd_noalloc's scratch on the
+ * current device instead (the last no-allocation forward on that device). */
 entmax_status entmax_last_device_status(const entmax_attn_desc *desc, const void *workspace,
                                         int *status_out, void *stream);
 
-/* Copies the forward's packed block mask and per-tile counters out of the workspace,
- * device to device, on `stream`.
+/* Copies the forward's packed block mask and the per-tile counters of both passes out of
+ * the workspace, device to device, on `stream`.
  *   - M is uint32 [B, H, Tr, ceil(Tc/32)], with Tr = Tc = ceil(L/128). Bit (jt % 32)
  *     of word jt/32 is set when some row of query tile it has a nonzero weight in key
  *     tile jt (Appendix C.4).
- *   - stats is int32 [B, H, Tr, 4]. Per query tile it holds: the refinement passes
- *     used, the S = Q K^T tiles computed (all passes), the flagged key tiles (the
- *     output pass), and the structurally active key tiles.
- * Either output may be NULL. */
+ *   - stats is int32 [B, H, Tr, 8]. Per query tile of the last forward: the refinement
+ *     passes used, the S = Q K^T tiles computed (all passes), the flagged key tiles
+ *     (the output pass), the structurally active key tiles; then SM clock cycles of the
+ *     CTA in the max pass, in threshold refinement and the mask decision, in the output
+ *     pass with its epilogue, and in total. (The fp32 forward leaves the cycles at 0.)
+ *   - bwd_stats is int32 [B, H, Tc, 8]. Per key tile of the last backward: the flagged
+ *     query tiles visited, the CTA's cycles in total, then the first row-owner warp's
+ *     cycles waiting for S and dA, waiting for the previous tile's gradient MMAs,
+ *     forming A and dS, and staging dQ for its reduce-add; two zero words.
+ * Any output may be NULL. */
 entmax_status entmax_attn_block_mask(const entmax_attn_desc *desc, const void *workspace,
-                                     uint32_t *M, int *stats, void *stream);
+                                     uint32_t *M, int *stats, int *bwd_stats, void *stream);
 
 /* Forward for callers that cannot allocate device memory. Some callers are handed
  * only their input and output buffers: a plugin inside a host framework that owns
@@ -144,9 +172,10 @@ entmax_status entmax_attn_block_mask(const entmax_attn_desc *desc, const void *w
  * minus the workspace. Its scratch is a fixed array of ENTMAX_NOALLOC_SCRATCH_BYTES
  * that the library keeps on every GPU that loads it, until the process exits.
  * The paper has no counterpart to this entry point; it exists for deployment only.
- *   - Limit: entmax_attn_workspace_bytes(desc) must not exceed
- *     ENTMAX_NOALLOC_SCRATCH_BYTES (16 MiB, roughly B*H*L <= 32000 rows). A larger
- *     problem returns ENTMAX_EUNSUPPORTED before anything is launched.
+ *   - Limit: the forward's part of the workspace (status word, block masks, per-tile
+ *     counters, and per row sum g, Ot and the fp16 copy of V: about 388 bytes per row)
+ *     must fit in ENTMAX_NOALLOC_SCRATCH_BYTES (16 MiB, roughly B*H*L <= 43000 rows).
+ *     A larger problem returns ENTMAX_EUNSUPPORTED before anything is launched.
  *   - Allocates nothing: no cudaMalloc, no cudaFree, no allocating library routine.
  *   - The first call on a device looks up the device address of the scratch array
  *     while that device is current. Make that first call before any stream capture.
@@ -154,8 +183,9 @@ entmax_status entmax_attn_block_mask(const entmax_attn_desc *desc, const void *w
  *     call's contents. Each call clears the parts that must start at zero. Calls whose
  *     GPU work overlaps (different streams, or host threads without ordering) race on
  *     the array and give undefined results, so serialise them.
- *   - Forward only: no workspace remains to pass to entmax_attn_bwd, and
- *     entmax_last_device_status / entmax_attn_block_mask cannot see this scratch. */
+ *   - Forward only: no workspace remains to pass to entmax_attn_bwd. The status word of
+ *     the last call on a device (no convergence, wait timeout, fp16 range) is read with
+ *     entmax_last_device_status(desc, NULL, &word, stream). */
 #define ENTMAX_NOALLOC_SCRATCH_BYTES (16u << 20)
 entmax_status entmax_attn_fwd_noalloc(const entmax_attn_desc *desc, const void *Q, const void *K,
                                       const void *V, float *O, float *tau, void *stream);

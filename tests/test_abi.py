@@ -42,10 +42,11 @@ def test_library_exports_every_declared_symbol(lib):
 
 def _desc(**kw):
     base = dict(B=1, H=2, L=300, d=64, alpha=1.5, scale=0.125, causal=0, window=-1, kv_len=None,
-                dtype=eb.ENTMAX_BF16, max_sweeps=0)
+                dtype=eb.ENTMAX_BF16, max_sweeps=0, wait_limit_us=0, selftest=0)
     base.update(kw)
     return eb.AttnDesc(base["B"], base["H"], base["L"], base["d"], base["alpha"], base["scale"], base["causal"],
-                       base["window"], base["kv_len"], base["dtype"], base["max_sweeps"])
+                       base["window"], base["kv_len"], base["dtype"], base["max_sweeps"], base["wait_limit_us"],
+                       base["selftest"])
 
 
 def test_workspace_bytes_valid_and_invalid(lib):
@@ -54,7 +55,8 @@ def test_workspace_bytes_valid_and_invalid(lib):
     # grows with L
     assert lib.entmax_attn_workspace_bytes(ctypes.byref(_desc(L=4096))) > n
     for bad in (dict(B=0), dict(L=0), dict(d=32), dict(alpha=1.25), dict(scale=0.0), dict(causal=2),
-                dict(max_sweeps=-1), dict(max_sweeps=65), dict(L=eb.ENTMAX_MAX_L + 1), dict(dtype=7)):
+                dict(max_sweeps=-1), dict(max_sweeps=65), dict(L=eb.ENTMAX_MAX_L + 1), dict(dtype=7),
+                dict(wait_limit_us=-1), dict(selftest=2)):
         assert lib.entmax_attn_workspace_bytes(ctypes.byref(_desc(**bad))) == 0, bad
 
 
@@ -66,6 +68,8 @@ def test_workspace_bytes_valid_and_invalid(lib):
     (dict(B=-1), eb.ENTMAX_EINVAL),
     (dict(scale=float("nan")), eb.ENTMAX_EINVAL),
     (dict(max_sweeps=100), eb.ENTMAX_EINVAL),
+    (dict(wait_limit_us=-5), eb.ENTMAX_EINVAL),
+    (dict(selftest=3), eb.ENTMAX_EINVAL),
 ])
 def test_forward_rejects_on_host(lib, bad, code):
     d = _desc(**bad)
@@ -89,9 +93,12 @@ def test_null_and_misaligned_pointers_rejected(lib):
 
 def test_rows_rejects_on_host(lib):
     p = ctypes.c_void_p(1 << 20)
-    assert lib.entmax_rows(p, 4, 0, 4, ctypes.c_float(1.5), p, p, None) == eb.ENTMAX_EINVAL   # n = 0
-    assert lib.entmax_rows(p, 4, 8, 6, ctypes.c_float(1.5), p, p, None) == eb.ENTMAX_EINVAL   # ld % 4
-    assert lib.entmax_rows(p, 4, 8, 4, ctypes.c_float(1.5), p, p, None) == eb.ENTMAX_EINVAL   # ld < n
-    assert lib.entmax_rows(p, 4, 8, 8, ctypes.c_float(1.2), p, p, None) == eb.ENTMAX_EUNSUPPORTED
-    assert lib.entmax_rows(p, -1, 8, 8, ctypes.c_float(1.5), p, p, None) == eb.ENTMAX_EINVAL
-    assert lib.entmax_rows(p, 0, 8, 8, ctypes.c_float(1.5), p, p, None) == eb.ENTMAX_OK      # empty: no-op
+    odd = ctypes.c_void_p((1 << 20) + 2)
+    f15 = ctypes.c_float(1.5)
+    assert lib.entmax_rows(p, 4, 0, 4, f15, p, p, None, None) == eb.ENTMAX_EINVAL   # n = 0
+    assert lib.entmax_rows(p, 4, 8, 6, f15, p, p, None, None) == eb.ENTMAX_EINVAL   # ld % 4
+    assert lib.entmax_rows(p, 4, 8, 4, f15, p, p, None, None) == eb.ENTMAX_EINVAL   # ld < n
+    assert lib.entmax_rows(p, 4, 8, 8, ctypes.c_float(1.2), p, p, None, None) == eb.ENTMAX_EUNSUPPORTED
+    assert lib.entmax_rows(p, -1, 8, 8, f15, p, p, None, None) == eb.ENTMAX_EINVAL
+    assert lib.entmax_rows(p, 4, 8, 8, f15, p, p, odd, None) == eb.ENTMAX_EINVAL     # misaligned status
+    assert lib.entmax_rows(p, 0, 8, 8, f15, p, p, None, None) == eb.ENTMAX_OK      # empty: no-op

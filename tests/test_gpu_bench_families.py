@@ -1,0 +1,74 @@
+"""Every input family bench.py times, checked against the fp64 oracle at its bench shape.
+
+bench.py times the long causal workload (L = 8192, d = 64, bf16) on two families beyond
+the headline inputs:
+  - iid Gaussian inputs with query scale sigma_Q in {1, 3, 8, 24} (AdaSplash-2 §4.2
+    sets sparsity through the query variance);
+  - planted block structure with rho in {1, 1/2, 1/4, 1/8, 1/16} of the key tiles
+    holding each query tile's support (a stand-in for trained models' block sparsity).
+Here one whole head of each extreme (sigma_Q = 24; rho = 1 and 1/16), at both alphas, runs
+at L = 8192 in the bench's launch configuration and is compared element by element:
+every row's tau and O, every row's dQ, every key's dK and dV, and the block mask. A
+smaller sigma_Q = 24 case with several heads and a ragged tail covers the same family at
+a size where the oracle also checks a second head.
+"""
+import numpy as np
+import pytest
+
+from entmax_sm_attention_b200 import binding as eb
+from entmax_sm_attention_b200.workloads import WORKLOADS, make_inputs, make_planted_inputs, small_case
+
+from parity import TOL_GRAD, TOL_O, TOL_TAU, alpha2_exclusions, check_mask, compare, gpu_run, oracle_problem
+
+pytestmark = pytest.mark.gpu
+
+HEAD = WORKLOADS["long_causal_L8192"].with_(B=1, H=1)
+
+
+def _check_head(inp, w, alpha, label):
+    g = gpu_run(inp, w, alpha, backward=True)
+    assert g["status"][0] == eb.ENTMAX_OK, g["status"]
+    pr = oracle_problem(inp, w, alpha)
+    ref = pr.backward()
+    err = {"tau": np.abs(g["tau"] - ref["tau"]).max(), "O": np.abs(g["O"] - ref["O"]).max()}
+    rows_ok = np.ones(ref["tau"].shape + (1,), bool)
+    keys_ok = rows_ok
+    if alpha == 2.0:
+        xr, xk = alpha2_exclusions(pr, ref["tau"], g["tau"])
+        rows_ok, keys_ok = ~xr[..., None], ~xk[..., None]
+        err["excluded_rows"], err["excluded_keys"] = int(xr.sum()), int(xk.sum())
+    err["dQ"] = np.abs(np.where(rows_ok, g["dQ"] - ref["dQ"], 0)).max()
+    err["dK"] = np.abs(np.where(keys_ok, g["dK"] - ref["dK"], 0)).max()
+    err["dV"] = np.abs(g["dV"] - ref["dV"]).max()
+    nbad, namb = check_mask(pr, ref["tau"], g["M"])
+    st = g["stats"].reshape(-1, eb.FWD_STATS)
+    err["block_sparsity"] = 1.0 - st[:, 2].sum() / st[:, 3].sum()
+    err["mask_bad"], err["mask_ambiguous"] = nbad, namb
+    print(label, alpha, {k: (float(v) if not isinstance(v, int) else v) for k, v in err.items()})
+    assert err["tau"] <= TOL_TAU, err
+    assert err["O"] <= TOL_O, err
+    assert max(err["dQ"], err["dK"], err["dV"]) <= TOL_GRAD, err
+    assert nbad == 0, err
+    return err
+
+
+@pytest.mark.parametrize("alpha", [1.5, 2.0])
+def test_iid_sigma24_L8192_head(alpha):
+    w = HEAD.with_(sigma_q=24.0)
+    _check_head(make_inputs(w, seed=7), w, alpha, "iid_sigma24_L8192")
+
+
+@pytest.mark.parametrize("alpha", [1.5, 2.0])
+@pytest.mark.parametrize("rho", [1.0, 0.0625])
+def test_planted_L8192_head(rho, alpha):
+    err = _check_head(make_planted_inputs(HEAD, rho, seed=7), HEAD, alpha, f"planted_rho{rho}_L8192")
+    if rho < 0.1:
+        assert err["block_sparsity"] > 0.85
+
+
+@pytest.mark.parametrize("alpha", [1.5, 2.0])
+def test_iid_sigma24_small(alpha):
+    w = small_case("sigma24_L1100", B=1, H=2, L=1100, causal=True, sigma_q=24.0)
+    rep = {}
+    compare(w, alpha, backward=True, report=rep)
+    print(w.name, alpha, {k: (float(v) if not isinstance(v, int) else v) for k, v in rep.items()})

@@ -17,13 +17,15 @@ from parity import MARGIN, TOL_GRAD, TOL_O, TOL_TAU, alpha2_exclusions, gpu_run
 
 pytestmark = pytest.mark.gpu
 
+# Three or more whole heads per workload: the first (0, 0), the last (B-1, H-1) and one
+# or two in between.
 FULL = [
-    ("gpt2_causal_L1024", 1.5, [(7, 11), (0, 0)]),
-    ("long_causal_L8192", 1.5, [(0, 5)]),
-    ("long_causal_L8192", 2.0, [(0, 3)]),
-    ("encoder_padded_L4096", 1.5, [(3, 2)]),
-    ("encoder_padded_L4096", 2.0, [(1, 7)]),
-    ("window_sink_L2048", 1.5, [(15, 11), (4, 0)]),
+    ("gpt2_causal_L1024", 1.5, [(0, 0), (3, 5), (7, 11)]),
+    ("long_causal_L8192", 1.5, [(0, 0), (0, 5), (0, 11)]),
+    ("long_causal_L8192", 2.0, [(0, 0), (0, 3), (0, 11)]),
+    ("encoder_padded_L4096", 1.5, [(0, 0), (3, 2), (3, 11)]),
+    ("encoder_padded_L4096", 2.0, [(0, 0), (1, 7), (3, 11)]),
+    ("window_sink_L2048", 1.5, [(0, 0), (4, 0), (9, 6), (15, 11)]),
 ]
 
 

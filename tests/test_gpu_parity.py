@@ -54,7 +54,8 @@ def test_entmax_rows(alpha):
         if n == 1000:
             S[3, 10:] = -float("inf")
             S[4, :999] = -float("inf")
-        P, tau = eb.rows(S.cuda(), alpha)
+        P, tau, st = eb.rows(S.cuda(), alpha, return_status=True)
+        assert st == 0
         P, tau = P.cpu().double().numpy(), tau.cpu().double().numpy()
         Pr, taur = oracle.entmax_rows(S, alpha)
         assert np.abs(tau - taur).max() <= 1e-5
@@ -86,7 +87,7 @@ def test_refinement_cap_reports_no_convergence():
         assert np.isfinite(g["O"]).all() and np.isfinite(g["tau"]).all()
         g = gpu_run(make_inputs(w), w, alpha, backward=False)
         assert g["status"][0] == eb.ENTMAX_OK, alpha
-        assert g["stats"].reshape(-1, 4)[:, 0].max() > 1   # it took more than one sweep
+        assert g["stats"].reshape(-1, eb.FWD_STATS)[:, 0].max() > 1   # it took more than one sweep
 
 
 def test_repeatable():
@@ -187,7 +188,7 @@ def test_planted_block_structure(alpha):
     for k in ("dQ", "dK", "dV"):
         assert np.abs(g[k] - ref[k]).max() <= 2e-2, k
     assert check_mask(pr, ref["tau"], g["M"])[0] == 0
-    st = g["stats"].reshape(-1, 4)
+    st = g["stats"].reshape(-1, eb.FWD_STATS)
     sparsity = 1.0 - st[:, 2].sum() / st[:, 3].sum()
     assert sparsity > 0.5, sparsity
 
@@ -208,3 +209,62 @@ def test_max_length_head():
     rep = {}
     compare(w, 1.5, backward=True, report=rep)
     print(w.name, {k: (float(v) if not isinstance(v, int) else v) for k, v in rep.items()})
+
+
+@pytest.mark.parametrize("stage", ["fwd", "bwd"])
+def test_wait_expiry_reports_timeout_and_context_survives(stage):
+    """The bounded-wait failure path, without faulting or hanging anything: with
+    ENTMAX_SELFTEST_STALL one thread of every CTA waits on a barrier that nothing
+    completes, so its wait expires after wait_limit_us (200 us here). The call must report
+    ENTMAX_ETIMEOUT; every other wait then returns at once, no copy or MMA is issued after
+    the abort, the CTA frees its tensor memory and exits. A normal call on the same stream
+    afterwards returns ENTMAX_OK and matches the oracle."""
+    from entmax_sm_attention_b200.workloads import make_inputs
+
+    w = small_case("stall", B=1, H=1, L=256, causal=True)
+    inp = make_inputs(w)
+    d = {k: v.cuda() for k, v in inp.items()}
+    kw = dict(alpha=1.5, scale=w.scale, causal=True)
+    if stage == "fwd":
+        O, tau, ctx = eb.forward(d["Q"], d["K"], d["V"], wait_limit_us=200, selftest=eb.ENTMAX_SELFTEST_STALL, **kw)
+        code, word = eb.entmax_last_device_status(*ctx)
+        assert code == eb.ENTMAX_ETIMEOUT and word & 2, (code, word)
+    else:
+        O, tau, ctx = eb.forward(d["Q"], d["K"], d["V"], **kw)
+        assert eb.entmax_last_device_status(*ctx)[0] == eb.ENTMAX_OK
+        desc, ws = ctx
+        stall = eb.make_desc(1, 1, w.L, alpha=1.5, scale=w.scale, causal=True, wait_limit_us=200,
+                             selftest=eb.ENTMAX_SELFTEST_STALL)
+        dQ, dK, dV = eb.backward((stall, ws), d["Q"], d["K"], d["V"], d["dO"], tau)
+        code, word = eb.entmax_last_device_status(stall, ws)
+        assert code == eb.ENTMAX_ETIMEOUT and word & 2, (code, word)
+    # The context is intact: a normal forward + backward on the same stream is correct.
+    O, tau, ctx = eb.forward(d["Q"], d["K"], d["V"], **kw)
+    dQ, dK, dV = eb.backward(ctx, d["Q"], d["K"], d["V"], d["dO"], tau)
+    assert eb.entmax_last_device_status(*ctx)[0] == eb.ENTMAX_OK
+    ref = oracle.Problem(inp["Q"], inp["K"], inp["V"], inp["dO"], alpha=1.5, scale=w.scale, causal=True).backward()
+    assert np.abs(tau.cpu().double().numpy() - ref["tau"]).max() <= TOL_TAU
+    assert np.abs(O.cpu().double().numpy() - ref["O"]).max() <= 1e-2
+    for k, v in (("dQ", dQ), ("dK", dK), ("dV", dV)):
+        assert np.abs(v.cpu().double().numpy() - ref[k]).max() <= 2e-2, k
+
+
+def test_backward_counters():
+    """The per-key-tile counters of the backward: flagged query tiles visited equal the set
+    bits of the transposed mask, and the phase cycles add up to at most the CTA total."""
+    from entmax_sm_attention_b200.workloads import make_inputs
+
+    w = small_case("bcount", B=1, H=2, L=700, causal=True)
+    d = {k: v.cuda() for k, v in make_inputs(w).items()}
+    O, tau, ctx = eb.forward(d["Q"], d["K"], d["V"], alpha=1.5, scale=w.scale, causal=True)
+    eb.backward(ctx, d["Q"], d["K"], d["V"], d["dO"], tau)
+    M, st = eb.block_mask(ctx)
+    bst = eb.bwd_counters(ctx).cpu().numpy().reshape(-1, eb.BWD_STATS).astype(np.int64)
+    Mb = M.cpu().numpy().view(np.uint32).reshape(2, -1)
+    T = Mb.shape[1]
+    per_key = np.array([[sum((int(Mb[h, it]) >> kt) & 1 for it in range(T)) for kt in range(T)] for h in range(2)])
+    assert np.array_equal(bst[:, 0], per_key.ravel())
+    assert (bst[:, 1] > 0).all()
+    assert (bst[:, 2:6].sum(1) <= bst[:, 1]).all()
+    fst = st.cpu().numpy().reshape(-1, eb.FWD_STATS).astype(np.int64)
+    assert (fst[:, 4:7].sum(1) <= fst[:, 7]).all() and (fst[:, 7] > 0).all()
