@@ -42,11 +42,15 @@
 // mbarrier wait costs ~200 cycles even when the phase is complete, so one issuer per
 // chain keeps each below the tile's tensor time.
 // TMEM (512 columns): during the sweeps, four S buffers at 0/128/256/384, so the MMA
-// warp runs up to three tiles ahead. During the output pass:
-//   - three S buffers at 0, 128 and 384 (tile k in buffer k % 3). The row owner of keys
+// warp runs up to three tiles ahead. During the output pass (OutLayout):
+//   - three S buffers at 0, 128 and 384, tile k in buffer k % 3. The row owner of keys
 //     [32q, 32q+32) writes their A (fp16 pairs) into columns [32q, 32q+16) and g into
 //     [32q+16, 32q+32): only over S columns it has read itself;
 //   - O at [256,320) and Ot at [320,384).
+// alpha = 1.5 splits g = g_hi + g_lo, both fp16: g_lo of tile k goes to shared-memory
+// buffer k % 3 (a K-major [128 rows][128 keys] operand), and the Ot chain adds g_lo V as
+// shared-memory MMAs. The three buffers (96 KB) reuse the tile maxima and candidate lists,
+// which are dead once the final mask is decided.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -64,12 +68,26 @@ constexpr int kProducerWarp = kMathWarps;
 constexpr int kMmaWarp = kMathWarps + 1;
 constexpr int kMma2Warp = kMathWarps + 2;     // second MMA issuer: the Ot = g V chain of the output pass
 constexpr int kMma3Warp = kMathWarps + 3;     // third MMA issuer: the O = A V chain of the output pass
-constexpr int kOBufs = 3;       // S/A buffers in the output pass (TMEM columns 0, 128, 384)
+constexpr int kOBufsMax = 3;    // S/A buffers in the output pass (at most; see OutLayout)
 constexpr int kSlots = 4;
 constexpr int kSBufs = 4;
 constexpr int kCandPerThread = kTile / kParts;   // candidates per (row, column part); 128 per row
 constexpr float kTolF = 3e-5f;         // |f(tau)| = |sum p - 1| small enough to stop sweeping
 constexpr int kMaxVotes = 72;
+
+// Diagnostic builds (-DENTMAX_DIAG, never the shipped library) also record, per query tile,
+// the cycles each role spends waiting: [8] row owner 0 on S in the max pass, [9] on S in
+// the sweeps, [10] on S in the output pass, [11] the first sweep loop in total, [12] the S
+// issuer on its barriers in the max pass and sweeps, [13] in the output pass, [14] the O
+// issuer on its barriers, [15] the TMA producer on free ring slots; then row owner 0's
+// steps per phase ([16..18] max pass: TMEM load, release, compute; [19..21] sweeps;
+// [22..24] output: TMEM load, compute, store + release) and the issuers' issue and commit
+// cycles ([25, 26] S issuer in the max pass and sweeps, [27, 28] O issuer).
+#ifdef ENTMAX_DIAG
+#define DIAG(...) __VA_ARGS__
+#else
+#define DIAG(...)
+#endif
 
 constexpr int kKindSweep = 0;
 constexpr int kKindOutput = 1;
@@ -78,7 +96,7 @@ struct Shared {
   uint64_t full[kSlots], empty[kSlots];
   uint64_t bar_q;
   uint64_t s_full[kSBufs], s_free[kSBufs];     // sweeps: MMA -> rows, rows -> MMA
-  uint64_t o_full[kOBufs], o_ready[kOBufs], pv_done[kOBufs];  // output pass, buffer c = k % 3
+  uint64_t o_full[kOBufsMax], o_ready[kOBufsMax], pv_done[kOBufsMax];  // output pass, buffer c = k % obufs
   uint64_t mma_drain;                          // end of kernel: every issuer's MMAs complete
   uint64_t never;                              // self-test: a barrier nothing completes
   uint32_t tmem_base;
@@ -141,6 +159,37 @@ __device__ __forceinline__ void ldw(uint32_t taddr, uint32_t (&o)[N]) {
     tmem_ld16(taddr, o);
   }
   tmem_wait_ld();
+}
+
+// Output-pass TMEM layout per alpha. alpha = 2: g is 0 or 1, exact in fp16, so three S/A
+// buffers at columns 0, 128, 384. alpha = 1.5: g = u is split into fp16 g_hi + g_lo (the
+// rounding of g alone would move delta = dO . Ot / sum g by 2^-12 relative, which dK
+// multiplies by |Q|); two S/A buffers at 0 and 128, and their g_lo blocks (64 columns of
+// fp16 pairs each) at 384 and 448. O and Ot sit at 256 and 320 in both layouts.
+template <int AK>
+struct OutLayout {
+  static constexpr int kBufs = 3;
+  static constexpr bool kSplitG = AK == kAlpha15;
+  __device__ static __forceinline__ uint32_t sbuf(int c) { return c == 0 ? 0u : (c == 1 ? 128u : 384u); }
+};
+constexpr int kGloBytes = 2 * kTileBytes;          // one g_lo buffer: [128 rows][128 keys] fp16
+constexpr int kGloRegion = 3 * kGloBytes;          // three buffers
+
+// Shared-memory layout of the forward (offsets from the 1024-aligned base): Q tile, K/V
+// ring, then a region holding the tile maxima [Tc][128] and the candidate lists during
+// the max pass and sweeps, and the g_lo buffers during the output pass, then partials.
+__host__ __device__ constexpr int fwd_off_region() { return kTileBytes * (1 + 4); }
+__host__ __device__ constexpr int fwd_region_bytes(int Tc) {
+  return Tc * kTile * 4 + 4 * 32 * kTile * 4 > kGloRegion ? Tc * kTile * 4 + 4 * 32 * kTile * 4 : kGloRegion;
+}
+
+// fp16 pair -> two floats (exact).
+__device__ __forceinline__ float2 unpack_f16x2(uint32_t w) {
+  float lo, hi;
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, h;\n\t}"
+      : "=f"(lo), "=f"(hi)
+      : "r"(w));
+  return make_float2(lo, hi);
 }
 
 // Adds one candidate at u = z - t to the sums of the current support (u > 0), without
@@ -247,14 +296,18 @@ __device__ __forceinline__ float solveN(const float (&v)[N], float cz, float lo,
 
 template <int AK>
 __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant__ FwdParams p) {
+  using OL = OutLayout<AK>;
+  constexpr int kOBufs = OL::kBufs;
   extern __shared__ uint8_t dsm_raw[];
   __shared__ Shared sh;
   uint8_t* dsm = align1024(dsm_raw);
+  static_assert(kSlots == 4 && kCandPerThread == 32 && kParts == 4, "fwd_region_bytes assumes these");
   uint8_t* sQ = dsm;
   uint8_t* ring = dsm + kTileBytes;
-  int* tmax = reinterpret_cast<int*>(dsm + kTileBytes * (1 + kSlots));   // [Tc][128], f2ord
+  int* tmax = reinterpret_cast<int*>(dsm + fwd_off_region());    // [Tc][128], f2ord
   float* cand = reinterpret_cast<float*>(tmax + p.Tc * kTile);   // [kParts][kCandPerThread][128]
-  float* part = cand + kParts * kCandPerThread * kTile;          // [kParts][4][128]
+  uint8_t* glo = dsm + fwd_off_region();                         // output pass: g_lo buffers (alpha 1.5)
+  float* part = reinterpret_cast<float*>(dsm + fwd_off_region() + fwd_region_bytes(p.Tc));   // [kParts][4][128]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bh = blockIdx.x % p.BH;
@@ -275,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       mbar_init(&sh.s_full[s], 1);
       mbar_init(&sh.s_free[s], kMathWarps);
     }
-    for (int s = 0; s < kOBufs; ++s) {
+    for (int s = 0; s < kOBufsMax; ++s) {
       mbar_init(&sh.o_full[s], 1);
       mbar_init(&sh.o_ready[s], kMathWarps);
       mbar_init(&sh.pv_done[s], 2);   // O chain and Ot chain
@@ -316,13 +369,16 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     // one per slot, are ever in flight, and the drain below sees each slot's last one.
     uint32_t seq = 0;
     bool live = true;
+    DIAG(long long dg_wait = 0);
     auto load = [&](const CUtensorMap* map, int jt) {
       if (!live) return;
       const int slot = seq % kSlots;
+      DIAG(const long long d0 = clock64());
       if (!mbar_wait(&sh.empty[slot], ((seq / kSlots) & 1) ^ 1, wc)) {
         live = false;
         return;
       }
+      DIAG(dg_wait += clock64() - d0);
       mbar_expect_tx(&sh.full[slot], kTileBytes);
       tma_load_3d(ring + slot * kTileBytes, map, &sh.full[slot], 0, jt * kTile, bh);
       ++seq;
@@ -355,6 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       __syncwarp();
       if (kind != kKindSweep) break;
     }
+    DIAG(if (lane == 0) p.stats[((size_t)bh * p.Tr + qt) * kFwdStats + 15] = (int)dg_wait);
     // Make sure no copy is still in flight when the CTA retires.
     if (lane == 0) {
       mbar_drain(&sh.bar_q, 0, status);
@@ -368,6 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     uint32_t sfree_par = 0;      // per sweep S buffer: parity of its uses so far (bit b)
     uint32_t sbuf = 0;           // next sweep S buffer
     bool live = true;            // false after a failed wait: no further MMA is issued
+    DIAG(long long dg_sw = 0; long long dg_out = 0; long long dg_iss = 0);
     const uint32_t idS = idesc_bf16(128, 128, 0, 0);
     const uint64_t qd0 = sdesc_sw128(smem_u32(sQ), 16, 1024);      // Q tile, K-major
     const uint64_t kd0 = sdesc_sw128(smem_u32(ring), 16, 1024);    // ring slot 0, K-major
@@ -385,13 +443,16 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       const uint32_t bf = sbuf;
       const uint32_t pos = seq++;
       // S buffer consumed by the row owners, and K tile landed.
+      DIAG(const long long d0 = clock64());
       live = live && mbar_wait2(&sh.s_free[bf], ((sfree_par >> bf) & 1) ^ 1, &sh.full[pos % kSlots],
                                 (pos / kSlots) & 1, wc);
+      DIAG(dg_sw += clock64() - d0);
       sfree_par ^= 1u << bf;
       if (live) {
         mma_s(pos, bf * 128);
         mma_commit(&sh.s_full[bf]);
       }
+      DIAG(dg_iss += clock64() - d0);
       sbuf = (sbuf + 1) & (kSBufs - 1);
     };
     if (lane == 0) {
@@ -421,16 +482,21 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           for (int k = 0; k < n; ++k) {
             const int c = k % kOBufs;
             const uint32_t pos = base + 2 * k;
+            DIAG(const long long d0 = clock64());
             if (k >= kOBufs)
               live = live && mbar_wait2(&sh.pv_done[c], ((k - kOBufs) / kOBufs) & 1, &sh.full[pos % kSlots],
                                         (pos / kSlots) & 1, wc);
             else
               live = live && mbar_wait(&sh.full[pos % kSlots], (pos / kSlots) & 1, wc);
+            DIAG(dg_out += clock64() - d0);
             if (!live) break;
-            mma_s(pos, c == 0 ? 0u : (c == 1 ? 128u : 384u));
+            mma_s(pos, OL::sbuf(c));
             mma_commit(&sh.o_full[c]);
           }
           seq = base + 2 * n;
+          DIAG(p.stats[((size_t)bh * p.Tr + qt) * kFwdStats + 12] = (int)dg_sw);
+          DIAG(p.stats[((size_t)bh * p.Tr + qt) * kFwdStats + 13] = (int)dg_out);
+          DIAG(p.stats[((size_t)bh * p.Tr + qt) * kFwdStats + 25] = (int)(dg_iss - dg_sw));
         }
       }
       __syncwarp();
@@ -440,6 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     // ------------------------------------------------ second MMA issuer (output pass)
     const uint32_t idO = idesc_f16(128, 64, 0, 1);
     const uint64_t vd0 = sdesc_sw128(smem_u32(ring), 8192, 1024);   // ring slot 0, MN-major
+    const uint64_t gd0 = sdesc_sw128(smem_u32(glo), 16, 1024);      // g_lo buffer 0, K-major
     uint32_t seq = 0;   // ring positions, tracked exactly like the producer's
     for_each_bit(act, kMaskWords, [&](int) { ++seq; });
     while (true) {
@@ -457,7 +524,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         const uint32_t base = seq;
         for (int k = 0; k < n; ++k) {
           const int c = k % kOBufs;
-          const uint32_t pa = c == 0 ? 0u : (c == 1 ? 128u : 384u);
+          const uint32_t pa = OL::sbuf(c);
           const uint32_t vpos = base + 2 * k + 1;
           const int vslot = vpos % kSlots;
           if (!mbar_wait2(&sh.full[vslot], (vpos / kSlots) & 1, &sh.o_ready[c], (k / kOBufs) & 1, wc)) break;
@@ -468,6 +535,13 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
             // keys 16t..16t+15: part 16t / kCols, pair columns ((16t) % kCols) / 2 of its A block
             const uint32_t col = pa + (16 * t / kCols) * kCols + ((16 * t) % kCols) / 2 + kCols / 2;   // g block
             mma_ts(T + 320, T + col, sdesc_add(vd, t * 2048), idO, (k > 0 || t > 0) ? 1u : 0u);
+          }
+          if constexpr (OL::kSplitG) {
+            // g_lo of keys 16t..16t+15: panel t / 4 of buffer c, 32-byte step t % 4.
+#pragma unroll
+            for (int t = 0; t < 8; ++t)
+              mma_ss(T + 320, sdesc_add(gd0, c * kGloBytes + (t >> 2) * kTileBytes + (t & 3) * 32),
+                     sdesc_add(vd, t * 2048), idO, 1u);
           }
           mma_commit(&sh.empty[vslot]);
           mma_commit(&sh.pv_done[c]);
@@ -494,13 +568,16 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       if (kind == kKindSweep) {
         seq += n;
       } else if (lane == 0) {
+        DIAG(long long dg_o = 0);
         const uint32_t base = seq;
         for (int k = 0; k < n; ++k) {
           const int c = k % kOBufs;
-          const uint32_t pa = c == 0 ? 0u : (c == 1 ? 128u : 384u);
+          const uint32_t pa = OL::sbuf(c);
           const uint32_t vpos = base + 2 * k + 1;
           const int vslot = vpos % kSlots;
+          DIAG(const long long d0 = clock64());
           if (!mbar_wait2(&sh.full[vslot], (vpos / kSlots) & 1, &sh.o_ready[c], (k / kOBufs) & 1, wc)) break;
+          DIAG(dg_o += clock64() - d0);
           tc_fence_after();
           const uint64_t vd = sdesc_add(vd0, vslot * kTileBytes);
 #pragma unroll
@@ -512,6 +589,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           mma_commit(&sh.empty[vslot]);
           mma_commit(&sh.pv_done[c]);
         }
+        DIAG(p.stats[((size_t)bh * p.Tr + qt) * kFwdStats + 14] = (int)dg_o);
       }
       __syncwarp();
       if (kind != kKindSweep) break;
@@ -527,18 +605,24 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     uint32_t sfull_par = 0, sbuf = 0;
     float m = -INFINITY;
     float top[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+    DIAG(long long dg_s1 = 0; long long dg_s2 = 0; long long dg_s3 = 0; long long dg_sw1 = 0);
+    DIAG(long long dgr[9] = {0, 0, 0, 0, 0, 0, 0, 0, 0}; long long dtk = 0);
 
     // Phase 1: per-key-tile row maxima over this thread's column part (combined in smem).
     for_each_bit(act, kMaskWords, [&](int jt) {
       const uint32_t bf = sbuf;
+      DIAG(const long long d0 = clock64());
       warp_wait(&sh.s_full[bf], (sfull_par >> bf) & 1, wc);
+      DIAG(const long long d1 = clock64(); dg_s1 += d1 - d0);
       sfull_par ^= 1u << bf;
       tc_fence_after();
       const int j0 = jt * kTile + qp * kCols;
       float s[kCols];
       ldc(tl + bf * 128 + qp * kCols, s);
+      DIAG(const long long d2 = clock64(); dgr[0] += d2 - d1);
       tc_fence_before();
       warp_arrive(&sh.s_free[bf]);
+      DIAG(dtk = clock64(); dgr[1] += dtk - d2);
       if (!pat.block_full(i0, i1, jt * kTile, jt * kTile + kTile)) {
 #pragma unroll
         for (int c = 0; c < kCols; ++c)
@@ -561,6 +645,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         top[k] = big;
       }
       sbuf = (sbuf + 1) & (kSBufs - 1);
+      DIAG(dgr[2] += clock64() - dtk);
     });
     // All column parts' four largest part-tile maxima: the row max and the values of the
     // initial threshold.
@@ -646,18 +731,21 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         int k = 0;
         for_each_bit(list, kMaskWords, [&](int jt) {
           const int c = k % kOBufs;
-          const uint32_t pa = c == 0 ? 0u : (c == 1 ? 128u : 384u);
+          const uint32_t pa = OL::sbuf(c);
+          DIAG(const long long d0 = clock64());
           warp_wait(&sh.o_full[c], (k / kOBufs) & 1, wc);
+          DIAG(const long long d1 = clock64(); dg_s3 += d1 - d0);
           tc_fence_after();
           const int j0 = jt * kTile + qp * kCols;
           float s[kCols];
           ldc(tl + pa + qp * kCols, s);
+          DIAG(const long long d2 = clock64(); dgr[6] += d2 - d1);
           if (!pat.block_full(i0, i1, jt * kTile, jt * kTile + kTile)) {
 #pragma unroll
             for (int cc = 0; cc < kCols; ++cc)
               if (!pat.active(i, j0 + cc)) s[cc] = -INFINITY;
           }
-          uint32_t aw[kCols / 2], gw[kCols / 2];
+          uint32_t aw[kCols / 2], gw[kCols / 2], lw[kCols / 2];
 #pragma unroll
           for (int cc = 0; cc < kCols / 2; ++cc) {
             const float2 u = __ffma2_rn(make_float2(s[2 * cc], s[2 * cc + 1]), make_float2(cz, cz),
@@ -667,6 +755,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
               const float2 a = __fmul2_rn(make_float2(v0, v1), make_float2(v0, v1));
               aw[cc] = pack_f16(a.x, a.y);
               gw[cc] = pack_f16(v0, v1);
+              const float2 gh = unpack_f16x2(gw[cc]);
+              const float2 gl = __ffma2_rn(gh, make_float2(-1.f, -1.f), make_float2(v0, v1));   // exact
+              lw[cc] = pack_f16(gl.x, gl.y);
               sg2 = __fadd2_rn(sg2, make_float2(v0, v1));
             } else {
               const float g0 = u.x > 0.f ? 1.f : 0.f, g1 = u.y > 0.f ? 1.f : 0.f;
@@ -679,14 +770,25 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           // A (fp16 pairs) in the first half, g in the second. Writing only into columns this
           // thread has read keeps the row's other parts from seeing overwritten S values.
           const uint32_t col = pa + qp * kCols;
+          DIAG(const long long d3 = clock64(); dgr[7] += d3 - d2);
 #pragma unroll
           for (int h = 0; h < kCols / 32; ++h) {
             tmem_st16(tl + col + 16 * h, *reinterpret_cast<uint32_t(*)[16]>(&aw[16 * h]));
             tmem_st16(tl + col + kCols / 2 + 16 * h, *reinterpret_cast<uint32_t(*)[16]>(&gw[16 * h]));
           }
+          if constexpr (OL::kSplitG) {
+            // keys [32 qp, 32 qp + 32): panel qp / 2, 16-byte chunks 4 (qp % 2) .. + 3 of the row.
+            uint8_t* gb = glo + c * kGloBytes + (qp >> 1) * kTileBytes;
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc)
+              *reinterpret_cast<uint4*>(gb + sw128_offset(row, ((qp & 1) * 4 + cc) * 8)) =
+                  make_uint4(lw[4 * cc], lw[4 * cc + 1], lw[4 * cc + 2], lw[4 * cc + 3]);
+            fence_proxy_async_smem();   // generic-proxy stores, read by the tensor cores
+          }
           tmem_wait_st();
           tc_fence_before();
           warp_arrive(&sh.o_ready[c]);
+          DIAG(dgr[8] += clock64() - d3);
           ++k;
           ++n_s;
         });
@@ -728,30 +830,74 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           int4* st = reinterpret_cast<int4*>(p.stats + ((size_t)bh * p.Tr + qt) * kFwdStats);
           st[0] = make_int4(sweeps, (int)n_s, n_out, na);
           st[1] = make_int4((int)(clk1 - clk0), (int)(clk2 - clk1), (int)(clk3 - clk2), (int)(clk3 - clk0));
+          DIAG(st[2] = make_int4((int)dg_s1, (int)dg_s2, (int)dg_s3, (int)dg_sw1));
+          DIAG(st[4] = make_int4((int)dgr[0], (int)dgr[1], (int)dgr[2], (int)dgr[3]));
+          DIAG(st[5] = make_int4((int)dgr[4], (int)dgr[5], (int)dgr[6], (int)dgr[7]));
+          DIAG(st[6].x = (int)dgr[8]);
         }
         break;
       }
 
-      // Phase 3: one refinement sweep at the current tau. Every sweep also collects this
+      // Phase 3: one refinement sweep at the current tau. Every sweep collects this
       // thread's candidates u > 0: when tau <= tau* (f >= 0) they hold the whole support.
+      // The first sweep runs at the tile-maxima bound tau_T <= tau*, so its candidates
+      // hold the support by construction and it only collects them: one max over the
+      // thread's 32 scores and a test against tau, with an element scan only when that
+      // max passes (rare). Later sweeps (rows whose candidates overflowed, or Newton
+      // steps) also accumulate S1, S2 and the count for f(tau) and f'(tau).
+      const bool cand_only = sweeps == 0;
       float S1 = 0.f, S2 = 0.f;
       int nc = 0;
       float* mycand = cand + qp * kCandPerThread * kTile + row;
       sbuf = 0;
+      DIAG(const long long dsw0 = clock64());
       for_each_bit(list, kMaskWords, [&](int jt) {
         const uint32_t bf = sbuf;
+        DIAG(const long long d0 = clock64());
         warp_wait(&sh.s_full[bf], (sfull_par >> bf) & 1, wc);
+        DIAG(const long long d1 = clock64(); dg_s2 += d1 - d0);
         sfull_par ^= 1u << bf;
         tc_fence_after();
         const int j0 = jt * kTile + qp * kCols;
         float s[kCols];
         ldc(tl + bf * 128 + qp * kCols, s);
+        DIAG(const long long d2 = clock64(); dgr[3] += d2 - d1);
         tc_fence_before();
         warp_arrive(&sh.s_free[bf]);
+        DIAG(dtk = clock64(); dgr[4] += dtk - d2);
         if (!pat.block_full(i0, i1, jt * kTile, jt * kTile + kTile)) {
 #pragma unroll
           for (int cc = 0; cc < kCols; ++cc)
             if (!pat.active(i, j0 + cc)) s[cc] = -INFINITY;
+        }
+        if (cand_only) {
+          // Maxima of the four 8-key groups (independent trees), then an element scan of
+          // only the groups whose maximum passes tau.
+          float gm[kCols / 8];
+#pragma unroll
+          for (int g = 0; g < kCols / 8; ++g) {
+            const float* x = s + 8 * g;
+            gm[g] = fmaxf(fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3])), fmaxf(fmaxf(x[4], x[5]), fmaxf(x[6], x[7])));
+          }
+          const float tm = fmaxf(fmaxf(gm[0], gm[1]), fmaxf(gm[2], gm[3]));
+          if (fmaf(tm, cz, -tau) > 0.f) {
+#pragma unroll
+            for (int g = 0; g < kCols / 8; ++g) {
+              if (fmaf(gm[g], cz, -tau) > 0.f) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                  if (fmaf(s[8 * g + e], cz, -tau) > 0.f) {
+                    if (nc < kCandPerThread) mycand[nc * kTile] = s[8 * g + e];
+                    ++nc;
+                  }
+                }
+              }
+            }
+          }
+          ++n_s;
+          sbuf = (sbuf + 1) & (kSBufs - 1);
+          DIAG(dgr[5] += clock64() - dtk);
+          return;
         }
         float2 s1[4], s2[4];
 #pragma unroll
@@ -798,6 +944,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         ++n_s;
         sbuf = (sbuf + 1) & (kSBufs - 1);
       });
+      DIAG(if (cand_only) dg_sw1 = clock64() - dsw0);
       // Combine the column parts of each row.
       float* mp = part + qp * 4 * kTile + row;
       mp[0] = S1;
@@ -821,7 +968,15 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       const float C = (float)ntot;   // support size at tau (alpha = 2: |f'(tau)|)
       named_bar(3, kMathThreads);   // partials consumed before anyone rewrites them
       ++sweeps;
-      if (!done) {
+      if (!done && cand_only) {
+        // tau = tau_T <= tau*: if the copies fit they hold the support; solve on them.
+        // Otherwise tau stays and the next sweep measures f(tau) and f'(tau).
+        float t;
+        if (fits && solve_list<AK>(cand + row, ncs, kCandPerThread * kTile, kTile, cz, tau, lo, hi, t)) {
+          tau = t;
+          done = true;
+        }
+      } else if (!done) {
         const float f = (AK == kAlpha15) ? S2 - 1.f : S1 - 1.f;
         const float fp = (AK == kAlpha15) ? 2.f * S1 : C;   // |f'(tau)|
         if (f > 0.f) lo = fmaxf(lo, tau); else hi = fminf(hi, tau);
@@ -862,9 +1017,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
   if (warp == kMmaWarp) tmem_dealloc(T, 512);
 }
 
-int fwd_smem_bytes(int Tc) {
-  return 1024 + kTileBytes * (1 + kSlots) + Tc * kTile * 4 + kParts * kCandPerThread * kTile * 4 + kParts * 4 * kTile * 4;
-}
+int fwd_smem_bytes(int Tc) { return 1024 + fwd_off_region() + fwd_region_bytes(Tc) + kParts * 4 * kTile * 4; }
 
 cudaError_t launch_fwd(bool alpha15, const FwdParams& p, int grid, cudaStream_t s) {
   const int smem = fwd_smem_bytes(p.Tc);

@@ -11,7 +11,12 @@ namespace entmax {
 //   (output pass), 3 structurally active key tiles, then SM clock cycles (clock64
 //   differences) of 4 the max pass, 5 threshold refinement and mask decision, 6 the output
 //   pass and epilogue, 7 the whole CTA.
+#ifdef ENTMAX_DIAG
+// Diagnostic builds append wait and step counters per query tile (see fwd.cu).
+constexpr int kFwdStats = 32;
+#else
 constexpr int kFwdStats = 8;
+#endif
 // Per-key-tile counters of the backward kernel: 0 flagged query tiles visited, then cycles
 // of 1 the whole CTA, and, for the first row-owner warp, 2 waiting for S and dA, 3 waiting
 // for the previous tile's gradient MMAs, 4 forming A and dS, 5 staging dQ (reduce-add).
