@@ -379,15 +379,16 @@ def run_ours(args):
     s_tiles, out_tiles, act_tiles = int(n_s.sum()), int(n_out.sum()), int(n_act.sum())
     work = pair_work(w, M.cpu(), st)
     # Algorithmic tensor work (the scope table's per-pair figures): forward
-    # (1+R) 2d |A_i| + 3 2d |F_i| summed over rows (max pass and R refinement passes over
-    # the active keys; S, A V and g V over the keys of flagged tiles), backward 5 2d |F_i|
-    # (S, dA, dV, dK, dQ). R is each query tile's measured refinement count.
+    # (1+R) 2d |A_i| + 2 2d |F_i| summed over rows (max pass and R refinement passes over
+    # the active keys; S and A V over the keys of flagged tiles: delta's g V term is not a
+    # tensor product here, the backward's delta kernel sums it over the support lists),
+    # backward 5 2d |F_i| (S, dA, dV, dK, dQ). R is each query tile's measured count.
     fwd_flops = work["fwd_flops"]
     bwd_flops = work["bwd_flops"]
     # The same at tile granularity (every 128x128 block counted whole, diagonal blocks
     # included), and the work the tensor cores are issued (dS enters dK and dQ as two
     # bf16 terms, hi + lo).
-    fwd_tile_flops = UNIT_FLOP * (s_tiles + 2 * out_tiles)
+    fwd_tile_flops = UNIT_FLOP * (s_tiles + out_tiles)
     bwd_tile_flops = UNIT_FLOP * 5 * out_tiles
     fwd_issued = fwd_tile_flops
     bwd_issued = UNIT_FLOP * 7 * out_tiles
@@ -533,7 +534,7 @@ def marginal_throughput(points) -> dict:
         b = sum((x - mx) * (y - my) for x, y in zip(xs, ys)) / sxx
         return b, my - b * mx
     out = {}
-    fl = [UNIT_FLOP * (p["s_tiles"] + 2 * p["flagged_tiles"]) for p in points]
+    fl = [UNIT_FLOP * (p["s_tiles"] + p["flagged_tiles"]) for p in points]
     bl = [UNIT_FLOP * 5 * p["flagged_tiles"] for p in points]
     for name, xs, ys in (("fwd", fl, [p["fwd_ms"] for p in points]), ("bwd", bl, [p["bwd_ms"] for p in points]),
                          ("fwd+bwd", [a + b for a, b in zip(fl, bl)], [p["ms"] for p in points])):
@@ -567,7 +568,7 @@ def block_pair_counts(w):
 def pair_work(w, M, st) -> dict:
     """Algorithmic tensor work at pair granularity from the block mask M (int32 bit
     patterns [B, H, T, words]) and the forward counters st ([B, H, T, 8]): forward
-    sum_i (1+R_i) 2d |A_i| + 3 2d |F_i|, backward 5 2d |F_i|, where A_i are the active keys
+    sum_i (1+R_i) 2d |A_i| + 2 2d |F_i|, backward 5 2d |F_i|, where A_i are the active keys
     of row i, F_i the active keys of row i inside flagged blocks, and R_i the refinement
     passes of row i's query tile."""
     import numpy as np
@@ -582,7 +583,7 @@ def pair_work(w, M, st) -> dict:
     active = np.broadcast_to(cnt.sum(-1)[:, None], flagged.shape)   # [B, H, T] active pairs per query tile
     R = st[..., 0].numpy().astype(np.int64)
     two_d = 2 * w.d
-    fwd = int(((1 + R) * active).sum() * two_d + 3 * flagged.sum() * two_d)
+    fwd = int(((1 + R) * active).sum() * two_d + 2 * flagged.sum() * two_d)
     bwd = int(5 * flagged.sum() * two_d)
     return {"fwd_flops": fwd, "bwd_flops": bwd, "active_pairs": int(active.sum()),
             "flagged_pairs": int(flagged.sum())}

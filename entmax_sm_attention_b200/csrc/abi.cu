@@ -195,6 +195,7 @@ extern "C" entmax_status entmax_attn_fwd(const entmax_attn_desc* d, const void* 
   p.tau = tau;
   p.sumg = reinterpret_cast<float*>(w + l.off_sumg);
   p.Ot = reinterpret_cast<float*>(w + l.off_Ot);
+  p.V16 = static_cast<const uint16_t*>(v16);
   p.M = reinterpret_cast<uint32_t*>(w + l.off_M);
   p.MT = reinterpret_cast<uint32_t*>(w + l.off_MT);
   p.stats = reinterpret_cast<int*>(w + l.off_stats);
@@ -260,11 +261,30 @@ extern "C" entmax_status entmax_attn_bwd(const entmax_attn_desc* d, const void* 
   p.wait_limit_ns = wait_limit_ns(d);
   p.selftest = d->selftest;
   const long rows = (long)l.BH * d->L;
+  DeltaParams dp;
+  std::memset(&dp, 0, sizeof(dp));
+  dp.Q = static_cast<const uint16_t*>(Q);
+  dp.K = static_cast<const uint16_t*>(K);
+  dp.V = static_cast<const uint16_t*>(V);
+  dp.dO = static_cast<const uint16_t*>(dO);
+  dp.tau = tau;
+  dp.V16 = reinterpret_cast<const uint16_t*>(w + l.off_v16);
+  dp.Ot = reinterpret_cast<const float*>(w + l.off_Ot);
+  dp.sumg = reinterpret_cast<const float*>(w + l.off_sumg);
+  dp.M = reinterpret_cast<const uint32_t*>(w + l.off_M);
+  dp.delta = delta;
+  dp.kv_len = d->kv_len;
+  dp.H = d->H;
+  dp.L = d->L;
+  dp.Tr = l.Tr;
+  dp.Wc = l.Wc;
+  dp.BH = l.BH;
+  dp.cz = (d->alpha - 1.0f) * d->scale;
+  dp.causal = d->causal || d->window >= 0;
+  dp.window = d->window < 0 ? -1 : d->window;
+  if (launch_delta(d->alpha == 1.5f, dp, s) != cudaSuccess) return ENTMAX_ECUDA;
   if (cudaMemsetAsync(dQ, 0, (size_t)rows * kD * 4, s) != cudaSuccess) return ENTMAX_ECUDA;
   if (launch_bf16_to_f16(dO, do16, rows * kD, reinterpret_cast<int*>(w + l.off_status), s) != cudaSuccess)
-    return ENTMAX_ECUDA;
-  if (launch_delta(static_cast<const uint16_t*>(dO), reinterpret_cast<const float*>(w + l.off_Ot),
-                   reinterpret_cast<const float*>(w + l.off_sumg), delta, rows, s) != cudaSuccess)
     return ENTMAX_ECUDA;
   return launch_bwd(d->alpha == 1.5f, p, l.BH * l.Tc, s) == cudaSuccess ? ENTMAX_OK : ENTMAX_ECUDA;
 }

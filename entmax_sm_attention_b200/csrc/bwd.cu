@@ -390,32 +390,137 @@ cudaError_t launch_bwd(bool alpha15, const BwdParams& p, int grid, cudaStream_t 
   return cudaGetLastError();
 }
 
-// delta_i = dO_i . Ot_i / sum_j g_ij for every row (the backward's per-row scalar).
-__global__ void bwd_delta_kernel(const uint16_t* __restrict__ dO, const float* __restrict__ Ot,
-                                 const float* __restrict__ sumg, float* __restrict__ delta, long rows) {
-  const long r = (long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (r >= rows) return;
-  const uint4* d = reinterpret_cast<const uint4*>(dO + r * kD);
-  const float4* o = reinterpret_cast<const float4*>(Ot + r * kD);
-  float acc = 0.f;
-#pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const uint4 w = d[k];
-    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float lo = __uint_as_float(ww[e] << 16), hi = __uint_as_float(ww[e] & 0xffff0000u);
-      const float4 ov = o[2 * k + (e >> 1)];
-      acc = fmaf(lo, (e & 1) ? ov.z : ov.x, acc);
-      acc = fmaf(hi, (e & 1) ? ov.w : ov.y, acc);
-    }
-  }
-  delta[r] = acc / sumg[r];
+// delta_i = sum_j g_ij dA_ij / sum_j g_ij = dO_i . Ot_i / sum_j g_ij, with dA_ij = dO_i . V_j,
+// g = u^{(2-alpha)/(alpha-1)} and u = (alpha-1) scale q_i . k_j - tau_i > 0 (the support).
+// The forward sums Ot_i = sum_j g_ij V_j and sum_j g_ij exactly (fp32) over each row's
+// support; one lane per row forms the dot here. A row whose support the forward could not
+// list (sum g = -1: the refinement cap, or a Newton finish on near-uniform rows) is served
+// by its whole warp afterwards: the lanes take the keys of the row's flagged key tiles,
+// recompute u from q_i . k_j in fp32 (exact bf16 products) and sum g dO_i . V_j.
+namespace {
+constexpr int kDeltaWarps = 4;
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+__device__ __forceinline__ float2 f16x2(uint32_t w) {
+  float lo, hi;
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, h;\n\t}"
+      : "=f"(lo), "=f"(hi)
+      : "r"(w));
+  return make_float2(lo, hi);
 }
 
-cudaError_t launch_delta(const uint16_t* dO, const float* Ot, const float* sumg, float* delta, long rows,
-                         cudaStream_t s) {
-  bwd_delta_kernel<<<(unsigned)((rows + 255) / 256), 256, 0, s>>>(dO, Ot, sumg, delta, rows);
+// dot of a bf16 (is_f16 = false) or fp16 row with 64 floats in shared memory (broadcast
+// reads: every lane reads the same x).
+__device__ __forceinline__ float dot_s(const uint4* __restrict__ row, const float* x, bool is_f16) {
+  float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const uint4 w = row[k];
+    const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = is_f16 ? f16x2(w4[e]) : make_float2(bf16lo(w4[e]), bf16hi(w4[e]));
+      a0 = fmaf(f.x, x[8 * k + 2 * e], a0);
+      a1 = fmaf(f.y, x[8 * k + 2 * e + 1], a1);
+    }
+  }
+  return a0 + a1;
+}
+}  // namespace
+
+template <int AK>
+__global__ void __launch_bounds__(32 * kDeltaWarps, 4) bwd_delta_kernel(const __grid_constant__ DeltaParams p) {
+  __shared__ float xs[kDeltaWarps][2][kD];   // brute-force path: q_i and dO_i of the row served
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long rows = (long)p.BH * p.L;
+  const long r0 = ((long)blockIdx.x * kDeltaWarps + warp) * 32;
+  if (r0 >= rows) return;
+  const long r = r0 + lane;
+  const bool valid = r < rows;
+  const long rc = valid ? r : r0;
+  const float sgf = p.sumg[rc];
+  const bool listed = sgf >= 0.f;
+  float delta = 0.f;
+  if (valid && listed) {
+    const uint4* dr = reinterpret_cast<const uint4*>(p.dO + rc * kD);
+    const float4* orow = reinterpret_cast<const float4*>(p.Ot + rc * kD);
+    float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const uint4 w = dr[k];
+      const float4 o0 = orow[2 * k], o1 = orow[2 * k + 1];
+      a0 = fmaf(bf16lo(w.x), o0.x, a0);
+      a1 = fmaf(bf16hi(w.x), o0.y, a1);
+      a0 = fmaf(bf16lo(w.y), o0.z, a0);
+      a1 = fmaf(bf16hi(w.y), o0.w, a1);
+      a0 = fmaf(bf16lo(w.z), o1.x, a0);
+      a1 = fmaf(bf16hi(w.z), o1.y, a1);
+      a0 = fmaf(bf16lo(w.w), o1.z, a0);
+      a1 = fmaf(bf16hi(w.w), o1.w, a1);
+    }
+    delta = (a0 + a1) / sgf;
+  }
+  uint32_t ovf = __ballot_sync(0xffffffffu, valid && !listed);
+  while (ovf) {
+    const int ol = __ffs(ovf) - 1;
+    ovf &= ovf - 1;
+    const long ro = r0 + ol;
+    const int i = (int)(ro % p.L), bho = (int)(ro / p.L);   // the warp's rows may span two heads
+    __syncwarp();
+    {
+      const uint32_t qw = reinterpret_cast<const uint32_t*>(p.Q + ro * kD)[lane];
+      const uint32_t dw = reinterpret_cast<const uint32_t*>(p.dO + ro * kD)[lane];
+      xs[warp][0][2 * lane] = bf16lo(qw);
+      xs[warp][0][2 * lane + 1] = bf16hi(qw);
+      xs[warp][1][2 * lane] = bf16lo(dw);
+      xs[warp][1][2 * lane + 1] = bf16hi(dw);
+    }
+    __syncwarp();
+    const float to = p.tau[ro];
+    const uint4* Ko = reinterpret_cast<const uint4*>(p.K + (size_t)bho * p.L * kD);
+    const uint4* Vo = reinterpret_cast<const uint4*>(p.V16 + (size_t)bho * p.L * kD);
+    const int b = bho / p.H;
+    const Pattern pat{p.L, p.kv_len ? min(max(p.kv_len[b], 1), p.L) : p.L, p.causal, p.window};
+    const uint32_t* words = p.M + ((size_t)bho * p.Tr + i / kTile) * p.Wc;
+    float og = 0.f, ogd = 0.f;
+    for (int w = 0; w < p.Wc; ++w) {
+      uint32_t bits = words[w];
+      while (bits) {
+        const int jt = w * 32 + __ffs(bits) - 1;
+        bits &= bits - 1;
+#pragma unroll
+        for (int jj = lane; jj < kTile; jj += 32) {   // four keys per lane, loads in flight together
+          const int jk = jt * kTile + jj;
+          if (jk < p.L && pat.active(i, jk)) {
+            const float uu = fmaf(dot_s(Ko + (size_t)jk * 8, xs[warp][0], false), p.cz, -to);
+            if (uu > 0.f) {
+              const float g = (AK == kAlpha15) ? uu : 1.f;
+              og += g;
+              ogd = fmaf(g, dot_s(Vo + (size_t)jk * 8, xs[warp][1], true), ogd);
+            }
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      og += __shfl_xor_sync(0xffffffffu, og, o);
+      ogd += __shfl_xor_sync(0xffffffffu, ogd, o);
+    }
+    if (lane == ol) delta = ogd / og;
+  }
+  if (valid) p.delta[r] = delta;
+}
+
+cudaError_t launch_delta(bool alpha15, const DeltaParams& p, cudaStream_t s) {
+  const long rows = (long)p.BH * p.L;
+  const long per_block = (long)kDeltaWarps * 32;
+  const unsigned grid = (unsigned)((rows + per_block - 1) / per_block);
+  if (alpha15)
+    bwd_delta_kernel<kAlpha15><<<grid, 32 * kDeltaWarps, 0, s>>>(p);
+  else
+    bwd_delta_kernel<kAlpha2><<<grid, 32 * kDeltaWarps, 0, s>>>(p);
   return cudaGetLastError();
 }
 

@@ -11,46 +11,42 @@
 //     tau_T <= tau* (entmax on a subset of the scores has fewer nonnegative terms in
 //     Eq. 4). It plays the role the paper gives its on-chip histogram (Phase 2), without
 //     an extra pass over K.
-//   Phase 3 (refinement): a sweep at tau accumulates S1 = sum u, S2 = sum u^2 and the
-//     count (u = [z - tau]_+) and copies every score with u > 0 into shared memory
-//     (32 per row and column part, 128 per row). While tau <= tau* (f(tau) >= 0, true at tau_T) those
-//     copies hold the whole support, so a row whose copies fit is solved exactly on
-//     chip: safeguarded Newton on Eq. 4 (§3.2), finished by the exact root of the
-//     current support's piece (alpha = 2: (S1-1)/C; alpha = 1.5: the smaller root of
-//     C d^2 - 2 S1 d + S2 - 1 = 0) once no candidate leaves the support. A row whose
-//     copies overflow takes one Newton step bracketed by §2.4 and sweeps again. Eq. 4's
-//     f is convex and decreasing in tau, so a Newton step from tau <= tau* stays
-//     <= tau*, and the next sweep's copies (fewer, above a higher tau) again qualify.
+//   Phase 3 (refinement): a sweep at tau copies every score with u = z - tau > 0 into
+//     shared memory (32 per row and column part, 128 per row). While tau <= tau*
+//     (f(tau) >= 0, true at tau_T) those copies hold the whole support, so a row whose
+//     copies fit is solved exactly on chip: safeguarded Newton on Eq. 4 (§3.2), finished
+//     by the exact root of the current support's piece (alpha = 2: (S1-1)/C; alpha =
+//     1.5: the smaller root of C d^2 - 2 S1 d + S2 - 1 = 0) once no candidate leaves the
+//     support. The first sweep runs at tau_T and only collects; a row whose copies
+//     overflow sweeps again, now also accumulating S1 = sum u, S2 = sum u^2 and the count
+//     for a Newton step bracketed by §2.4. Eq. 4's f is convex and decreasing in tau, so a
+//     Newton step from tau <= tau* stays <= tau*, and the next sweep's copies (fewer,
+//     above a higher tau) again qualify.
 //   Block mask: bit (query tile, key tile) = some row has a key-tile max above its
 //     final tau. Packed 32 key tiles per uint32 (Appendix C.4), plus the transpose for
 //     the backward.
-//   Phase 4 (output): only the flagged key tiles. Recompute S and form
-//     A = u^{1/(alpha-1)} and g = u^{(2-alpha)/(alpha-1)}. Both go to TMEM in fp16,
-//     over the S columns they replace. Then the tensor cores compute O += A V and
-//     Ot += g V, reading the A operand from TMEM, with B an fp16 copy of V. fp16 rounds
-//     at 2^-11; a bf16 A or g (2^-8) would cost more than the output and gradient
-//     tolerances once g reaches dK through delta. sum_j g_ij is kept per row for the
-//     backward.
+//   Phase 4 (output): only the flagged key tiles. Recompute S, form A = u^{1/(alpha-1)}
+//     in fp16 (2^-11 rounding; bf16 would give 2^-8) over the S columns it replaces, and
+//     compute O += A V on the tensor cores with the A operand read from TMEM and B an fp16
+//     copy of V. The backward's delta = sum_j g_ij dO_i . V_j / sum_j g_ij needs the
+//     support of each row, not a g V product: the row owners list every key with u > 0
+//     (index and u) per row and column part, and a small kernel of the backward sums over
+//     those lists in fp32.
 //
 // Roles (640 threads): warps 0-15 are row owners. Warp w reads TMEM lanes 32(w%4)..+31
 // (one query row per lane) and columns [32(w/4), 32(w/4)+32) of every S tile, so four
 // threads share a row and combine partial sums in shared memory; four warps per SM
-// sub-partition hide the latency of the per-score work. Warp 16 issues TMA
-// loads into a 4-slot ring of 16 KB K/V tiles. Warp 17 owns TMEM and issues the S = Q K^T
-// MMAs of every phase; in the output pass warp 19 issues the O = A V chain and warp 18
-// the Ot = g V chain. One thread issues an N=64 MMA only every ~54 cycles and each
-// mbarrier wait costs ~200 cycles even when the phase is complete, so one issuer per
-// chain keeps each below the tile's tensor time.
-// TMEM (512 columns): during the sweeps, four S buffers at 0/128/256/384, so the MMA
-// warp runs up to three tiles ahead. During the output pass (OutLayout):
+// sub-partition hide the latency of the per-score work. Warp 16 issues TMA loads into a
+// 4-slot ring of 16 KB K/V tiles. Warps 17 and 18 issue the S = Q K^T MMAs of the max pass
+// and the sweeps, alternating tiles (one thread blocks while its MMAs enter the tensor
+// pipe, so two issuers keep the pipe fed while each probes barriers and commits); warp 17
+// owns TMEM and issues the output pass's S tiles, and warp 19 the O = A V chain.
+// TMEM (512 columns): during the sweeps, four S buffers at 0/128/256/384, so the issuers
+// run up to three tiles ahead. During the output pass (OutLayout):
 //   - three S buffers at 0, 128 and 384, tile k in buffer k % 3. The row owner of keys
-//     [32q, 32q+32) writes their A (fp16 pairs) into columns [32q, 32q+16) and g into
-//     [32q+16, 32q+32): only over S columns it has read itself;
-//   - O at [256,320) and Ot at [320,384).
-// alpha = 1.5 splits g = g_hi + g_lo, both fp16: g_lo of tile k goes to shared-memory
-// buffer k % 3 (a K-major [128 rows][128 keys] operand), and the Ot chain adds g_lo V as
-// shared-memory MMAs. The three buffers (96 KB) reuse the tile maxima and candidate lists,
-// which are dead once the final mask is decided.
+//     [32q, 32q+32) writes their A (fp16 pairs) into columns [32q, 32q+16): only over S
+//     columns it has read itself;
+//   - O at [256,320).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -65,13 +61,14 @@ constexpr int kOCols = kD / kParts;           // output columns per thread in th
 constexpr int kThreads = (kMathWarps + 4) * 32;
 constexpr int kMathThreads = kMathWarps * 32;
 constexpr int kProducerWarp = kMathWarps;
-constexpr int kMmaWarp = kMathWarps + 1;
-constexpr int kMma2Warp = kMathWarps + 2;     // second MMA issuer: the Ot = g V chain of the output pass
-constexpr int kMma3Warp = kMathWarps + 3;     // third MMA issuer: the O = A V chain of the output pass
+constexpr int kMmaWarp = kMathWarps + 1;      // S issuer 0 (even tiles of the max pass and sweeps; the output pass)
+constexpr int kSWarp2 = kMathWarps + 2;       // S issuer 1 (odd tiles of the max pass and sweeps)
+constexpr int kOWarp = kMathWarps + 3;        // the O = A V chain of the output pass
 constexpr int kOBufsMax = 3;    // S/A buffers in the output pass (at most; see OutLayout)
 constexpr int kSlots = 4;
 constexpr int kSBufs = 4;
-constexpr int kCandPerThread = kTile / kParts;   // candidates per (row, column part); 128 per row
+constexpr int kCandPerThread = kTile / kParts;   // candidates per (row, column part) for L <= 8192
+constexpr int kCandLong = 24;                     // the same above 64 key tiles (shared memory)
 constexpr float kTolF = 3e-5f;         // |f(tau)| = |sum p - 1| small enough to stop sweeping
 constexpr int kMaxVotes = 72;
 
@@ -169,18 +166,17 @@ __device__ __forceinline__ void ldw(uint32_t taddr, uint32_t (&o)[N]) {
 template <int AK>
 struct OutLayout {
   static constexpr int kBufs = 3;
-  static constexpr bool kSplitG = AK == kAlpha15;
   __device__ static __forceinline__ uint32_t sbuf(int c) { return c == 0 ? 0u : (c == 1 ? 128u : 384u); }
 };
-constexpr int kGloBytes = 2 * kTileBytes;          // one g_lo buffer: [128 rows][128 keys] fp16
-constexpr int kGloRegion = 3 * kGloBytes;          // three buffers
 
 // Shared-memory layout of the forward (offsets from the 1024-aligned base): Q tile, K/V
-// ring, then a region holding the tile maxima [Tc][128] and the candidate lists during
-// the max pass and sweeps, and the g_lo buffers during the output pass, then partials.
+// ring, the tile maxima [Tc][128], the candidate scores [4][cap][128] (fp32) and key
+// indices [4][cap][128] (uint16), the partials. cap = 32 candidates per row and column part
+// up to 64 key tiles, 24 beyond (so that L = 16384 fits in 227 KB).
+__host__ __device__ constexpr int fwd_cand_cap(int Tc) { return Tc > 64 ? kCandLong : kCandPerThread; }
 __host__ __device__ constexpr int fwd_off_region() { return kTileBytes * (1 + 4); }
 __host__ __device__ constexpr int fwd_region_bytes(int Tc) {
-  return Tc * kTile * 4 + 4 * 32 * kTile * 4 > kGloRegion ? Tc * kTile * 4 + 4 * 32 * kTile * 4 : kGloRegion;
+  return Tc * kTile * 4 + 4 * fwd_cand_cap(Tc) * kTile * (4 + 2);
 }
 
 // fp16 pair -> two floats (exact).
@@ -190,6 +186,22 @@ __device__ __forceinline__ float2 unpack_f16x2(uint32_t w) {
       : "=f"(lo), "=f"(hi)
       : "r"(w));
   return make_float2(lo, hi);
+}
+
+// Appends the scores of an 8-key group that pass tau (u = s cz - tau > 0) to this thread's
+// candidate copies, without branches: every element is written to slot min(nc, cap-1) and
+// nc advances only on a pass. A failing element lands in the next free slot, which the next
+// passing one overwrites; once the list is full (nc >= cap) the copies are not used.
+__device__ __forceinline__ void collect8(const float* s, int j, float cz, float tau, int cap, float* mycand,
+                                         uint16_t* myidx, int& nc) {
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const bool pass = fmaf(s[e], cz, -tau) > 0.f;
+    const int slot = min(nc, cap - 1);
+    mycand[slot * kTile] = s[e];
+    myidx[slot * kTile] = (uint16_t)(j + e);
+    nc += pass ? 1 : 0;
+  }
 }
 
 // Adds one candidate at u = z - t to the sums of the current support (u > 0), without
@@ -301,12 +313,13 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
   extern __shared__ uint8_t dsm_raw[];
   __shared__ Shared sh;
   uint8_t* dsm = align1024(dsm_raw);
-  static_assert(kSlots == 4 && kCandPerThread == 32 && kParts == 4, "fwd_region_bytes assumes these");
+  static_assert(kSlots == 4 && kParts == 4, "fwd_region_bytes assumes these");
   uint8_t* sQ = dsm;
   uint8_t* ring = dsm + kTileBytes;
   int* tmax = reinterpret_cast<int*>(dsm + fwd_off_region());    // [Tc][128], f2ord
-  float* cand = reinterpret_cast<float*>(tmax + p.Tc * kTile);   // [kParts][kCandPerThread][128]
-  uint8_t* glo = dsm + fwd_off_region();                         // output pass: g_lo buffers (alpha 1.5)
+  const int cap = fwd_cand_cap(p.Tc);
+  float* cand = reinterpret_cast<float*>(tmax + p.Tc * kTile);   // [kParts][cap][128] scores
+  uint16_t* cidx = reinterpret_cast<uint16_t*>(cand + kParts * cap * kTile);   // [kParts][cap][128] key indices
   float* part = reinterpret_cast<float*>(dsm + fwd_off_region() + fwd_region_bytes(p.Tc));   // [kParts][4][128]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -321,7 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
   if (tid == 0) {
     for (int s = 0; s < kSlots; ++s) {
       mbar_init(&sh.full[s], 1);
-      mbar_init(&sh.empty[s], 2);   // two commits: one per MMA issuer reading the slot
+      mbar_init(&sh.empty[s], 1);   // one commit by the MMA issuer that reads the slot
     }
     mbar_init(&sh.bar_q, 1);
     for (int s = 0; s < kSBufs; ++s) {
@@ -331,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     for (int s = 0; s < kOBufsMax; ++s) {
       mbar_init(&sh.o_full[s], 1);
       mbar_init(&sh.o_ready[s], kMathWarps);
-      mbar_init(&sh.pv_done[s], 2);   // O chain and Ot chain
+      mbar_init(&sh.pv_done[s], 1);   // the O chain
     }
     mbar_init(&sh.mma_drain, 3);   // one commit per MMA issuer
     mbar_init(&sh.never, 1);
@@ -419,12 +432,16 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         mbar_drain(&sh.full[k % kSlots], (k / kSlots) & 1, status);
     }
     __syncwarp();
-  } else if (warp == kMmaWarp) {
+  } else if (warp == kMmaWarp || warp == kSWarp2) {
     // ------------------------------------------------------------------- MMA issuer
     uint32_t seq = 0;            // next ring position (sweeps consume in order)
     uint32_t sfree_par = 0;      // per sweep S buffer: parity of its uses so far (bit b)
     uint32_t sbuf = 0;           // next sweep S buffer
     bool live = true;            // false after a failed wait: no further MMA is issued
+    // Two S issuers share the max pass and the sweeps: issuer me takes the tiles whose
+    // buffer (tile index % 4) has parity me, so each one's barrier probes and commits
+    // overlap the other's MMAs. Both walk every tile to keep the positions and parities.
+    const uint32_t me = warp == kMmaWarp ? 0u : 1u;
     DIAG(long long dg_sw = 0; long long dg_out = 0; long long dg_iss = 0);
     const uint32_t idS = idesc_bf16(128, 128, 0, 0);
     const uint64_t qd0 = sdesc_sw128(smem_u32(sQ), 16, 1024);      // Q tile, K-major
@@ -436,27 +453,28 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       const uint64_t kd = sdesc_add(kd0, slot * kTileBytes);
 #pragma unroll
       for (int k = 0; k < 4; ++k) mma_ss(T + dcol, sdesc_add(qd0, k * 32), sdesc_add(kd, k * 32), idS, k > 0);
-      mma_commit(&sh.empty[slot]);   // a K slot is read by this issuer only: both arrivals here
-      mma_commit(&sh.empty[slot]);
+      mma_commit(&sh.empty[slot]);   // a K slot is read by this issuer only
     };
     auto sweep_tile = [&]() {
       const uint32_t bf = sbuf;
       const uint32_t pos = seq++;
-      // S buffer consumed by the row owners, and K tile landed.
-      DIAG(const long long d0 = clock64());
-      live = live && mbar_wait2(&sh.s_free[bf], ((sfree_par >> bf) & 1) ^ 1, &sh.full[pos % kSlots],
-                                (pos / kSlots) & 1, wc);
-      DIAG(dg_sw += clock64() - d0);
-      sfree_par ^= 1u << bf;
-      if (live) {
-        mma_s(pos, bf * 128);
-        mma_commit(&sh.s_full[bf]);
+      if ((bf & 1u) == me) {
+        // S buffer consumed by the row owners, and K tile landed.
+        DIAG(const long long d0 = clock64());
+        live = live && mbar_wait2(&sh.s_free[bf], ((sfree_par >> bf) & 1) ^ 1, &sh.full[pos % kSlots],
+                                  (pos / kSlots) & 1, wc);
+        DIAG(dg_sw += clock64() - d0);
+        if (live) {
+          mma_s(pos, bf * 128);
+          mma_commit(&sh.s_full[bf]);
+        }
+        DIAG(dg_iss += clock64() - d0);
       }
-      DIAG(dg_iss += clock64() - d0);
+      sfree_par ^= 1u << bf;
       sbuf = (sbuf + 1) & (kSBufs - 1);
     };
     if (lane == 0) {
-      if (p.selftest & kSelftestStall) live = mbar_wait(&sh.never, 0, wc);   // expires: nothing completes it
+      if ((p.selftest & kSelftestStall) && me == 0) live = mbar_wait(&sh.never, 0, wc);   // expires: nothing completes it
       live = live && mbar_wait(&sh.bar_q, 0, wc);
       for_each_bit(act, kMaskWords, [&](int) { sweep_tile(); });
     }
@@ -471,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         if (kind == kKindSweep) {
           sbuf = 0;
           for_each_bit(list, kMaskWords, [&](int) { sweep_tile(); });
-        } else {
+        } else if (me == 0) {
           // Output pass: this warp issues only the S tiles; tile k uses buffer c = k % 3
           // at TMEM column 0, 128 or 384, which is free once O and Ot of tile k-3 are done.
           // K_k is at ring position base + 2k, V_k at base + 2k + 1.
@@ -502,56 +520,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       __syncwarp();
       if (kind != kKindSweep) break;
     }
-  } else if (warp == kMma2Warp) {
-    // ------------------------------------------------ second MMA issuer (output pass)
-    const uint32_t idO = idesc_f16(128, 64, 0, 1);
-    const uint64_t vd0 = sdesc_sw128(smem_u32(ring), 8192, 1024);   // ring slot 0, MN-major
-    const uint64_t gd0 = sdesc_sw128(smem_u32(glo), 16, 1024);      // g_lo buffer 0, K-major
-    uint32_t seq = 0;   // ring positions, tracked exactly like the producer's
-    for_each_bit(act, kMaskWords, [&](int) { ++seq; });
-    while (true) {
-      named_bar(1, kThreads);
-      const int kind = sh.ctl_kind;
-      uint32_t list[kMaskWords];
-#pragma unroll
-      for (int w = 0; w < kMaskWords; ++w) list[w] = sh.lists[sh.ctl_buf][w];
-      int n = 0;
-#pragma unroll
-      for (int w = 0; w < kMaskWords; ++w) n += __popc(list[w]);
-      if (kind == kKindSweep) {
-        seq += n;
-      } else if (lane == 0) {
-        const uint32_t base = seq;
-        for (int k = 0; k < n; ++k) {
-          const int c = k % kOBufs;
-          const uint32_t pa = OL::sbuf(c);
-          const uint32_t vpos = base + 2 * k + 1;
-          const int vslot = vpos % kSlots;
-          if (!mbar_wait2(&sh.full[vslot], (vpos / kSlots) & 1, &sh.o_ready[c], (k / kOBufs) & 1, wc)) break;
-          tc_fence_after();
-          const uint64_t vd = sdesc_add(vd0, vslot * kTileBytes);
-#pragma unroll
-          for (int t = 0; t < 8; ++t) {
-            // keys 16t..16t+15: part 16t / kCols, pair columns ((16t) % kCols) / 2 of its A block
-            const uint32_t col = pa + (16 * t / kCols) * kCols + ((16 * t) % kCols) / 2 + kCols / 2;   // g block
-            mma_ts(T + 320, T + col, sdesc_add(vd, t * 2048), idO, (k > 0 || t > 0) ? 1u : 0u);
-          }
-          if constexpr (OL::kSplitG) {
-            // g_lo of keys 16t..16t+15: panel t / 4 of buffer c, 32-byte step t % 4.
-#pragma unroll
-            for (int t = 0; t < 8; ++t)
-              mma_ss(T + 320, sdesc_add(gd0, c * kGloBytes + (t >> 2) * kTileBytes + (t & 3) * 32),
-                     sdesc_add(vd, t * 2048), idO, 1u);
-          }
-          mma_commit(&sh.empty[vslot]);
-          mma_commit(&sh.pv_done[c]);
-        }
-      }
-      __syncwarp();
-      if (kind != kKindSweep) break;
-    }
-  } else if (warp == kMma3Warp) {
-    // ------------------------------------------------- third MMA issuer (output pass)
+  } else if (warp == kOWarp) {
+    // ------------------------------------------------------ O issuer (output pass)
     const uint32_t idO = idesc_f16(128, 64, 0, 1);
     const uint64_t vd0 = sdesc_sw128(smem_u32(ring), 8192, 1024);   // ring slot 0, MN-major
     uint32_t seq = 0;   // ring positions, tracked exactly like the producer's
@@ -586,7 +556,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
             const uint32_t col = pa + (16 * t / kCols) * kCols + ((16 * t) % kCols) / 2;   // A block
             mma_ts(T + 256, T + col, sdesc_add(vd, t * 2048), idO, (k > 0 || t > 0) ? 1u : 0u);
           }
-          mma_commit(&sh.empty[vslot]);
+          mma_commit(&sh.empty[vslot]);   // V_k is read by this issuer only
           mma_commit(&sh.pv_done[c]);
         }
         DIAG(p.stats[((size_t)bh * p.Tr + qt) * kFwdStats + 14] = (int)dg_o);
@@ -668,13 +638,15 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     float hi = mz - ((AK == kAlpha15) ? rsqrtf((float)n_act) : 1.f / (float)n_act);
     float tau = INFINITY;
     bool done = !valid;
+    bool listed = false;   // solved on candidate copies that hold the whole support
+    bool near_once = false;   // a Newton correction within tolerance was taken while the copies overflowed
+    int nc = 0;            // this thread's candidate count in the sweep that solved its row
     if (valid) {
       // The row's largest part-tile maxima are a subset of its scores, so the threshold
       // of entmax on them is a lower bound tau_T <= tau*.
       const float t = solveN<AK, 4 * kParts>(vt, cz, lo, hi);
       tau = fminf(fmaxf(t, lo), hi);
     }
-    float2 sg2 = make_float2(0.f, 0.f);   // sum_j g_ij, two chains
     int sweeps = 0;
     uint32_t n_s = 0;   // S tiles computed (phase 1, sweeps, output) for the counters
     for_each_bit(act, kMaskWords, [&](int) { ++n_s; });
@@ -745,7 +717,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
             for (int cc = 0; cc < kCols; ++cc)
               if (!pat.active(i, j0 + cc)) s[cc] = -INFINITY;
           }
-          uint32_t aw[kCols / 2], gw[kCols / 2], lw[kCols / 2];
+          // A = u^{1/(alpha-1)} in fp16 pairs.
+          uint32_t aw[kCols / 2];
 #pragma unroll
           for (int cc = 0; cc < kCols / 2; ++cc) {
             const float2 u = __ffma2_rn(make_float2(s[2 * cc], s[2 * cc + 1]), make_float2(cz, cz),
@@ -754,37 +727,17 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
             if (AK == kAlpha15) {
               const float2 a = __fmul2_rn(make_float2(v0, v1), make_float2(v0, v1));
               aw[cc] = pack_f16(a.x, a.y);
-              gw[cc] = pack_f16(v0, v1);
-              const float2 gh = unpack_f16x2(gw[cc]);
-              const float2 gl = __ffma2_rn(gh, make_float2(-1.f, -1.f), make_float2(v0, v1));   // exact
-              lw[cc] = pack_f16(gl.x, gl.y);
-              sg2 = __fadd2_rn(sg2, make_float2(v0, v1));
             } else {
-              const float g0 = u.x > 0.f ? 1.f : 0.f, g1 = u.y > 0.f ? 1.f : 0.f;
               aw[cc] = pack_f16(v0, v1);
-              gw[cc] = pack_f16(g0, g1);
-              sg2 = __fadd2_rn(sg2, make_float2(g0, g1));
             }
           }
-          // This part's keys qp*kCols.. go back into its own S columns [qp*kCols, +kCols):
-          // A (fp16 pairs) in the first half, g in the second. Writing only into columns this
-          // thread has read keeps the row's other parts from seeing overwritten S values.
+          // This part's keys qp*kCols.. go back into its own S columns [qp*kCols, +kCols/2):
+          // writing only into columns this thread has read keeps the row's other parts from
+          // seeing overwritten S values.
           const uint32_t col = pa + qp * kCols;
           DIAG(const long long d3 = clock64(); dgr[7] += d3 - d2);
 #pragma unroll
-          for (int h = 0; h < kCols / 32; ++h) {
-            tmem_st16(tl + col + 16 * h, *reinterpret_cast<uint32_t(*)[16]>(&aw[16 * h]));
-            tmem_st16(tl + col + kCols / 2 + 16 * h, *reinterpret_cast<uint32_t(*)[16]>(&gw[16 * h]));
-          }
-          if constexpr (OL::kSplitG) {
-            // keys [32 qp, 32 qp + 32): panel qp / 2, 16-byte chunks 4 (qp % 2) .. + 3 of the row.
-            uint8_t* gb = glo + c * kGloBytes + (qp >> 1) * kTileBytes;
-#pragma unroll
-            for (int cc = 0; cc < 4; ++cc)
-              *reinterpret_cast<uint4*>(gb + sw128_offset(row, ((qp & 1) * 4 + cc) * 8)) =
-                  make_uint4(lw[4 * cc], lw[4 * cc + 1], lw[4 * cc + 2], lw[4 * cc + 3]);
-            fence_proxy_async_smem();   // generic-proxy stores, read by the tensor cores
-          }
+          for (int h = 0; h < kCols / 32; ++h) tmem_st16(tl + col + 16 * h, *reinterpret_cast<uint32_t(*)[16]>(&aw[16 * h]));
           tmem_wait_st();
           tc_fence_before();
           warp_arrive(&sh.o_ready[c]);
@@ -793,10 +746,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           ++n_s;
         });
         const int n_out = k;
-        // Epilogue: O and Ot from TMEM (each thread of a row writes kOCols of the 64 columns).
+        // Epilogue: O from TMEM (each thread of a row writes kOCols of the 64 columns).
         if (n_out > 0) warp_wait(&sh.pv_done[(n_out - 1) % kOBufs], ((n_out - 1) / kOBufs) & 1, wc);
         tc_fence_after();
-        part[(qp * 4 + 1) * kTile + row] = sg2.x + sg2.y;
         uint32_t o[kOCols];
         ldw(tl + 256 + qp * kOCols, o);
         if (valid) {
@@ -806,22 +758,59 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
             dst[cc] = make_float4(__uint_as_float(o[4 * cc]), __uint_as_float(o[4 * cc + 1]),
                                   __uint_as_float(o[4 * cc + 2]), __uint_as_float(o[4 * cc + 3]));
         }
-        __syncwarp();
-        ldw(tl + 320 + qp * kOCols, o);
+        // The backward's delta needs Ot_i = sum_j g_ij V_j and sum_j g_ij over row i's support.
+        // A row solved on its candidate copies has them all in shared memory (scores and key
+        // indices from the sweep that solved it), so each of its four threads sums g V_j
+        // over 16 of the 64 columns in fp32, gathering the fp16 V rows (just streamed by this
+        // CTA, so in L2). A row without complete copies (refinement cap, or a Newton finish)
+        // gets sum g = -1, and the backward recomputes its support.
         if (valid) {
-          float4* dst = reinterpret_cast<float4*>(p.Ot + ((size_t)bh * p.L + i) * kD + qp * kOCols);
+          const size_t rix = (size_t)bh * p.L + i;
+          if (listed) {
+            float acc[kOCols];
 #pragma unroll
-          for (int cc = 0; cc < kOCols / 4; ++cc)
-            dst[cc] = make_float4(__uint_as_float(o[4 * cc]), __uint_as_float(o[4 * cc + 1]),
-                                  __uint_as_float(o[4 * cc + 2]), __uint_as_float(o[4 * cc + 3]));
-        }
-        named_bar(3, kMathThreads);
-        if (valid && qp == 0) {
-          float sg = 0.f;
+            for (int cc = 0; cc < kOCols; ++cc) acc[cc] = 0.f;
+            float sgv = 0.f;
+            const uint4* vbase = reinterpret_cast<const uint4*>(p.V16 + (size_t)bh * p.L * kD + qp * kOCols);
+            for (int q = 0; q < kParts; ++q) {
+              const int nq = (int)part[(q * 4 + 2) * kTile + row];
+              for (int k0 = 0; k0 < nq; k0 += 4) {   // four V rows in flight
+                float gk[4];
+                uint4 vw[4][kOCols / 8];
 #pragma unroll
-          for (int q = 0; q < kParts; ++q) sg += part[(q * 4 + 1) * kTile + row];
-          p.tau[(size_t)bh * p.L + i] = tau;
-          p.sumg[(size_t)bh * p.L + i] = sg;
+                for (int t = 0; t < 4; ++t) {
+                  const int e = (q * cap + min(k0 + t, nq - 1)) * kTile + row;
+                  const float u = fmaf(cand[e], cz, -tau);
+                  gk[t] = (k0 + t < nq && u > 0.f) ? ((AK == kAlpha15) ? u : 1.f) : 0.f;
+                  const uint4* vr = vbase + (size_t)cidx[e] * (kD / 8);
+#pragma unroll
+                  for (int h = 0; h < kOCols / 8; ++h) vw[t][h] = vr[h];
+                }
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                  sgv += gk[t];
+#pragma unroll
+                  for (int h = 0; h < kOCols / 8; ++h) {
+                    const uint32_t w4[4] = {vw[t][h].x, vw[t][h].y, vw[t][h].z, vw[t][h].w};
+#pragma unroll
+                    for (int c2 = 0; c2 < 4; ++c2) {
+                      const float2 f = unpack_f16x2(w4[c2]);
+                      acc[8 * h + 2 * c2] = fmaf(gk[t], f.x, acc[8 * h + 2 * c2]);
+                      acc[8 * h + 2 * c2 + 1] = fmaf(gk[t], f.y, acc[8 * h + 2 * c2 + 1]);
+                    }
+                  }
+                }
+              }
+            }
+            float4* dst = reinterpret_cast<float4*>(p.Ot + rix * kD + qp * kOCols);
+#pragma unroll
+            for (int cc = 0; cc < kOCols / 4; ++cc)
+              dst[cc] = make_float4(acc[4 * cc], acc[4 * cc + 1], acc[4 * cc + 2], acc[4 * cc + 3]);
+            if (qp == 0) p.sumg[rix] = sgv;
+          } else if (qp == 0) {
+            p.sumg[rix] = -1.f;
+          }
+          if (qp == 0) p.tau[rix] = tau;
         }
         if (tid == 0) {
           int na = 0;
@@ -845,10 +834,13 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       // thread's 32 scores and a test against tau, with an element scan only when that
       // max passes (rare). Later sweeps (rows whose candidates overflowed, or Newton
       // steps) also accumulate S1, S2 and the count for f(tau) and f'(tau).
+      // A row already solved keeps the copies (and count) of the sweep that solved it.
       const bool cand_only = sweeps == 0;
+      const bool collect = !done;
       float S1 = 0.f, S2 = 0.f;
-      int nc = 0;
-      float* mycand = cand + qp * kCandPerThread * kTile + row;
+      if (collect) nc = 0;
+      float* mycand = cand + qp * cap * kTile + row;
+      uint16_t* myidx = cidx + qp * cap * kTile + row;
       sbuf = 0;
       DIAG(const long long dsw0 = clock64());
       for_each_bit(list, kMaskWords, [&](int jt) {
@@ -879,21 +871,12 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
             const float* x = s + 8 * g;
             gm[g] = fmaxf(fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3])), fmaxf(fmaxf(x[4], x[5]), fmaxf(x[6], x[7])));
           }
-          const float tm = fmaxf(fmaxf(gm[0], gm[1]), fmaxf(gm[2], gm[3]));
-          if (fmaf(tm, cz, -tau) > 0.f) {
+          // Groups are scanned when any lane of the warp has a candidate in them (a
+          // warp-uniform branch), each lane then runs the same branch-free append.
 #pragma unroll
-            for (int g = 0; g < kCols / 8; ++g) {
-              if (fmaf(gm[g], cz, -tau) > 0.f) {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                  if (fmaf(s[8 * g + e], cz, -tau) > 0.f) {
-                    if (nc < kCandPerThread) mycand[nc * kTile] = s[8 * g + e];
-                    ++nc;
-                  }
-                }
-              }
-            }
-          }
+          for (int g = 0; g < kCols / 8; ++g)
+            if (__any_sync(0xffffffffu, collect && fmaf(gm[g], cz, -tau) > 0.f))
+              if (collect) collect8(s + 8 * g, j0 + 8 * g, cz, tau, cap, mycand, myidx, nc);
           ++n_s;
           sbuf = (sbuf + 1) & (kSBufs - 1);
           DIAG(dgr[5] += clock64() - dtk);
@@ -923,20 +906,10 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           s1[g & 3] = __fadd2_rn(s1[g & 3], gs);
           gmask |= (gs.x + gs.y > 0.f ? 1u : 0u) << g;
         }
-        if (gmask) {
 #pragma unroll
-          for (int g = 0; g < kCols / 8; ++g) {
-            if ((gmask >> g) & 1u) {
-#pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                if (fmaf(s[8 * g + e], cz, -tau) > 0.f) {
-                  if (nc < kCandPerThread) mycand[nc * kTile] = s[8 * g + e];
-                  ++nc;
-                }
-              }
-            }
-          }
-        }
+        for (int g = 0; g < kCols / 8; ++g)
+          if (__any_sync(0xffffffffu, collect && ((gmask >> g) & 1u)))
+            if (collect) collect8(s + 8 * g, j0 + 8 * g, cz, tau, cap, mycand, myidx, nc);
         const float2 s1t = __fadd2_rn(__fadd2_rn(s1[0], s1[1]), __fadd2_rn(s1[2], s1[3]));
         const float2 s2t = __fadd2_rn(__fadd2_rn(s2[0], s2[1]), __fadd2_rn(s2[2], s2[3]));
         S1 += s1t.x + s1t.y;
@@ -963,7 +936,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         S2 += pq[kTile];
         ncs[q] = (int)pq[2 * kTile];
         ntot += ncs[q];
-        fits = fits && ncs[q] <= kCandPerThread;
+        fits = fits && ncs[q] < cap;   // collect8 keeps the last slot free
       }
       const float C = (float)ntot;   // support size at tau (alpha = 2: |f'(tau)|)
       named_bar(3, kMathThreads);   // partials consumed before anyone rewrites them
@@ -972,9 +945,10 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         // tau = tau_T <= tau*: if the copies fit they hold the support; solve on them.
         // Otherwise tau stays and the next sweep measures f(tau) and f'(tau).
         float t;
-        if (fits && solve_list<AK>(cand + row, ncs, kCandPerThread * kTile, kTile, cz, tau, lo, hi, t)) {
+        if (fits && solve_list<AK>(cand + row, ncs, cap * kTile, kTile, cz, tau, lo, hi, t)) {
           tau = t;
           done = true;
+          listed = true;
         }
       } else if (!done) {
         const float f = (AK == kAlpha15) ? S2 - 1.f : S1 - 1.f;
@@ -984,17 +958,27 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           // tau <= tau*, so every score of the support is in the candidate lists: the
           // exact solve on chip ends the refinement.
           float t;
-          if (solve_list<AK>(cand + row, ncs, kCandPerThread * kTile, kTile, cz, tau, lo, hi, t)) {
+          if (solve_list<AK>(cand + row, ncs, cap * kTile, kTile, cz, tau, lo, hi, t)) {
             tau = t;
             done = true;
+            listed = true;
           }
         }
         if (!done) {
           // f is a sum of C positive terms in fp32; its rounding error grows with C.
           const float tolf = fmaxf(kTolF, C * 0x1p-22f);
-          if (fabsf(f) <= tolf && fp > 0.f) {
-            tau += f / fp;   // final Newton correction, no further sweep needed
+          if (fabsf(f) <= tolf && fp > 0.f && (fits || near_once)) {
+            // Final Newton correction, no further sweep needed. The copies of this sweep
+            // hold the support when they fit (tau moves by at most the tolerance over the
+            // slope). When they do not, the row first sweeps once more at the corrected
+            // tau, where fewer scores qualify; only a row whose support exceeds the copies
+            // then ends without them.
+            tau += f / fp;
             done = true;
+            listed = fits;
+          } else if (fabsf(f) <= tolf && fp > 0.f) {
+            tau += f / fp;
+            near_once = true;
           } else {
             float t = tau + f / fp;
             if (!(t > lo && t <= hi && t != tau)) t = 0.5f * (lo + hi);   // safeguard; the root may sit at hi
@@ -1007,7 +991,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
 
   // No MMA may still write tensor memory when it is freed: each issuer commits once more
   // and waits for all three commits (a drain, bounded and independent of the abort flag).
-  if ((warp == kMmaWarp || warp == kMma2Warp || warp == kMma3Warp) && lane == 0) {
+  if ((warp == kMmaWarp || warp == kSWarp2 || warp == kOWarp) && lane == 0) {
     mma_commit(&sh.mma_drain);
     mbar_drain(&sh.mma_drain, 0, status);
   }

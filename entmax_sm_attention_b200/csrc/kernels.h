@@ -29,8 +29,9 @@ struct FwdParams {
   CUtensorMap tQ, tK, tV;   // [B*H][L][64], box 64 x 128 x 1, 128-byte swizzle (Q, K bf16; V fp16)
   float* O;                 // [B*H][L][64]
   float* tau;               // [B*H][L]
-  float* sumg;              // [B*H][L]      sum_j g_ij
+  float* sumg;              // [B*H][L]      sum_j g_ij over the support (-1: not listed, see fwd.cu)
   float* Ot;                // [B*H][L][64]  sum_j g_ij V_j
+  const uint16_t* V16;      // [B*H][L][64]  fp16 copy of V
   uint32_t* M;              // [B*H][Tr][Wc]
   uint32_t* MT;             // [B*H][Tc][Wr] (zeroed before the launch)
   int* stats;               // [B*H][Tr][kFwdStats] (layout above)
@@ -63,6 +64,24 @@ struct BwdParams {
   int selftest;
 };
 
+// Inputs of the backward's delta kernel (bwd.cu).
+struct DeltaParams {
+  const uint16_t* Q;            // bf16 [B*H][L][64]
+  const uint16_t* K;
+  const uint16_t* V;
+  const uint16_t* V16;          // fp16 copy of V (made by the forward)
+  const uint16_t* dO;
+  const float* tau;             // [B*H][L]
+  const float* Ot;              // [B*H][L][64]
+  const float* sumg;            // [B*H][L] (-1: the forward did not list the row's support)
+  const uint32_t* M;            // [B*H][Tr][Wc]
+  float* delta;                 // [B*H][L]
+  const int* kv_len;
+  int H, L, Tr, Wc, BH;
+  float cz;
+  int causal, window;
+};
+
 struct FwdF32Params {
   const float* Q;           // fp32 [B*H][L][64]
   const float* K;
@@ -87,8 +106,7 @@ cudaError_t launch_fwd(bool alpha15, const FwdParams& p, int grid, cudaStream_t 
 cudaError_t launch_fwd_f32(bool alpha15, const FwdF32Params& p, int grid, cudaStream_t s);
 cudaError_t launch_bwd(bool alpha15, const BwdParams& p, int grid, cudaStream_t s);
 cudaError_t launch_bf16_to_f16(const void* src, void* dst, long elems, int* status, cudaStream_t s);
-cudaError_t launch_delta(const uint16_t* dO, const float* Ot, const float* sumg, float* delta, long rows,
-                         cudaStream_t s);
+cudaError_t launch_delta(bool alpha15, const DeltaParams& p, cudaStream_t s);
 cudaError_t launch_rows(bool alpha15, const float* S, int rows, int n, long ld, float* P, float* tau, int* status,
                         cudaStream_t s);
 

@@ -42,7 +42,7 @@ def test_marginal_throughput_recovers_the_slope():
     pts = []
     for flagged in (24000, 12000, 6000, 3000, 1500):
         s_tiles = 24960 + 2 * flagged
-        fl = bench.UNIT_FLOP * (s_tiles + 2 * flagged)
+        fl = bench.UNIT_FLOP * (s_tiles + flagged)
         bl = bench.UNIT_FLOP * 5 * flagged
         f_ms = 0.2 + fl / 500e12 * 1e3
         b_ms = 0.05 + bl / 600e12 * 1e3
@@ -109,7 +109,7 @@ def test_pair_work_matches_brute_force():
                 a_i = act.sum(1)
                 f_i = (act & blk).sum(1)
                 r_i = R[b, h][np.arange(w.L) // 128]
-                fwd += int(((1 + r_i) * a_i).sum() * 128 + 3 * f_i.sum() * 128)
+                fwd += int(((1 + r_i) * a_i).sum() * 128 + 2 * f_i.sum() * 128)
                 bwd += int(5 * f_i.sum() * 128)
                 act_total += int(a_i.sum())
                 fl_total += int(f_i.sum())
