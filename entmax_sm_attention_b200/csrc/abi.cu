@@ -195,7 +195,7 @@ extern "C" entmax_status entmax_attn_fwd(const entmax_attn_desc* d, const void* 
   p.tau = tau;
   p.sumg = reinterpret_cast<float*>(w + l.off_sumg);
   p.Ot = reinterpret_cast<float*>(w + l.off_Ot);
-  p.V16 = static_cast<const uint16_t*>(v16);
+  p.Vb = static_cast<const uint16_t*>(V);
   p.M = reinterpret_cast<uint32_t*>(w + l.off_M);
   p.MT = reinterpret_cast<uint32_t*>(w + l.off_MT);
   p.stats = reinterpret_cast<int*>(w + l.off_stats);

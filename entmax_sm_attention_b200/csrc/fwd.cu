@@ -577,6 +577,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     float top[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
     DIAG(long long dg_s1 = 0; long long dg_s2 = 0; long long dg_s3 = 0; long long dg_sw1 = 0);
     DIAG(long long dgr[9] = {0, 0, 0, 0, 0, 0, 0, 0, 0}; long long dtk = 0);
+    DIAG(long long dgx[6] = {0, 0, 0, 0, 0, 0});   // [26] tau_T solve, [27] decisions, [28] post-sweep solves, [29] epilogue
 
     // Phase 1: per-key-tile row maxima over this thread's column part (combined in smem).
     for_each_bit(act, kMaskWords, [&](int jt) {
@@ -644,8 +645,10 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     if (valid) {
       // The row's largest part-tile maxima are a subset of its scores, so the threshold
       // of entmax on them is a lower bound tau_T <= tau*.
+      DIAG(const long long ds0 = clock64());
       const float t = solveN<AK, 4 * kParts>(vt, cz, lo, hi);
       tau = fminf(fmaxf(t, lo), hi);
+      DIAG(dgx[0] += clock64() - ds0);
     }
     int sweeps = 0;
     uint32_t n_s = 0;   // S tiles computed (phase 1, sweeps, output) for the counters
@@ -653,6 +656,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
 
     // Decision points: publish either one more refinement sweep or the final mask.
     for (int r = 0;; ++r) {
+      DIAG(const long long dd0 = clock64());
       const int buf = r & 1;
       const bool need = !done && sweeps < p.max_sweeps;
       const bool final_mask = !rows_any(need, sh.votes, r, lane, kMathThreads);
@@ -688,6 +692,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
 #pragma unroll
       for (int w = 0; w < kMaskWords; ++w) list[w] = sh.lists[buf][w];
       named_bar(1, kThreads);
+      DIAG(dgx[1] += clock64() - dd0);
 
       if (final_mask) {
         clk2 = clock64();
@@ -746,8 +751,10 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           ++n_s;
         });
         const int n_out = k;
+        DIAG(const long long de0 = clock64());
         // Epilogue: O from TMEM (each thread of a row writes kOCols of the 64 columns).
         if (n_out > 0) warp_wait(&sh.pv_done[(n_out - 1) % kOBufs], ((n_out - 1) / kOBufs) & 1, wc);
+        DIAG(const long long de1 = clock64(); dgx[4] += de1 - de0);
         tc_fence_after();
         uint32_t o[kOCols];
         ldw(tl + 256 + qp * kOCols, o);
@@ -760,58 +767,70 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         }
         // The backward's delta needs Ot_i = sum_j g_ij V_j and sum_j g_ij over row i's support.
         // A row solved on its candidate copies has them all in shared memory (scores and key
-        // indices from the sweep that solved it), so each of its four threads sums g V_j
-        // over 16 of the 64 columns in fp32, gathering the fp16 V rows (just streamed by this
-        // CTA, so in L2). A row without complete copies (refinement cap, or a Newton finish)
-        // gets sum g = -1, and the backward recomputes its support.
-        if (valid) {
-          const size_t rix = (size_t)bh * p.L + i;
-          if (listed) {
-            float acc[kOCols];
+        // indices from the sweep that solved it). The gather of the bf16 V rows (exact;
+        // widened with shifts) is laid out for the memory system rather than for TMEM: eight
+        // lanes per row, each lane 8 of the 64 columns, so one load instruction reads four
+        // whole 128-byte V rows, and the warps take 64 rows per round. A row without complete
+        // copies (refinement cap, or a Newton finish) gets sum g = -1, and the backward
+        // recomputes its support.
+        DIAG(const long long de2 = clock64(); dgx[5] += de2 - de1);
+        if (qp == 0) {
+          part[3 * kTile + row] = tau;
+          part[7 * kTile + row] = (valid && listed) ? 1.f : 0.f;
+          if (valid) p.tau[(size_t)bh * p.L + i] = tau;
+        }
+        named_bar(3, kMathThreads);
+        {
+          const int sub = lane & 7;                      // columns 8 sub .. 8 sub + 7
+          const uint4* vbase = reinterpret_cast<const uint4*>(p.Vb + (size_t)bh * p.L * kD) + sub;
+          for (int rr = 0; rr < kTile; rr += 4 * kMathWarps) {
+            const int r = rr + warp * 4 + (lane >> 3);     // the row this lane serves
+            const int ir = i0 + r;
+            if (ir < p.L) {
+              const size_t rix = (size_t)bh * p.L + ir;
+              if (part[7 * kTile + r] != 0.f) {
+                const float tr = part[3 * kTile + r];
+                float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                float sgv = 0.f;
+                int pe[kParts + 1];
+                pe[0] = 0;
 #pragma unroll
-            for (int cc = 0; cc < kOCols; ++cc) acc[cc] = 0.f;
-            float sgv = 0.f;
-            const uint4* vbase = reinterpret_cast<const uint4*>(p.V16 + (size_t)bh * p.L * kD + qp * kOCols);
-            for (int q = 0; q < kParts; ++q) {
-              const int nq = (int)part[(q * 4 + 2) * kTile + row];
-              for (int k0 = 0; k0 < nq; k0 += 4) {   // four V rows in flight
-                float gk[4];
-                uint4 vw[4][kOCols / 8];
+                for (int q = 0; q < kParts; ++q) pe[q + 1] = pe[q] + (int)part[(q * 4 + 2) * kTile + r];
+                const int ntot = pe[kParts];
+                for (int k0 = 0; k0 < ntot; k0 += 4) {   // four V rows in flight
+                  float gk[4];
+                  uint4 vw[4];
 #pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                  const int e = (q * cap + min(k0 + t, nq - 1)) * kTile + row;
-                  const float u = fmaf(cand[e], cz, -tau);
-                  gk[t] = (k0 + t < nq && u > 0.f) ? ((AK == kAlpha15) ? u : 1.f) : 0.f;
-                  const uint4* vr = vbase + (size_t)cidx[e] * (kD / 8);
+                  for (int t = 0; t < 4; ++t) {
+                    const int f = min(k0 + t, ntot - 1);
+                    const int q = (f >= pe[1]) + (f >= pe[2]) + (f >= pe[3]);
+                    const int e = (q * cap + (f - pe[q])) * kTile + r;
+                    const float u = fmaf(cand[e], cz, -tr);
+                    gk[t] = (k0 + t < ntot && u > 0.f) ? ((AK == kAlpha15) ? u : 1.f) : 0.f;
+                    vw[t] = vbase[(size_t)cidx[e] * (kD / 8)];
+                  }
 #pragma unroll
-                  for (int h = 0; h < kOCols / 8; ++h) vw[t][h] = vr[h];
-                }
+                  for (int t = 0; t < 4; ++t) {
+                    sgv += gk[t];
+                    const uint32_t w4[4] = {vw[t].x, vw[t].y, vw[t].z, vw[t].w};
 #pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                  sgv += gk[t];
-#pragma unroll
-                  for (int h = 0; h < kOCols / 8; ++h) {
-                    const uint32_t w4[4] = {vw[t][h].x, vw[t][h].y, vw[t][h].z, vw[t][h].w};
-#pragma unroll
-                    for (int c2 = 0; c2 < 4; ++c2) {
-                      const float2 f = unpack_f16x2(w4[c2]);
-                      acc[8 * h + 2 * c2] = fmaf(gk[t], f.x, acc[8 * h + 2 * c2]);
-                      acc[8 * h + 2 * c2 + 1] = fmaf(gk[t], f.y, acc[8 * h + 2 * c2 + 1]);
+                    for (int c2 = 0; c2 < 4; ++c2) {   // bf16 pair -> two floats: shifts, exact
+                      acc[2 * c2] = fmaf(gk[t], __uint_as_float(w4[c2] << 16), acc[2 * c2]);
+                      acc[2 * c2 + 1] = fmaf(gk[t], __uint_as_float(w4[c2] & 0xffff0000u), acc[2 * c2 + 1]);
                     }
                   }
                 }
+                float4* dst = reinterpret_cast<float4*>(p.Ot + rix * kD + 8 * sub);
+                dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+                dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+                if (sub == 0) p.sumg[rix] = sgv;
+              } else if (sub == 0) {
+                p.sumg[rix] = -1.f;
               }
             }
-            float4* dst = reinterpret_cast<float4*>(p.Ot + rix * kD + qp * kOCols);
-#pragma unroll
-            for (int cc = 0; cc < kOCols / 4; ++cc)
-              dst[cc] = make_float4(acc[4 * cc], acc[4 * cc + 1], acc[4 * cc + 2], acc[4 * cc + 3]);
-            if (qp == 0) p.sumg[rix] = sgv;
-          } else if (qp == 0) {
-            p.sumg[rix] = -1.f;
           }
-          if (qp == 0) p.tau[rix] = tau;
         }
+        DIAG(dgx[3] += clock64() - de0);
         if (tid == 0) {
           int na = 0;
           for (int w = 0; w < kMaskWords; ++w) na += __popc(act[w]);
@@ -823,6 +842,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           DIAG(st[4] = make_int4((int)dgr[0], (int)dgr[1], (int)dgr[2], (int)dgr[3]));
           DIAG(st[5] = make_int4((int)dgr[4], (int)dgr[5], (int)dgr[6], (int)dgr[7]));
           DIAG(st[6].x = (int)dgr[8]);
+          DIAG(st[6].z = (int)dgx[0]; st[6].w = (int)dgx[1]; st[7].x = (int)dgx[2]; st[7].y = (int)dgx[3]; st[7].z = (int)dgx[4]; st[7].w = (int)dgx[5]);
         }
         break;
       }
@@ -918,6 +938,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         sbuf = (sbuf + 1) & (kSBufs - 1);
       });
       DIAG(if (cand_only) dg_sw1 = clock64() - dsw0);
+      DIAG(const long long dp0 = clock64());
       // Combine the column parts of each row.
       float* mp = part + qp * 4 * kTile + row;
       mp[0] = S1;
@@ -986,6 +1007,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           }
         }
       }
+      DIAG(dgx[2] += clock64() - dp0);
     }
   }
 

@@ -31,7 +31,7 @@ struct FwdParams {
   float* tau;               // [B*H][L]
   float* sumg;              // [B*H][L]      sum_j g_ij over the support (-1: not listed, see fwd.cu)
   float* Ot;                // [B*H][L][64]  sum_j g_ij V_j
-  const uint16_t* V16;      // [B*H][L][64]  fp16 copy of V
+  const uint16_t* Vb;       // [B*H][L][64]  V as given (bf16)
   uint32_t* M;              // [B*H][Tr][Wc]
   uint32_t* MT;             // [B*H][Tc][Wr] (zeroed before the launch)
   int* stats;               // [B*H][Tr][kFwdStats] (layout above)
