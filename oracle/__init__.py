@@ -27,6 +27,7 @@ _lib = None
 
 METHOD_SORT = 0
 METHOD_BISECT = 1
+METHOD_AUTO = 2     # the sorting solver for alpha in {1.5, 2}, bisection otherwise
 
 
 def build(force: bool = False) -> str:
@@ -111,7 +112,7 @@ def tau_bisect(z, alpha: float, iters: int = 200) -> float:
     return float(_load().orc_tau_bisect(_p(z), z.size, float(alpha), int(iters)))
 
 
-def entmax_rows(S, alpha: float, method: int = METHOD_SORT):
+def entmax_rows(S, alpha: float, method: int = METHOD_AUTO):
     """alpha-entmax of each row of raw scores S [rows, n] (-inf = inactive).
 
     Returns (P [rows, n], tau [rows]) with P = [(alpha-1) S - tau]_+^{1/(alpha-1)} (Eq. 3).
@@ -169,7 +170,7 @@ class Problem:
                                    _p(out["O"]), _p(out["tau"]), _p(out["sumg"]), _p(out["Ot"]),
                                    _p(out.get("delta")), _p(out.get("dQ")))
         if rc != 0:
-            raise ValueError("oracle attention supports alpha in {1.5, 2}")
+            raise ValueError("oracle attention needs alpha > 1")
         return out
 
     def cols(self, tau_all: np.ndarray, delta_all: np.ndarray, cols=None) -> dict:
@@ -183,7 +184,7 @@ class Problem:
         rc = _load().orc_attn_cols(*self._shape(), _p(self.Q), _p(self.K), _p(self.V), _p(self.dO),
                                    _p(tau_all), _p(delta_all), _p(cols, ctypes.c_long), n, _p(dK), _p(dV))
         if rc != 0:
-            raise ValueError("oracle attention supports alpha in {1.5, 2}")
+            raise ValueError("oracle attention needs alpha > 1")
         return {"dK": dK, "dV": dV}
 
     def forward(self) -> dict:

@@ -34,6 +34,7 @@
 
 #define ORC_METHOD_SORT 0
 #define ORC_METHOD_BISECT 1
+#define ORC_METHOD_AUTO 2   /* sort for alpha in {1.5, 2}, bisection otherwise */
 
 int orc_max_threads(void) {
 #ifdef _OPENMP
@@ -120,11 +121,15 @@ double orc_tau_bisect(const double *z, int n, double alpha, int iters) {
 }
 
 /* One row of alpha-entmax on raw scores s (entries equal to -inf are inactive).
- * Writes p (Eq. 3) and returns tau (Eq. 3 units). work holds n doubles. */
+ * Writes p (Eq. 3) and returns tau (Eq. 3 units). work holds n doubles. For alpha outside
+ * {1.5, 2} the sorting solver has no closed form per support, and ORC_METHOD_AUTO takes
+ * the bisection of Eq. 4 over the §2.4 bracket (200 halvings of a bracket of width < 1:
+ * down to fp64 resolution). */
 double orc_entmax_row(const double *s, int n, double alpha, int method, double *p, double *work) {
     int na = 0;
     for (int j = 0; j < n; ++j)
         if (s[j] != -INFINITY) work[na++] = (alpha - 1.0) * s[j];
+    if (method == ORC_METHOD_AUTO) method = (alpha == 1.5 || alpha == 2.0) ? ORC_METHOD_SORT : ORC_METHOD_BISECT;
     double tau = (method == ORC_METHOD_SORT) ? orc_tau_sort(work, na, alpha)
                                              : orc_tau_bisect(work, na, alpha, 200);
     double e = 1.0 / (alpha - 1.0);
@@ -188,7 +193,7 @@ static void attn_row(const orc_shape *sh, int b, int h, int i, const double *Q, 
     for (int j = 0; j < L; ++j)
         srow[j] = is_active(i, j, sh->causal, sh->window, kv) ? sh->scale * dotd(q, K + head + (size_t)j * d, d)
                                                                : -INFINITY;
-    double tau = orc_entmax_row(srow, L, alpha, ORC_METHOD_SORT, p, work);
+    double tau = orc_entmax_row(srow, L, alpha, ORC_METHOD_AUTO, p, work);
     double sg = 0, ge = (2.0 - alpha) / (alpha - 1.0);
     for (int j = 0; j < L; ++j) {
         double u = (srow[j] == -INFINITY) ? -1.0 : (alpha - 1.0) * srow[j] - tau;
@@ -241,7 +246,7 @@ int orc_attn_rows(int B, int H, int L, int d, double alpha, double scale, int ca
                   const double *dO, const long *rows, long nrows, double *O, double *tau,
                   double *sumg, double *Ot, double *delta, double *dQ) {
     orc_shape sh = mkshape(B, H, L, d, alpha, scale, causal, window, kv_len);
-    if (!(alpha == 1.5 || alpha == 2.0)) return 1;
+    if (!(alpha > 1.0)) return 1;
 #pragma omp parallel
     {
         double *buf = (double *)malloc(sizeof(double) * 4 * (size_t)L);
@@ -268,7 +273,7 @@ int orc_attn_cols(int B, int H, int L, int d, double alpha, double scale, int ca
                   const double *dO, const double *tau, const double *delta, const long *cols,
                   long ncols, double *dK, double *dV) {
     orc_shape sh = mkshape(B, H, L, d, alpha, scale, causal, window, kv_len);
-    if (!(alpha == 1.5 || alpha == 2.0)) return 1;
+    if (!(alpha > 1.0)) return 1;
     const double e = 1.0 / (alpha - 1.0), ge = (2.0 - alpha) / (alpha - 1.0);
 #pragma omp parallel for schedule(dynamic, 8)
     for (long c = 0; c < ncols; ++c) {

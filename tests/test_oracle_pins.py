@@ -18,6 +18,8 @@ import oracle
 
 GOLD = os.path.join(os.path.dirname(__file__), "golden", "closed_forms.json")
 ALPHAS = (1.5, 2.0)
+GENERAL = (1.25, 3.0)            # alpha outside {1.5, 2}: the oracle takes the bisection of Eq. 4
+ALL_ALPHAS = ALPHAS + GENERAL
 
 
 def _row(vals):
@@ -34,7 +36,8 @@ def test_closed_forms(case):
         want_eq3 = (alpha - 1) * eval(case["tau_score"], {}, env)
     else:
         want_eq3 = eval(case["tau_eq3"], {}, env)
-    for method in (oracle.METHOD_SORT, oracle.METHOD_BISECT):
+    methods = (oracle.METHOD_SORT, oracle.METHOD_BISECT) if alpha in ALPHAS else (oracle.METHOD_BISECT,)
+    for method in methods + (oracle.METHOD_AUTO,):
         P, tau = oracle.entmax_rows(s[None, :], alpha, method)
         tol = 1e-13 if method == oracle.METHOD_SORT else 1e-12
         assert abs(tau[0] - want_eq3) < tol, (method, tau[0], want_eq3)
@@ -63,7 +66,7 @@ def _brute_tau(z, alpha):
     return found
 
 
-@pytest.mark.parametrize("alpha", ALPHAS)
+@pytest.mark.parametrize("alpha", ALL_ALPHAS)
 @pytest.mark.parametrize("n", [1, 2, 3, 5, 8])
 def test_brute_force_supports(alpha, n):
     rng = np.random.default_rng(100 + n)
@@ -72,7 +75,11 @@ def test_brute_force_supports(alpha, n):
         z = (alpha - 1) * s
         found = _brute_tau(z, alpha)
         assert len(found) == 1, found          # exactly one consistent support (uniqueness)
-        assert abs(oracle.tau_sort(z, alpha) - found[0]) < 1e-12
+        if alpha in ALPHAS:
+            assert abs(oracle.tau_sort(z, alpha) - found[0]) < 1e-12
+        assert abs(oracle.tau_bisect(z, alpha) - found[0]) < 1e-11
+        _, tau = oracle.entmax_rows(s[None, :], alpha)   # the row solver the attention uses
+        assert abs(tau[0] - found[0]) < 1e-11
 
 
 # ------------------------------------------------------------ variational definition
@@ -82,7 +89,7 @@ def _tsallis_obj(p, s, alpha):
     return p @ s + np.sum(p - np.maximum(p, 0) ** alpha) / (alpha * (alpha - 1))
 
 
-@pytest.mark.parametrize("alpha", ALPHAS)
+@pytest.mark.parametrize("alpha", ALL_ALPHAS)
 def test_tsallis_argmax(alpha):
     """distilbert-mnli-full-adasplash card, 'Tsallis alpha-Entropy Simplex Formulation':
     entmax is the argmax over the simplex of p^T s + H_alpha(p). Checked two ways:
@@ -119,7 +126,7 @@ def test_sparsemax_is_simplex_projection():
 
 
 # ------------------------------------------------------------------------- invariants
-@pytest.mark.parametrize("alpha", ALPHAS)
+@pytest.mark.parametrize("alpha", ALL_ALPHAS)
 def test_row_invariants(alpha):
     rng = np.random.default_rng(11)
     S = rng.normal(0, 2.0, size=(64, 257))
@@ -130,8 +137,12 @@ def test_row_invariants(alpha):
     z = (alpha - 1) * S
     assert np.array_equal(P > 0, z > tau[:, None])          # p_j = 0 exactly when z_j <= tau
     # Sort-based and bisection solvers agree (§2.4: two different solvers of Eq. 4).
-    _, tau_b = oracle.entmax_rows(S, alpha, oracle.METHOD_BISECT)
-    np.testing.assert_allclose(tau, tau_b, atol=1e-12, rtol=0)
+    if alpha in ALPHAS:
+        _, tau_b = oracle.entmax_rows(S, alpha, oracle.METHOD_BISECT)
+        np.testing.assert_allclose(tau, tau_b, atol=1e-12, rtol=0)
+    else:
+        f = [oracle.f_root(z[r][np.isfinite(z[r])], alpha, tau[r]) for r in range(S.shape[0])]
+        assert np.abs(f).max() < 1e-10
     # Shift invariance: s + c gives the same p and tau shifted by (alpha-1) c.
     P2, tau2 = oracle.entmax_rows(S + 3.25, alpha)
     np.testing.assert_allclose(P2, P, atol=1e-12)
@@ -178,7 +189,7 @@ ATTN_CASES = [
 ]
 
 
-@pytest.mark.parametrize("alpha", ALPHAS)
+@pytest.mark.parametrize("alpha", ALL_ALPHAS)
 @pytest.mark.parametrize("case", ATTN_CASES, ids=lambda c: f"c{int(c['causal'])}w{c['window']}kv{c['kv']}")
 def test_attention_forward_vs_dense_composition(alpha, case):
     """The oracle's row loops against S = scale Q K^T and O = P V done with numpy matmul,
@@ -210,7 +221,7 @@ def _loss(pr, dO):
     return float(np.sum(pr.forward()["O"] * dO))
 
 
-@pytest.mark.parametrize("alpha", ALPHAS)
+@pytest.mark.parametrize("alpha", ALL_ALPHAS)
 @pytest.mark.parametrize("case", ATTN_CASES[:3], ids=["full", "causal", "window"])
 def test_backward_finite_differences(alpha, case):
     """dQ, dK, dV from the derived Jacobian against central differences of <dO, O>
@@ -218,7 +229,9 @@ def test_backward_finite_differences(alpha, case):
     on the support), so this is its pin."""
     rng = np.random.default_rng(31 + int(alpha * 10))
     B, H, L, d = 1, 1, 10, 6
-    Q, K, V, dO = (rng.normal(0, s, size=(B, H, L, d)) for s in (2.5, 1.0, 1.0, 1.0))
+    # Query spread 1.25 / (alpha - 1): z = (alpha-1) s has the same spread at every alpha,
+    # so rows keep supports of several keys (nonzero gradients) at alpha = 3 as well.
+    Q, K, V, dO = (rng.normal(0, s, size=(B, H, L, d)) for s in (1.25 / (alpha - 1), 1.0, 1.0, 1.0))
     kw = dict(alpha=alpha, scale=1 / math.sqrt(d), causal=case["causal"], window=case["window"])
     g = oracle.Problem(Q, K, V, dO, **kw).backward()
     h = 1e-6
@@ -257,7 +270,7 @@ def test_backward_sparsemax_jacobian():
         np.testing.assert_allclose(g["dQ"][0, 0, i], scale * K[0, 0].T @ (J @ dp), atol=1e-12)
 
 
-@pytest.mark.parametrize("alpha", ALPHAS)
+@pytest.mark.parametrize("alpha", ALL_ALPHAS)
 def test_backward_invariants(alpha):
     """Gradients vanish off the support (§3.3 'Backward pass'), and the score
     gradient of every row sums to zero (softmax-like shift invariance). So
@@ -281,7 +294,7 @@ def test_backward_invariants(alpha):
 
 
 # -------------------------------------------------------------------------- block mask
-@pytest.mark.parametrize("alpha", ALPHAS)
+@pytest.mark.parametrize("alpha", ALL_ALPHAS)
 def test_block_mask_brute_force(alpha):
     """Appendix C.4 packing, against a dense numpy reduction of A > 0 over tiles."""
     rng = np.random.default_rng(61)
