@@ -17,6 +17,7 @@ namespace {
 
 constexpr int kDefaultSweeps = 12;
 constexpr int kMaxSweeps = 64;
+constexpr float kMaxAlpha = 16.f;   // largest alpha accepted (u^{1/(alpha-1)} keeps fp32 sense)
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -78,9 +79,15 @@ entmax_status check_desc(const entmax_attn_desc* d) {
   if (d->selftest != 0 && d->selftest != ENTMAX_SELFTEST_STALL) return ENTMAX_EINVAL;
   if (d->d != kD) return ENTMAX_EUNSUPPORTED;
   if (d->L > ENTMAX_MAX_L) return ENTMAX_EUNSUPPORTED;
-  if (d->alpha != 1.5f && d->alpha != 2.0f) return ENTMAX_EUNSUPPORTED;
+  if (!(d->alpha > 1.0f) || !std::isfinite(d->alpha)) return ENTMAX_EINVAL;
+  if (d->alpha > kMaxAlpha) return ENTMAX_EUNSUPPORTED;
+  // fp32 inputs: the CUDA-core forward has closed-form powers for alpha in {1.5, 2} only.
+  if (d->dtype == ENTMAX_FP32 && d->alpha != 1.5f && d->alpha != 2.0f) return ENTMAX_EUNSUPPORTED;
   return ENTMAX_OK;
 }
+
+// The kernels' alpha variant: closed-form powers for 1.5 and 2, the run-time one otherwise.
+int alpha_kind(float alpha) { return alpha == 1.5f ? kAlpha15 : (alpha == 2.0f ? kAlpha2 : kAlphaGen); }
 
 bool aligned(const void* p, size_t a) { return p && (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -212,9 +219,11 @@ extern "C" entmax_status entmax_attn_fwd(const entmax_attn_desc* d, const void* 
   p.causal = d->causal || d->window >= 0;
   p.window = d->window < 0 ? -1 : d->window;
   p.max_sweeps = d->max_sweeps == 0 ? kDefaultSweeps : d->max_sweeps;
+  p.ae = 1.0f / (d->alpha - 1.0f);
+  p.am1 = d->alpha - 1.0f;
   p.wait_limit_ns = wait_limit_ns(d);
   p.selftest = d->selftest;
-  return launch_fwd(d->alpha == 1.5f, p, l.BH * l.Tr, s) == cudaSuccess ? ENTMAX_OK : ENTMAX_ECUDA;
+  return launch_fwd(alpha_kind(d->alpha), p, l.BH * l.Tr, s) == cudaSuccess ? ENTMAX_OK : ENTMAX_ECUDA;
 }
 
 extern "C" entmax_status entmax_attn_bwd(const entmax_attn_desc* d, const void* Q, const void* K, const void* V,
@@ -256,6 +265,7 @@ extern "C" entmax_status entmax_attn_bwd(const entmax_attn_desc* d, const void* 
   p.BH = l.BH;
   p.cz = (d->alpha - 1.0f) * d->scale;
   p.scale = d->scale;
+  p.ae = 1.0f / (d->alpha - 1.0f);
   p.causal = d->causal || d->window >= 0;
   p.window = d->window < 0 ? -1 : d->window;
   p.wait_limit_ns = wait_limit_ns(d);
@@ -280,13 +290,14 @@ extern "C" entmax_status entmax_attn_bwd(const entmax_attn_desc* d, const void* 
   dp.Wc = l.Wc;
   dp.BH = l.BH;
   dp.cz = (d->alpha - 1.0f) * d->scale;
+  dp.ae = 1.0f / (d->alpha - 1.0f);
   dp.causal = d->causal || d->window >= 0;
   dp.window = d->window < 0 ? -1 : d->window;
-  if (launch_delta(d->alpha == 1.5f, dp, s) != cudaSuccess) return ENTMAX_ECUDA;
+  if (launch_delta(alpha_kind(d->alpha), dp, s) != cudaSuccess) return ENTMAX_ECUDA;
   if (cudaMemsetAsync(dQ, 0, (size_t)rows * kD * 4, s) != cudaSuccess) return ENTMAX_ECUDA;
   if (launch_bf16_to_f16(dO, do16, rows * kD, reinterpret_cast<int*>(w + l.off_status), s) != cudaSuccess)
     return ENTMAX_ECUDA;
-  return launch_bwd(d->alpha == 1.5f, p, l.BH * l.Tc, s) == cudaSuccess ? ENTMAX_OK : ENTMAX_ECUDA;
+  return launch_bwd(alpha_kind(d->alpha), p, l.BH * l.Tc, s) == cudaSuccess ? ENTMAX_OK : ENTMAX_ECUDA;
 }
 
 extern "C" entmax_status entmax_rows(const float* S, int rows, int n, int ld, float alpha, float* P, float* tau,

@@ -297,14 +297,22 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
           const float2 u = __ffma2_rn(make_float2(s0, s1), make_float2(cz, cz), make_float2(-tau, -tau));
           const float v0 = fmaxf(u.x, 0.f), v1 = fmaxf(u.y, 0.f);
           const float d0 = __uint_as_float(ar[c]) - dl, d1 = __uint_as_float(ar[c + 1]) - dl;
-          if (AK == kAlpha15) {
+          if constexpr (AK == kAlpha15) {
             const float2 a = __fmul2_rn(make_float2(v0, v1), make_float2(v0, v1));
             const float2 ds = __fmul2_rn(make_float2(v0, v1), make_float2(d0, d1));
             ah[e] = pack_f16(a.x, a.y);
             split_bf16x2(ds.x, ds.y, dh[e], dl2[e]);
-          } else {
+          } else if constexpr (AK == kAlpha2) {
             ah[e] = pack_f16(v0, v1);
             split_bf16x2(u.x > 0.f ? d0 : 0.f, u.y > 0.f ? d1 : 0.f, dh[e], dl2[e]);
+          } else {
+            // A = u^e and g = u^{e-1} from one logarithm each.
+            const float l0 = __log2f(u.x > 0.f ? u.x : 1.f), l1 = __log2f(u.y > 0.f ? u.y : 1.f);
+            const float a0 = u.x > 0.f ? exp2f(p.ae * l0) : 0.f, a1 = u.y > 0.f ? exp2f(p.ae * l1) : 0.f;
+            const float g0 = u.x > 0.f ? exp2f((p.ae - 1.f) * l0) : 0.f;
+            const float g1 = u.y > 0.f ? exp2f((p.ae - 1.f) * l1) : 0.f;
+            ah[e] = pack_f16(a0, a1);
+            split_bf16x2(g0 * d0, g1 * d1, dh[e], dl2[e]);
           }
         }
         const uint32_t off = pan + sw128_offset(row, ((qc & 1) * 4 + cc) * 8);
@@ -381,9 +389,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
   if (warp == kMmaWarp) tmem_dealloc(T, 512);
 }
 
-cudaError_t launch_bwd(bool alpha15, const BwdParams& p, int grid, cudaStream_t s) {
+cudaError_t launch_bwd(int alpha_kind, const BwdParams& p, int grid, cudaStream_t s) {
   const int smem = bwd_smem_bytes();
-  auto kern = alpha15 ? bwd_kernel<kAlpha15> : bwd_kernel<kAlpha2>;
+  auto kern = alpha_kind == kAlpha15 ? bwd_kernel<kAlpha15>
+             : alpha_kind == kAlpha2 ? bwd_kernel<kAlpha2>
+                                     : bwd_kernel<kAlphaGen>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   kern<<<grid, kThreads, smem, s>>>(p);
@@ -495,7 +505,7 @@ __global__ void __launch_bounds__(32 * kDeltaWarps, 4) bwd_delta_kernel(const __
           if (jk < p.L && pat.active(i, jk)) {
             const float uu = fmaf(dot_s(Ko + (size_t)jk * 8, xs[warp][0], false), p.cz, -to);
             if (uu > 0.f) {
-              const float g = (AK == kAlpha15) ? uu : 1.f;
+              const float g = (AK == kAlpha15) ? uu : (AK == kAlpha2 ? 1.f : pow_pos(uu, p.ae - 1.f));
               og += g;
               ogd = fmaf(g, dot_s(Vo + (size_t)jk * 8, xs[warp][1], true), ogd);
             }
@@ -513,14 +523,16 @@ __global__ void __launch_bounds__(32 * kDeltaWarps, 4) bwd_delta_kernel(const __
   if (valid) p.delta[r] = delta;
 }
 
-cudaError_t launch_delta(bool alpha15, const DeltaParams& p, cudaStream_t s) {
+cudaError_t launch_delta(int alpha_kind, const DeltaParams& p, cudaStream_t s) {
   const long rows = (long)p.BH * p.L;
   const long per_block = (long)kDeltaWarps * 32;
   const unsigned grid = (unsigned)((rows + per_block - 1) / per_block);
-  if (alpha15)
+  if (alpha_kind == kAlpha15)
     bwd_delta_kernel<kAlpha15><<<grid, 32 * kDeltaWarps, 0, s>>>(p);
-  else
+  else if (alpha_kind == kAlpha2)
     bwd_delta_kernel<kAlpha2><<<grid, 32 * kDeltaWarps, 0, s>>>(p);
+  else
+    bwd_delta_kernel<kAlphaGen><<<grid, 32 * kDeltaWarps, 0, s>>>(p);
   return cudaGetLastError();
 }
 

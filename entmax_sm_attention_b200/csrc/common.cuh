@@ -12,9 +12,15 @@ constexpr int kTileBytes = kTile * kD * 2;   // one bf16 [128][64] tile = 16 KB
 constexpr int kMaxTc = 128;     // longest sequence = 128 key tiles = 16384 tokens
 constexpr int kMaskWords = kMaxTc / 32;
 
-// Alpha variants with closed-form powers: A = u^{1/(alpha-1)}, g = u^{(2-alpha)/(alpha-1)}.
+// Alpha variants: A = u^{1/(alpha-1)}, g = u^{(2-alpha)/(alpha-1)} for u = z - tau > 0.
 //   kAlpha15: A = u^2, g = u          kAlpha2: A = u, g = [u > 0]
-enum AlphaKind { kAlpha15 = 0, kAlpha2 = 1 };
+//   kAlphaGen: any alpha > 1 at run time, with e = 1/(alpha-1): A = u^e, g = u^{e-1},
+//     through exp2(e log2 u) (the hardware's approximate base-2 exponential and
+//     logarithm: relative error near 2^-22 each).
+enum AlphaKind { kAlpha15 = 0, kAlpha2 = 1, kAlphaGen = 2 };
+
+// u^x for u > 0 (exp2 of x log2 u); callers pass only positive u.
+__device__ __forceinline__ float pow_pos(float u, float x) { return exp2f(x * __log2f(u)); }
 
 // Structural attention pattern of one (batch, head).
 struct Pattern {

@@ -179,15 +179,6 @@ __host__ __device__ constexpr int fwd_region_bytes(int Tc) {
   return Tc * kTile * 4 + 4 * fwd_cand_cap(Tc) * kTile * (4 + 2);
 }
 
-// fp16 pair -> two floats (exact).
-__device__ __forceinline__ float2 unpack_f16x2(uint32_t w) {
-  float lo, hi;
-  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, h;\n\t}"
-      : "=f"(lo), "=f"(hi)
-      : "r"(w));
-  return make_float2(lo, hi);
-}
-
 // Appends the scores of an 8-key group that pass tau (u = s cz - tau > 0) to this thread's
 // candidate copies, without branches: every element is written to slot min(nc, cap-1) and
 // nc advances only on a pass. A failing element lands in the next free slot, which the next
@@ -205,28 +196,69 @@ __device__ __forceinline__ void collect8(const float* s, int j, float cz, float 
 }
 
 // Adds one candidate at u = z - t to the sums of the current support (u > 0), without
-// a branch: the lanes of a warp follow one path whatever their candidates.
-__device__ __forceinline__ void accumulate(float u, float& S1, float& S2, float& C, float& umin) {
+// a branch: the lanes of a warp follow one path whatever their candidates. S1 and S2 are
+// sum u and sum u^2 (alpha = 1.5, 2); for the run-time variant they are sum g = sum u^{e-1}
+// and sum p = sum u^e. In every case f = sum p - 1 and |f'| = e sum g (see root_terms).
+template <int AK>
+__device__ __forceinline__ void accumulate(float u, float e, float& S1, float& S2, float& C, float& umin) {
   const bool in = u > 0.f;
-  const float v = in ? u : 0.f;
-  S1 += v;
-  S2 = fmaf(v, v, S2);
+  if constexpr (AK == kAlphaGen) {
+    const float l = __log2f(in ? u : 1.f);
+    S1 += in ? exp2f((e - 1.f) * l) : 0.f;
+    S2 += in ? exp2f(e * l) : 0.f;
+  } else {
+    const float v = in ? u : 0.f;
+    S1 += v;
+    S2 = fmaf(v, v, S2);
+  }
   C += in ? 1.f : 0.f;
   umin = fminf(umin, in ? u : INFINITY);
 }
 
+// f(t) = sum_j p_j - 1 (Eq. 4) and |f'(t)| = e sum_j g_j from the sums of accumulate.
+template <int AK>
+__device__ __forceinline__ void root_terms(float S1, float S2, float C, float e, float& f, float& fp) {
+  if constexpr (AK == kAlpha15) {
+    f = S2 - 1.f;
+    fp = 2.f * S1;
+  } else if constexpr (AK == kAlpha2) {
+    f = S1 - 1.f;
+    fp = C;
+  } else {
+    f = S2 - 1.f;
+    fp = e * S1;
+  }
+}
+
+// Exact root of Eq. 4 restricted to the current support (alpha = 1.5: the smaller root of
+// C d^2 - 2 S1 d + S2 - 1 = 0; alpha = 2: (S1-1)/C), as the step d from t; -1 when there is
+// no closed form (run-time alpha) or no real root.
+template <int AK>
+__device__ __forceinline__ float piece_root(float S1, float S2, float C) {
+  if constexpr (AK == kAlpha15) {
+    const float disc = S1 * S1 - C * (S2 - 1.f);
+    return disc >= 0.f ? (S2 - 1.f) / (S1 + sqrtf(disc)) : -1.f;   // = (S1 - sqrt(disc)) / C
+  } else if constexpr (AK == kAlpha2) {
+    return (S1 - 1.f) / C;
+  } else {
+    return -1.f;
+  }
+}
+
 // Support sums of list[k*stride], k < n, at t: four independent partial sums, so the
 // adds do not form one serial chain.
-__device__ __forceinline__ void sum_list(const float* list, int n, int stride, float cz, float t, float& S1,
+template <int AK>
+__device__ __forceinline__ void sum_list(const float* list, int n, int stride, float cz, float t, float e, float& S1,
                                          float& S2, float& C, float& umin) {
   float a1[4] = {0.f, 0.f, 0.f, 0.f}, a2[4] = {0.f, 0.f, 0.f, 0.f}, ac[4] = {0.f, 0.f, 0.f, 0.f};
   float am[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
   int k = 0;
   for (; k + 4 <= n; k += 4) {
 #pragma unroll
-    for (int q = 0; q < 4; ++q) accumulate(fmaf(list[(k + q) * stride], cz, -t), a1[q], a2[q], ac[q], am[q]);
+    for (int q = 0; q < 4; ++q)
+      accumulate<AK>(fmaf(list[(k + q) * stride], cz, -t), e, a1[q], a2[q], ac[q], am[q]);
   }
-  for (; k < n; ++k) accumulate(fmaf(list[k * stride], cz, -t), a1[0], a2[0], ac[0], am[0]);
+  for (; k < n; ++k) accumulate<AK>(fmaf(list[k * stride], cz, -t), e, a1[0], a2[0], ac[0], am[0]);
   S1 += (a1[0] + a1[1]) + (a1[2] + a1[3]);
   S2 += (a2[0] + a2[1]) + (a2[2] + a2[3]);
   C += (ac[0] + ac[1]) + (ac[2] + ac[3]);
@@ -239,33 +271,41 @@ __device__ __forceinline__ void sum_list(const float* list, int n, int stride, f
 // true with the exact root up to fp32 rounding.
 template <int AK>
 __device__ bool solve_list(const float* vals, const int (&n)[kParts], int list_stride, int stride, float cz,
-                           float t, float lo, float hi, float& t_out) {
-  for (int it = 0; it < 48; ++it) {
+                           float e, float t, float lo, float hi, float& t_out) {
+  // The run-time alpha variant has no closed form; for alpha > 2, f is concave with an
+  // unbounded slope where a candidate enters the support, so Newton can crawl: every
+  // fourth step bisects, which halves the bracket at least that often.
+  constexpr int kIters = AK == kAlphaGen ? 96 : 48;
+  for (int it = 0; it < kIters; ++it) {
     float S1 = 0.f, S2 = 0.f, C = 0.f, umin = INFINITY;
 #pragma unroll
-    for (int q = 0; q < kParts; ++q) sum_list(vals + q * list_stride, n[q], stride, cz, t, S1, S2, C, umin);
-    const float f = (AK == kAlpha15) ? S2 - 1.f : S1 - 1.f;
-    const float fp = (AK == kAlpha15) ? 2.f * S1 : C;   // |f'(t)|
+    for (int q = 0; q < kParts; ++q) sum_list<AK>(vals + q * list_stride, n[q], stride, cz, t, e, S1, S2, C, umin);
+    float f, fp;   // f(t) and |f'(t)|
+    root_terms<AK>(S1, S2, C, e, f, fp);
     if (C > 0.f) {
-      float d = -1.f;
-      if (AK == kAlpha15) {
-        const float disc = S1 * S1 - C * (S2 - 1.f);
-        if (disc >= 0.f) d = (S2 - 1.f) / (S1 + sqrtf(disc));   // = (S1 - sqrt(disc)) / C
-      } else {
-        d = (S1 - 1.f) / C;
-      }
+      const float d = piece_root<AK>(S1, S2, C);
       if (d >= 0.f && d < umin) {   // no candidate leaves the support at t + d: exact
         t_out = t + d;
         return true;
       }
     }
-    if (fabsf(f) <= 1e-7f && fp > 0.f) {
+    // Without a closed form, Newton stops once f is at the rounding level of its sum (the
+    // powers come from approximate exp2 / log2, relative error near 2^-21 per term).
+    const float tol = AK == kAlphaGen ? fmaxf(4e-6f, C * 0x1p-19f) : 1e-7f;
+    if (fabsf(f) <= tol && fp > 0.f) {
       t_out = t + f / fp;
       return true;
     }
     if (f > 0.f) lo = t; else hi = t;
+    // Where f is nearly vertical (alpha > 2, a key just inside the support) |f| may never
+    // reach its tolerance: the bracket reaching fp32 resolution ends the solve instead.
+    if (AK == kAlphaGen && hi - lo <= fmaxf(fabsf(lo), 1.f) * 0x1p-22f) {
+      t_out = 0.5f * (lo + hi);
+      return true;
+    }
     float tn = t + f / fp;
     if (!(tn > lo && tn <= hi && tn != t)) tn = 0.5f * (lo + hi);   // the root may sit at hi; a stalled step bisects
+    if (AK == kAlphaGen && (it & 3) == 3) tn = 0.5f * (lo + hi);
     t = tn;
   }
   t_out = t;
@@ -277,25 +317,19 @@ __device__ bool solve_list(const float* vals, const int (&n)[kParts], int list_s
 // support's piece once no value leaves the support. A subset of the row's scores has a
 // threshold at or below the row's tau*, so the result is a lower bound on tau*.
 template <int AK, int N>
-__device__ __forceinline__ float solveN(const float (&v)[N], float cz, float lo, float hi) {
+__device__ __forceinline__ float solveN(const float (&v)[N], float cz, float e, float lo, float hi) {
   float t = lo;
   for (int it = 0; it < 24; ++it) {
     float S1 = 0.f, S2 = 0.f, C = 0.f, umin = INFINITY;
 #pragma unroll
-    for (int q = 0; q < N; ++q) accumulate(fmaf(v[q], cz, -t), S1, S2, C, umin);
-    const float f = (AK == kAlpha15) ? S2 - 1.f : S1 - 1.f;
-    const float fp = (AK == kAlpha15) ? 2.f * S1 : C;
+    for (int q = 0; q < N; ++q) accumulate<AK>(fmaf(v[q], cz, -t), e, S1, S2, C, umin);
+    float f, fp;
+    root_terms<AK>(S1, S2, C, e, f, fp);
     if (C > 0.f) {
-      float d = -1.f;
-      if (AK == kAlpha15) {
-        const float disc = S1 * S1 - C * (S2 - 1.f);
-        if (disc >= 0.f) d = (S2 - 1.f) / (S1 + sqrtf(disc));
-      } else {
-        d = (S1 - 1.f) / C;
-      }
+      const float d = piece_root<AK>(S1, S2, C);
       if (d >= 0.f && d < umin) return t + d;
     }
-    if (fabsf(f) <= 1e-7f && fp > 0.f) return t + f / fp;
+    if (fabsf(f) <= (AK == kAlphaGen ? 1e-6f : 1e-7f) && fp > 0.f) return t + f / fp;
     if (f > 0.f) lo = t; else hi = t;
     float tn = t + f / fp;
     if (!(tn > lo && tn <= hi && tn != t)) tn = 0.5f * (lo + hi);
@@ -636,7 +670,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     const int n_act = valid ? pat.count(i) : 1;
     const float mz = m * cz;
     float lo = mz - 1.f;
-    float hi = mz - ((AK == kAlpha15) ? rsqrtf((float)n_act) : 1.f / (float)n_act);
+    float hi = mz - ((AK == kAlpha15)  ? rsqrtf((float)n_act)
+                     : (AK == kAlpha2) ? 1.f / (float)n_act
+                                       : pow_pos((float)n_act, -p.am1));   // n^{1-alpha}
     float tau = INFINITY;
     bool done = !valid;
     bool listed = false;   // solved on candidate copies that hold the whole support
@@ -646,7 +682,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       // The row's largest part-tile maxima are a subset of its scores, so the threshold
       // of entmax on them is a lower bound tau_T <= tau*.
       DIAG(const long long ds0 = clock64());
-      const float t = solveN<AK, 4 * kParts>(vt, cz, lo, hi);
+      const float t = solveN<AK, 4 * kParts>(vt, cz, p.ae, lo, hi);
       tau = fminf(fmaxf(t, lo), hi);
       DIAG(dgx[0] += clock64() - ds0);
     }
@@ -729,11 +765,13 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
             const float2 u = __ffma2_rn(make_float2(s[2 * cc], s[2 * cc + 1]), make_float2(cz, cz),
                                         make_float2(-tau, -tau));
             const float v0 = fmaxf(u.x, 0.f), v1 = fmaxf(u.y, 0.f);
-            if (AK == kAlpha15) {
+            if constexpr (AK == kAlpha15) {
               const float2 a = __fmul2_rn(make_float2(v0, v1), make_float2(v0, v1));
               aw[cc] = pack_f16(a.x, a.y);
-            } else {
+            } else if constexpr (AK == kAlpha2) {
               aw[cc] = pack_f16(v0, v1);
+            } else {
+              aw[cc] = pack_f16(v0 > 0.f ? pow_pos(v0, p.ae) : 0.f, v1 > 0.f ? pow_pos(v1, p.ae) : 0.f);
             }
           }
           // This part's keys qp*kCols.. go back into its own S columns [qp*kCols, +kCols/2):
@@ -806,7 +844,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
                     const int q = (f >= pe[1]) + (f >= pe[2]) + (f >= pe[3]);
                     const int e = (q * cap + (f - pe[q])) * kTile + r;
                     const float u = fmaf(cand[e], cz, -tr);
-                    gk[t] = (k0 + t < ntot && u > 0.f) ? ((AK == kAlpha15) ? u : 1.f) : 0.f;
+                    const float gu = AK == kAlpha15 ? u : (AK == kAlpha2 ? 1.f : pow_pos(fmaxf(u, 1e-30f), p.ae - 1.f));
+                    gk[t] = (k0 + t < ntot && u > 0.f) ? gu : 0.f;
                     vw[t] = vbase[(size_t)cidx[e] * (kD / 8)];
                   }
 #pragma unroll
@@ -910,7 +949,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         }
         // Groups of 8 scores: u+ summed per group (feeds S1), straight-line for all groups;
         // then only the groups with a positive sum (rare: a support candidate) are scanned
-        // element by element.
+        // element by element. The run-time alpha variant sums g = u^{e-1} into S1 and
+        // p = u^e into S2 instead.
         uint32_t gmask = 0;
 #pragma unroll
         for (int g = 0; g < kCols / 8; ++g) {
@@ -920,10 +960,16 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
             const float2 u = __ffma2_rn(make_float2(s[8 * g + 2 * e], s[8 * g + 2 * e + 1]), make_float2(cz, cz),
                                         make_float2(-tau, -tau));
             v[e] = make_float2(fmaxf(u.x, 0.f), fmaxf(u.y, 0.f));
-            s2[e] = __ffma2_rn(v[e], v[e], s2[e]);
+            if constexpr (AK == kAlphaGen) {
+              float dummy_c = 0.f, dummy_m = INFINITY;
+              accumulate<AK>(u.x, p.ae, s1[e].x, s2[e].x, dummy_c, dummy_m);
+              accumulate<AK>(u.y, p.ae, s1[e].y, s2[e].y, dummy_c, dummy_m);
+            } else {
+              s2[e] = __ffma2_rn(v[e], v[e], s2[e]);
+            }
           }
           const float2 gs = __fadd2_rn(__fadd2_rn(v[0], v[1]), __fadd2_rn(v[2], v[3]));
-          s1[g & 3] = __fadd2_rn(s1[g & 3], gs);
+          if constexpr (AK != kAlphaGen) s1[g & 3] = __fadd2_rn(s1[g & 3], gs);
           gmask |= (gs.x + gs.y > 0.f ? 1u : 0u) << g;
         }
 #pragma unroll
@@ -966,29 +1012,35 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         // tau = tau_T <= tau*: if the copies fit they hold the support; solve on them.
         // Otherwise tau stays and the next sweep measures f(tau) and f'(tau).
         float t;
-        if (fits && solve_list<AK>(cand + row, ncs, cap * kTile, kTile, cz, tau, lo, hi, t)) {
+        if (fits && solve_list<AK>(cand + row, ncs, cap * kTile, kTile, cz, p.ae, tau, lo, hi, t)) {
           tau = t;
           done = true;
           listed = true;
         }
       } else if (!done) {
-        const float f = (AK == kAlpha15) ? S2 - 1.f : S1 - 1.f;
-        const float fp = (AK == kAlpha15) ? 2.f * S1 : C;   // |f'(tau)|
+        float f, fp;   // f(tau) and |f'(tau)|
+        root_terms<AK>(S1, S2, C, p.ae, f, fp);
         if (f > 0.f) lo = fmaxf(lo, tau); else hi = fminf(hi, tau);
         if (f >= 0.f && fits) {
           // tau <= tau*, so every score of the support is in the candidate lists: the
           // exact solve on chip ends the refinement.
           float t;
-          if (solve_list<AK>(cand + row, ncs, cap * kTile, kTile, cz, tau, lo, hi, t)) {
+          if (solve_list<AK>(cand + row, ncs, cap * kTile, kTile, cz, p.ae, tau, lo, hi, t)) {
             tau = t;
             done = true;
             listed = true;
           }
         }
         if (!done) {
-          // f is a sum of C positive terms in fp32; its rounding error grows with C.
-          const float tolf = fmaxf(kTolF, C * 0x1p-22f);
-          if (fabsf(f) <= tolf && fp > 0.f && (fits || near_once)) {
+          // f is a sum of C positive terms in fp32; its rounding error grows with C (and,
+          // for the run-time alpha variant, with the approximate powers).
+          const float tolf = AK == kAlphaGen ? fmaxf(4.f * kTolF, C * 0x1p-19f) : fmaxf(kTolF, C * 0x1p-22f);
+          const bool narrow = AK == kAlphaGen && hi - lo <= fmaxf(fabsf(lo), 1.f) * 0x1p-22f;
+          if (narrow) {   // bracket at fp32 resolution (see solve_list)
+            tau = 0.5f * (lo + hi);
+            done = true;
+            listed = fits && f >= 0.f;
+          } else if (fabsf(f) <= tolf && fp > 0.f && (fits || near_once)) {
             // Final Newton correction, no further sweep needed. The copies of this sweep
             // hold the support when they fit (tau moves by at most the tolerance over the
             // slope). When they do not, the row first sweeps once more at the corrected
@@ -1025,9 +1077,11 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
 
 int fwd_smem_bytes(int Tc) { return 1024 + fwd_off_region() + fwd_region_bytes(Tc) + kParts * 4 * kTile * 4; }
 
-cudaError_t launch_fwd(bool alpha15, const FwdParams& p, int grid, cudaStream_t s) {
+cudaError_t launch_fwd(int alpha_kind, const FwdParams& p, int grid, cudaStream_t s) {
   const int smem = fwd_smem_bytes(p.Tc);
-  auto kern = alpha15 ? fwd_kernel<kAlpha15> : fwd_kernel<kAlpha2>;
+  auto kern = alpha_kind == kAlpha15 ? fwd_kernel<kAlpha15>
+             : alpha_kind == kAlpha2 ? fwd_kernel<kAlpha2>
+                                     : fwd_kernel<kAlphaGen>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   kern<<<grid, kThreads, smem, s>>>(p);

@@ -39,6 +39,7 @@ struct FwdParams {
   const int* kv_len;        // [B] or nullptr
   int H, L, Tr, Tc, Wc, Wr, BH;
   float cz;                 // (alpha - 1) * scale
+  float ae, am1;            // 1 / (alpha - 1) and alpha - 1 (the run-time alpha variant)
   int causal, window, max_sweeps;
   unsigned long long wait_limit_ns;   // bound on every in-kernel wait
   int selftest;             // kSelftestStall: one wait per CTA on a barrier nothing completes
@@ -59,6 +60,7 @@ struct BwdParams {
   int H, L, Tr, Tc, Wr, BH;
   float cz;                      // (alpha - 1) * scale
   float scale;
+  float ae;                      // 1 / (alpha - 1)
   int causal, window;
   unsigned long long wait_limit_ns;
   int selftest;
@@ -79,6 +81,7 @@ struct DeltaParams {
   const int* kv_len;
   int H, L, Tr, Wc, BH;
   float cz;
+  float ae;                     // 1 / (alpha - 1)
   int causal, window;
 };
 
@@ -102,11 +105,11 @@ struct FwdF32Params {
 // dynamic shared-memory limit and launch on `s`; they return the launch error.
 int fwd_smem_bytes(int Tc);
 int bwd_smem_bytes();
-cudaError_t launch_fwd(bool alpha15, const FwdParams& p, int grid, cudaStream_t s);
+cudaError_t launch_fwd(int alpha_kind, const FwdParams& p, int grid, cudaStream_t s);
 cudaError_t launch_fwd_f32(bool alpha15, const FwdF32Params& p, int grid, cudaStream_t s);
-cudaError_t launch_bwd(bool alpha15, const BwdParams& p, int grid, cudaStream_t s);
+cudaError_t launch_bwd(int alpha_kind, const BwdParams& p, int grid, cudaStream_t s);
 cudaError_t launch_bf16_to_f16(const void* src, void* dst, long elems, int* status, cudaStream_t s);
-cudaError_t launch_delta(bool alpha15, const DeltaParams& p, cudaStream_t s);
+cudaError_t launch_delta(int alpha_kind, const DeltaParams& p, cudaStream_t s);
 cudaError_t launch_rows(bool alpha15, const float* S, int rows, int n, long ld, float* P, float* tau, int* status,
                         cudaStream_t s);
 

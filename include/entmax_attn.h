@@ -21,7 +21,8 @@
  * g = p^{2-alpha}. The pages state only that gradients live on the support (§3.3); this
  * formula comes from implicit differentiation of sum_j p_j = 1. Hence
  *   dS_ij = g_ij (dO_i . V_j - delta_i),   delta_i = dO_i . Ot_i / sum_j g_ij,
- *   Ot_i  = sum_j g_ij V_j                (written by the forward into the workspace),
+ *   Ot_i  = sum_j g_ij V_j                (summed by the forward in fp32 over the support
+ *                                          of each row, and kept in the workspace),
  *   dQ = scale dS K,  dK = scale dS^T Q,  dV = P^T dO.
  *
  * Conventions for every entry point:
@@ -75,7 +76,14 @@ typedef enum { ENTMAX_BF16 = 0, ENTMAX_FP32 = 1 } entmax_dtype;
 typedef struct {
     int B, H, L, d;       /* batch, heads, sequence length, head dim. d must be 64;
                              1 <= L <= ENTMAX_MAX_L.                                     */
-    float alpha;          /* 1.5 or 2.0; any other value -> ENTMAX_EUNSUPPORTED           */
+    float alpha;          /* 1 < alpha <= 16 (alpha <= 1 or NaN -> ENTMAX_EINVAL, above 16
+                             -> ENTMAX_EUNSUPPORTED). 1.5 and 2 use closed-form powers and
+                             an exact on-chip solve; other alpha take u^{1/(alpha-1)} through
+                             exp2/log2 and a safeguarded Newton solve (§3.2). With fp32 inputs
+                             only 1.5 and 2 are supported. For alpha > 2 the backward's
+                             g = p^{2-alpha} is unbounded as p -> 0 (a property of the
+                             Jacobian), so gradients of keys at the support's edge are
+                             ill-conditioned.                                             */
     float scale;          /* score scale, usually 1/sqrt(d); must be > 0                 */
     int causal;           /* 0: every key j < kv_len is active; 1: only keys j <= i      */
     int window;           /* < 0: no window. >= 0: active = {0} U [max(1, i-window), i];

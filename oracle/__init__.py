@@ -56,7 +56,7 @@ def _load():
         lib.orc_tau_bisect.restype = d_
         lib.orc_entmax_rows.argtypes = [dp, ctypes.c_long, i, ctypes.c_long, d_, i, dp, dp]
         lib.orc_entmax_rows.restype = None
-        shape = [i, i, i, i, d_, d_, i, i, ip]
+        shape = [i, i, i, i, d_, d_, i, i, ip, dp]   # ..., kv_len, alibi slopes
         lib.orc_attn_rows.argtypes = shape + [dp, dp, dp, dp, lp, ctypes.c_long, dp, dp, dp, dp, dp, dp]
         lib.orc_attn_rows.restype = i
         lib.orc_attn_cols.argtypes = shape + [dp, dp, dp, dp, dp, dp, lp, ctypes.c_long, dp, dp]
@@ -130,7 +130,7 @@ class Problem:
     """One attention problem held in float64: Q, K, V, dO [B, H, L, d] and its options."""
 
     def __init__(self, Q, K, V, dO=None, *, alpha: float, scale: float, causal: bool = False,
-                 window: int = -1, kv_len=None):
+                 window: int = -1, kv_len=None, alibi=None):
         self.Q, self.K, self.V = _f64(Q), _f64(K), _f64(V)
         self.dO = _f64(dO) if dO is not None else None
         self.B, self.H, self.L, self.d = self.Q.shape
@@ -140,10 +140,13 @@ class Problem:
             self.kv_len = None
         else:
             self.kv_len = np.ascontiguousarray(np.asarray(kv_len, dtype=np.int32).reshape(self.B))
+        # ALiBi slopes m_h per head (score units per position), or None.
+        self.alibi = None if alibi is None else np.ascontiguousarray(np.asarray(alibi, dtype=np.float64).reshape(self.H))
 
     def _shape(self):
         kv = self.kv_len.ctypes.data_as(ctypes.POINTER(ctypes.c_int)) if self.kv_len is not None else None
-        return [self.B, self.H, self.L, self.d, self.alpha, self.scale, self.causal, self.window, kv]
+        ab = self.alibi.ctypes.data_as(ctypes.POINTER(ctypes.c_double)) if self.alibi is not None else None
+        return [self.B, self.H, self.L, self.d, self.alpha, self.scale, self.causal, self.window, kv, ab]
 
     def all_rows(self) -> np.ndarray:
         return np.arange(self.B * self.H * self.L, dtype=np.int64)

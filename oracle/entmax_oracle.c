@@ -19,6 +19,9 @@
  *   - same page, Appendix C.4: bit-packed block mask, 32 column blocks per uint32.
  *   - "Hooshaai/gpt2-adasplash-attention" model card, "Causal Splash Masking with
  *     Sink Preservation": active set {0} U {j <= i : i - j <= W}.
+ *   - "AdaSplash-2", §4.3: NAPE gives half of the heads no positional encoding and half
+ *     ALiBi (Press et al.), a per-head linear penalty on the scores by query-key distance:
+ *     s_ij = scale q_i . k_j - m_h |i - j| (m_h = 0 for a head without it).
  *
  * Everything is fp64 with no intermediate rounding; inputs are widened exactly
  * from whatever the caller drew (bf16 or fp32). Rows are parallelised with
@@ -153,6 +156,12 @@ void orc_entmax_rows(const double *S, long rows, int n, long ld, double alpha, i
     }
 }
 
+static double dotd(const double *a, const double *b, int d) {
+    double acc = 0;
+    for (int k = 0; k < d; ++k) acc += a[k] * b[k];
+    return acc;
+}
+
 /* ---------------------------------------------------------------------------------
  * Attention. Tensors are contiguous [B, H, L, d] fp64; kv_len is int[B] (or NULL = L).
  * z_ij = (alpha-1) * scale * q_i . k_j for active j.
@@ -170,12 +179,14 @@ typedef struct {
     double alpha, scale;
     int causal, window;
     const int *kv_len;
+    const double *alibi;   /* per-head slopes m_h [H], or NULL */
 } orc_shape;
 
-static double dotd(const double *a, const double *b, int d) {
-    double acc = 0;
-    for (int k = 0; k < d; ++k) acc += a[k] * b[k];
-    return acc;
+/* The score of an active pair: scale q_i . k_j, minus the ALiBi penalty m_h |i - j|. */
+static double score(const orc_shape *sh, int h, long i, long j, const double *q, const double *k) {
+    double s = sh->scale * dotd(q, k, sh->d);
+    if (sh->alibi) s -= sh->alibi[h] * (double)(i > j ? i - j : j - i);
+    return s;
 }
 
 static int kvl(const orc_shape *sh, int b) { return sh->kv_len ? sh->kv_len[b] : sh->L; }
@@ -191,7 +202,7 @@ static void attn_row(const orc_shape *sh, int b, int h, int i, const double *Q, 
     const size_t head = ((size_t)b * sh->H + h) * (size_t)L * d;
     const double *q = Q + head + (size_t)i * d;
     for (int j = 0; j < L; ++j)
-        srow[j] = is_active(i, j, sh->causal, sh->window, kv) ? sh->scale * dotd(q, K + head + (size_t)j * d, d)
+        srow[j] = is_active(i, j, sh->causal, sh->window, kv) ? score(sh, h, i, j, q, K + head + (size_t)j * d)
                                                                : -INFINITY;
     double tau = orc_entmax_row(srow, L, alpha, ORC_METHOD_AUTO, p, work);
     double sg = 0, ge = (2.0 - alpha) / (alpha - 1.0);
@@ -233,8 +244,8 @@ static void attn_row(const orc_shape *sh, int b, int h, int i, const double *Q, 
 }
 
 static orc_shape mkshape(int B, int H, int L, int d, double alpha, double scale, int causal,
-                         int window, const int *kv_len) {
-    orc_shape sh = {B, H, L, d, alpha, scale, causal, window, kv_len};
+                         int window, const int *kv_len, const double *alibi) {
+    orc_shape sh = {B, H, L, d, alpha, scale, causal, window, kv_len, alibi};
     return sh;
 }
 
@@ -242,10 +253,10 @@ static orc_shape mkshape(int B, int H, int L, int d, double alpha, double scale,
  * rows[r] = (b*H + h)*L + i. Outputs are indexed by r: O[r*d], tau[r], sumg[r], Ot[r*d],
  * delta[r], dQ[r*d]; any may be NULL. */
 int orc_attn_rows(int B, int H, int L, int d, double alpha, double scale, int causal, int window,
-                  const int *kv_len, const double *Q, const double *K, const double *V,
+                  const int *kv_len, const double *alibi, const double *Q, const double *K, const double *V,
                   const double *dO, const long *rows, long nrows, double *O, double *tau,
                   double *sumg, double *Ot, double *delta, double *dQ) {
-    orc_shape sh = mkshape(B, H, L, d, alpha, scale, causal, window, kv_len);
+    orc_shape sh = mkshape(B, H, L, d, alpha, scale, causal, window, kv_len, alibi);
     if (!(alpha > 1.0)) return 1;
 #pragma omp parallel
     {
@@ -269,10 +280,10 @@ int orc_attn_rows(int B, int H, int L, int d, double alpha, double scale, int ca
  * Needs tau and delta of every row of the head (indexed [(b*H+h)*L + i]).
  * Writes dK[c*d], dV[c*d]. */
 int orc_attn_cols(int B, int H, int L, int d, double alpha, double scale, int causal, int window,
-                  const int *kv_len, const double *Q, const double *K, const double *V,
+                  const int *kv_len, const double *alibi, const double *Q, const double *K, const double *V,
                   const double *dO, const double *tau, const double *delta, const long *cols,
                   long ncols, double *dK, double *dV) {
-    orc_shape sh = mkshape(B, H, L, d, alpha, scale, causal, window, kv_len);
+    orc_shape sh = mkshape(B, H, L, d, alpha, scale, causal, window, kv_len, alibi);
     if (!(alpha > 1.0)) return 1;
     const double e = 1.0 / (alpha - 1.0), ge = (2.0 - alpha) / (alpha - 1.0);
 #pragma omp parallel for schedule(dynamic, 8)
@@ -280,7 +291,7 @@ int orc_attn_cols(int B, int H, int L, int d, double alpha, double scale, int ca
         long flat = cols[c];
         int j = (int)(flat % L);
         long bh = flat / L;
-        int b = (int)(bh / H);
+        int b = (int)(bh / H), h = (int)(bh % H);
         const size_t head = (size_t)bh * (size_t)L * d;
         const int kv = kvl(&sh, b);
         double *dKj = dK + c * d, *dVj = dV + c * d;
@@ -289,7 +300,7 @@ int orc_attn_cols(int B, int H, int L, int d, double alpha, double scale, int ca
         for (int i = 0; i < L; ++i) {
             if (!is_active(i, j, sh.causal, sh.window, kv)) continue;
             const double *qi = Q + head + (size_t)i * d;
-            double u = (alpha - 1.0) * scale * dotd(qi, kj, d) - tau[bh * L + i];
+            double u = (alpha - 1.0) * score(&sh, h, i, j, qi, kj) - tau[bh * L + i];
             if (!(u > 0)) continue;
             double p = pow(u, e), g = pow(u, ge);
             const double *dOi = dO + head + (size_t)i * d;
@@ -311,9 +322,10 @@ int orc_attn_cols(int B, int H, int L, int d, double alpha, double scale, int ca
  * deciding entries lie within `margin` of tau can be told apart (M_lo != M_hi).
  * tau is indexed [(b*H+h)*L + i]. Any of M, M_lo, M_hi may be NULL. */
 int orc_block_mask(int B, int H, int L, int d, double alpha, double scale, int causal, int window,
-                   const int *kv_len, const double *Q, const double *K, const double *tau, int Br,
-                   int Bc, double margin, uint32_t *M, uint32_t *M_lo, uint32_t *M_hi) {
-    orc_shape sh = mkshape(B, H, L, d, alpha, scale, causal, window, kv_len);
+                   const int *kv_len, const double *alibi, const double *Q, const double *K,
+                   const double *tau, int Br, int Bc, double margin, uint32_t *M, uint32_t *M_lo,
+                   uint32_t *M_hi) {
+    orc_shape sh = mkshape(B, H, L, d, alpha, scale, causal, window, kv_len, alibi);
     const int Tr = (L + Br - 1) / Br, Tc = (L + Bc - 1) / Bc, Wc = (Tc + 31) / 32;
     const size_t words = (size_t)B * H * Tr * Wc;
     if (M) memset(M, 0, words * sizeof(uint32_t));
@@ -323,7 +335,7 @@ int orc_block_mask(int B, int H, int L, int d, double alpha, double scale, int c
     for (long bht = 0; bht < (long)B * H * Tr; ++bht) {
         int it = (int)(bht % Tr);
         long bh = bht / Tr;
-        int b = (int)(bh / H);
+        int b = (int)(bh / H), h = (int)(bh % H);
         const size_t head = (size_t)bh * (size_t)L * d;
         const int kv = kvl(&sh, b);
         uint32_t *row = M ? M + (size_t)bht * Wc : NULL;
@@ -333,7 +345,7 @@ int orc_block_mask(int B, int H, int L, int d, double alpha, double scale, int c
             const double t = tau[bh * L + i];
             for (int j = 0; j < L; ++j) {
                 if (!is_active(i, j, sh.causal, sh.window, kv)) continue;
-                double z = (alpha - 1.0) * scale * dotd(Q + head + (size_t)i * d, K + head + (size_t)j * d, d);
+                double z = (alpha - 1.0) * score(&sh, h, i, j, Q + head + (size_t)i * d, K + head + (size_t)j * d);
                 uint32_t bit = 1u << ((j / Bc) % 32);
                 size_t w = (size_t)(j / Bc) / 32;
                 if (row && z > t) row[w] |= bit;

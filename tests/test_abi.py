@@ -54,7 +54,7 @@ def test_workspace_bytes_valid_and_invalid(lib):
     assert n > 0 and n % 256 == 0
     # grows with L
     assert lib.entmax_attn_workspace_bytes(ctypes.byref(_desc(L=4096))) > n
-    for bad in (dict(B=0), dict(L=0), dict(d=32), dict(alpha=1.25), dict(scale=0.0), dict(causal=2),
+    for bad in (dict(B=0), dict(L=0), dict(d=32), dict(alpha=1.0), dict(alpha=17.0), dict(scale=0.0), dict(causal=2),
                 dict(max_sweeps=-1), dict(max_sweeps=65), dict(L=eb.ENTMAX_MAX_L + 1), dict(dtype=7),
                 dict(wait_limit_us=-1), dict(selftest=2)):
         assert lib.entmax_attn_workspace_bytes(ctypes.byref(_desc(**bad))) == 0, bad
@@ -62,7 +62,10 @@ def test_workspace_bytes_valid_and_invalid(lib):
 
 @pytest.mark.parametrize("bad,code", [
     (dict(d=128), eb.ENTMAX_EUNSUPPORTED),
-    (dict(alpha=3.0), eb.ENTMAX_EUNSUPPORTED),
+    (dict(alpha=17.0), eb.ENTMAX_EUNSUPPORTED),
+    (dict(alpha=1.0), eb.ENTMAX_EINVAL),
+    (dict(alpha=0.5), eb.ENTMAX_EINVAL),
+    (dict(alpha=1.25, dtype=eb.ENTMAX_FP32), eb.ENTMAX_EUNSUPPORTED),
     (dict(dtype=9), eb.ENTMAX_EINVAL),
     (dict(L=eb.ENTMAX_MAX_L + 128), eb.ENTMAX_EUNSUPPORTED),
     (dict(B=-1), eb.ENTMAX_EINVAL),
@@ -102,3 +105,9 @@ def test_rows_rejects_on_host(lib):
     assert lib.entmax_rows(p, -1, 8, 8, f15, p, p, None, None) == eb.ENTMAX_EINVAL
     assert lib.entmax_rows(p, 4, 8, 8, f15, p, p, odd, None) == eb.ENTMAX_EINVAL     # misaligned status
     assert lib.entmax_rows(p, 0, 8, 8, f15, p, p, None, None) == eb.ENTMAX_OK      # empty: no-op
+
+
+def test_general_alpha_accepted(lib):
+    """Any 1 < alpha <= 16 is a valid bf16 attention problem (run-time alpha variant)."""
+    for a in (1.01, 1.25, 1.75, 3.0, 16.0):
+        assert lib.entmax_attn_workspace_bytes(ctypes.byref(_desc(alpha=a))) > 0, a

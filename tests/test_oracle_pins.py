@@ -315,3 +315,94 @@ def test_block_mask_brute_force(alpha):
                 assert got == want, (h, it, jt)
     # margin masks bracket the exact one
     assert np.all((Mlo & ~M) == 0) and np.all((M & ~Mhi) == 0)
+
+
+# ---------------------------------------------------------------- ALiBi (NAPE heads)
+# AdaSplash-2 §4.3: NAPE heads use no positional encoding or ALiBi (Press et al.), a
+# per-head linear penalty m_h |i - j| subtracted from the scores.
+SLOPES = np.array([0.0, 0.25, 0.7])
+
+
+@pytest.mark.parametrize("alpha", (1.5, 2.0, 1.25))
+@pytest.mark.parametrize("causal", (True, False))
+def test_alibi_forward_vs_dense_composition(alpha, causal):
+    rng = np.random.default_rng(81)
+    B, H, L, d = 1, 3, 19, 8
+    Q, K, V = (rng.normal(0, s, size=(B, H, L, d)) for s in (1.5, 1.0, 1.0))
+    scale = 1 / math.sqrt(d)
+    out = oracle.Problem(Q, K, V, alpha=alpha, scale=scale, causal=causal, alibi=SLOPES).forward()
+    i = np.arange(L)[:, None]
+    j = np.arange(L)[None, :]
+    for h in range(H):
+        S = scale * Q[0, h] @ K[0, h].T - SLOPES[h] * np.abs(i - j)
+        if causal:
+            S[j > i] = -np.inf
+        P, tau = oracle.entmax_rows(S, alpha)
+        np.testing.assert_allclose(out["tau"][0, h], tau, atol=1e-13)
+        np.testing.assert_allclose(out["O"][0, h], P @ V[0, h], atol=1e-12)
+        G = np.where(P > 0, P ** (2 - alpha), 0.0)
+        np.testing.assert_allclose(out["Ot"][0, h], G @ V[0, h], atol=1e-12)
+    # A zero slope is no bias at all.
+    plain = oracle.Problem(Q, K, V, alpha=alpha, scale=scale, causal=causal).forward()
+    np.testing.assert_allclose(out["O"][0, 0], plain["O"][0, 0], atol=1e-14)
+
+
+@pytest.mark.parametrize("m", (0.3, 0.8, 1.5))
+def test_alibi_two_keys_sparsemax_closed_form(m):
+    """Q = 0 makes every raw score 0, so row 1 of a causal head sees the biased scores
+    (-m, 0). At alpha = 2 (sparsemax, Eq. 3) two scores a < b give p = ((1-(b-a))/2,
+    (1+(b-a))/2) while b - a < 1, and (0, 1) beyond."""
+    L, d = 2, 4
+    Q = np.zeros((1, 1, L, d))
+    rng = np.random.default_rng(3)
+    K, V = rng.normal(size=(1, 1, L, d)), rng.normal(size=(1, 1, L, d))
+    out = oracle.Problem(Q, K, V, alpha=2.0, scale=0.5, causal=True, alibi=[m]).forward()
+    p0 = max(0.0, (1 - m) / 2)
+    p = np.array([p0, 1 - p0])
+    np.testing.assert_allclose(out["O"][0, 0, 1], p @ V[0, 0], atol=1e-14)
+    np.testing.assert_allclose(out["tau"][0, 0, 1], (-m - 1) / 2 if m < 1 else -1.0, atol=1e-14)
+
+
+@pytest.mark.parametrize("alpha", (1.5, 1.25))
+def test_alibi_backward_finite_differences(alpha):
+    """The bias has no parameters, so the Jacobian formulas are unchanged; central
+    differences of <dO, O> check dQ, dK, dV with ALiBi on."""
+    rng = np.random.default_rng(91)
+    B, H, L, d = 1, 2, 9, 5
+    Q, K, V, dO = (rng.normal(0, s, size=(B, H, L, d)) for s in (1.25 / (alpha - 1), 1.0, 1.0, 1.0))
+    kw = dict(alpha=alpha, scale=1 / math.sqrt(d), causal=True, alibi=[0.2, 0.6])
+    g = oracle.Problem(Q, K, V, dO, **kw).backward()
+    h = 1e-6
+    for name, X in (("dQ", Q), ("dK", K), ("dV", V)):
+        fd = np.zeros_like(X)
+        for idx in np.ndindex(X.shape):
+            Xp, Xm = X.copy(), X.copy()
+            Xp[idx] += h
+            Xm[idx] -= h
+            args = {"Q": Q, "K": K, "V": V}
+            args[name[1]] = Xp
+            lp = _loss(oracle.Problem(args["Q"], args["K"], args["V"], **kw), dO)
+            args[name[1]] = Xm
+            lm = _loss(oracle.Problem(args["Q"], args["K"], args["V"], **kw), dO)
+            fd[idx] = (lp - lm) / (2 * h)
+        err = np.abs(fd - g[name]).max() / max(1e-3, np.abs(fd).max())
+        assert err < 1e-6, (name, err)
+
+
+def test_alibi_block_mask_brute_force():
+    rng = np.random.default_rng(97)
+    B, H, L, d, Br, Bc = 1, 2, 70, 8, 16, 8
+    Q, K, V = (rng.normal(0, s, size=(B, H, L, d)) for s in (2.0, 1.0, 1.0))
+    pr = oracle.Problem(Q, K, V, alpha=1.5, scale=1 / math.sqrt(d), causal=True, alibi=[0.1, 0.5])
+    tau = pr.forward()["tau"]
+    M, _, _ = pr.block_mask(tau, Br, Bc)
+    i = np.arange(L)[:, None]
+    j = np.arange(L)[None, :]
+    for h, m in enumerate((0.1, 0.5)):
+        S = (Q[0, h] @ K[0, h].T) / math.sqrt(d) - m * np.abs(i - j)
+        S[j > i] = -np.inf
+        P, _ = oracle.entmax_rows(S, 1.5)
+        for it in range(-(-L // Br)):
+            for jt in range(-(-L // Bc)):
+                want = (P[it * Br:(it + 1) * Br, jt * Bc:(jt + 1) * Bc] > 0).any()
+                assert bool((M[0, h, it, jt // 32] >> (jt % 32)) & 1) == want
