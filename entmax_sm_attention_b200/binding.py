@@ -43,7 +43,7 @@ class AttnDesc(ctypes.Structure):
         ("alpha", ctypes.c_float), ("scale", ctypes.c_float),
         ("causal", ctypes.c_int), ("window", ctypes.c_int),
         ("kv_len", ctypes.c_void_p), ("dtype", ctypes.c_int), ("max_sweeps", ctypes.c_int),
-        ("wait_limit_us", ctypes.c_int), ("selftest", ctypes.c_int),
+        ("wait_limit_us", ctypes.c_int), ("alibi_slopes", ctypes.c_void_p), ("selftest", ctypes.c_int),
     ]
 
 
@@ -116,13 +116,16 @@ class Options:
 def make_desc(B: int, H: int, L: int, d: int = 64, *, alpha: float = 1.5, scale: float | None = None,
               causal: bool = False, window: int = -1, kv_len: torch.Tensor | None = None,
               dtype: int = ENTMAX_BF16, max_sweeps: int = 0, wait_limit_us: int = 0,
-              selftest: int = 0) -> AttnDesc:
-    """Fill an entmax_attn_desc. kv_len, if given, is a device int32 tensor [B]."""
+              alibi: torch.Tensor | None = None, selftest: int = 0) -> AttnDesc:
+    """Fill an entmax_attn_desc. kv_len, if given, is a device int32 tensor [B]; alibi, if
+    given, a device float32 tensor [H] of ALiBi slopes."""
     if kv_len is not None and (kv_len.dtype != torch.int32 or not kv_len.is_cuda):
         raise ValueError("kv_len must be a CUDA int32 tensor")
+    if alibi is not None and (alibi.dtype != torch.float32 or not alibi.is_cuda or alibi.numel() != H):
+        raise ValueError("alibi must be a CUDA float32 tensor of H slopes")
     return AttnDesc(B, H, L, d, float(alpha), float(scale if scale is not None else d ** -0.5),
                     int(bool(causal) or window >= 0), int(window), _ptr(kv_len), int(dtype), int(max_sweeps),
-                    int(wait_limit_us), int(selftest))
+                    int(wait_limit_us), _ptr(alibi), int(selftest))
 
 
 def entmax_attn_workspace_bytes(desc: AttnDesc) -> int:
@@ -183,12 +186,13 @@ def mask_shape(desc: AttnDesc) -> tuple:
 
 def forward(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, *, alpha: float = 1.5, scale=None,
             causal: bool = False, window: int = -1, kv_len=None, max_sweeps: int = 0, wait_limit_us: int = 0,
-            selftest: int = 0):
+            alibi=None, selftest: int = 0):
     """O, tau and the (desc, workspace) context of one forward call on [B, H, L, 64] tensors."""
     B, H, L, d = Q.shape
     dtype = ENTMAX_BF16 if Q.dtype == torch.bfloat16 else ENTMAX_FP32
     desc = make_desc(B, H, L, d, alpha=alpha, scale=scale, causal=causal, window=window, kv_len=kv_len,
-                     dtype=dtype, max_sweeps=max_sweeps, wait_limit_us=wait_limit_us, selftest=selftest)
+                     dtype=dtype, max_sweeps=max_sweeps, wait_limit_us=wait_limit_us, alibi=alibi,
+                     selftest=selftest)
     ws = alloc_workspace(desc, Q.device)
     O = torch.empty((B, H, L, d), dtype=torch.float32, device=Q.device)
     tau = torch.empty((B, H, L), dtype=torch.float32, device=Q.device)

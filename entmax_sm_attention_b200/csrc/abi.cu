@@ -83,6 +83,7 @@ entmax_status check_desc(const entmax_attn_desc* d) {
   if (d->alpha > kMaxAlpha) return ENTMAX_EUNSUPPORTED;
   // fp32 inputs: the CUDA-core forward has closed-form powers for alpha in {1.5, 2} only.
   if (d->dtype == ENTMAX_FP32 && d->alpha != 1.5f && d->alpha != 2.0f) return ENTMAX_EUNSUPPORTED;
+  if (d->dtype == ENTMAX_FP32 && d->alibi_slopes) return ENTMAX_EUNSUPPORTED;   // bf16 path only
   return ENTMAX_OK;
 }
 
@@ -221,6 +222,8 @@ extern "C" entmax_status entmax_attn_fwd(const entmax_attn_desc* d, const void* 
   p.max_sweeps = d->max_sweeps == 0 ? kDefaultSweeps : d->max_sweeps;
   p.ae = 1.0f / (d->alpha - 1.0f);
   p.am1 = d->alpha - 1.0f;
+  p.alibi = d->alibi_slopes;
+  p.inv_scale = 1.0f / d->scale;
   p.wait_limit_ns = wait_limit_ns(d);
   p.selftest = d->selftest;
   return launch_fwd(alpha_kind(d->alpha), p, l.BH * l.Tr, s) == cudaSuccess ? ENTMAX_OK : ENTMAX_ECUDA;
@@ -266,6 +269,7 @@ extern "C" entmax_status entmax_attn_bwd(const entmax_attn_desc* d, const void* 
   p.cz = (d->alpha - 1.0f) * d->scale;
   p.scale = d->scale;
   p.ae = 1.0f / (d->alpha - 1.0f);
+  p.alibi = d->alibi_slopes;
   p.causal = d->causal || d->window >= 0;
   p.window = d->window < 0 ? -1 : d->window;
   p.wait_limit_ns = wait_limit_ns(d);
@@ -291,6 +295,8 @@ extern "C" entmax_status entmax_attn_bwd(const entmax_attn_desc* d, const void* 
   dp.BH = l.BH;
   dp.cz = (d->alpha - 1.0f) * d->scale;
   dp.ae = 1.0f / (d->alpha - 1.0f);
+  dp.alibi = d->alibi_slopes;
+  dp.scale = d->scale;
   dp.causal = d->causal || d->window >= 0;
   dp.window = d->window < 0 ? -1 : d->window;
   if (launch_delta(alpha_kind(d->alpha), dp, s) != cudaSuccess) return ENTMAX_ECUDA;

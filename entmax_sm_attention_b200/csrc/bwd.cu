@@ -227,6 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     const int row = quad * 32 + lane;
     const uint32_t tl = T + ((uint32_t)(quad * 32) << 16);
     const float cz = p.cz;
+    const float cb = p.alibi ? p.alibi[bh % p.H] / p.scale : 0.f;   // ALiBi, raw score units
     uint32_t seq = 0;
     int prev_it = -1;
     long long cyc_s = 0, cyc_mma = 0, cyc_form = 0, cyc_flush = 0;   // first row-owner warp's breakdown
@@ -289,6 +290,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
         for (int e = 0; e < 4; ++e) {
           const int c = cc * 8 + 2 * e;
           float s0 = __uint_as_float(sr[c]), s1 = __uint_as_float(sr[c + 1]);
+          if (cb != 0.f) {   // ALiBi: -cb |i - j| on the raw scores
+            const float dj = (float)(i - (j0 + qc * 32 + c));
+            s0 = fmaf(-cb, fabsf(dj), s0);
+            s1 = fmaf(-cb, fabsf(dj - 1.f), s1);
+          }
           if (!full) {
             const int jj = j0 + qc * 32 + c;
             if (!pat.active(i, jj)) s0 = -INFINITY;
@@ -488,6 +494,7 @@ __global__ void __launch_bounds__(32 * kDeltaWarps, 4) bwd_delta_kernel(const __
     }
     __syncwarp();
     const float to = p.tau[ro];
+    const float cbo = p.alibi ? p.alibi[bho % p.H] / p.scale : 0.f;   // ALiBi of the row's head
     const uint4* Ko = reinterpret_cast<const uint4*>(p.K + (size_t)bho * p.L * kD);
     const uint4* Vo = reinterpret_cast<const uint4*>(p.V16 + (size_t)bho * p.L * kD);
     const int b = bho / p.H;
@@ -503,7 +510,8 @@ __global__ void __launch_bounds__(32 * kDeltaWarps, 4) bwd_delta_kernel(const __
         for (int jj = lane; jj < kTile; jj += 32) {   // four keys per lane, loads in flight together
           const int jk = jt * kTile + jj;
           if (jk < p.L && pat.active(i, jk)) {
-            const float uu = fmaf(dot_s(Ko + (size_t)jk * 8, xs[warp][0], false), p.cz, -to);
+            const float sraw = dot_s(Ko + (size_t)jk * 8, xs[warp][0], false) - cbo * fabsf((float)(i - jk));
+            const float uu = fmaf(sraw, p.cz, -to);
             if (uu > 0.f) {
               const float g = (AK == kAlpha15) ? uu : (AK == kAlpha2 ? 1.f : pow_pos(uu, p.ae - 1.f));
               og += g;

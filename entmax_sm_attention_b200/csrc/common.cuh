@@ -19,6 +19,16 @@ constexpr int kMaskWords = kMaxTc / 32;
 //     logarithm: relative error near 2^-22 each).
 enum AlphaKind { kAlpha15 = 0, kAlpha2 = 1, kAlphaGen = 2 };
 
+// ALiBi ("AdaSplash-2" §4.3, NAPE heads; Press et al.): the score of key j for query i
+// is lowered by m_h |i - j|. The kernels work on raw scores s = q . k (z = cz s), so they
+// subtract cb |i - j| with cb = m_h / scale from the raw scores of keys j0 + c.
+template <int N>
+__device__ __forceinline__ void alibi_apply(float (&s)[N], float cb, int i, int j0) {
+  const float base = (float)(i - j0);
+#pragma unroll
+  for (int c = 0; c < N; ++c) s[c] = fmaf(-cb, fabsf(base - (float)c), s[c]);
+}
+
 // u^x for u > 0 (exp2 of x log2 u); callers pass only positive u.
 __device__ __forceinline__ float pow_pos(float u, float x) { return exp2f(x * __log2f(u)); }
 

@@ -606,6 +606,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     const bool valid = i < p.L;
     const uint32_t tl = T + ((uint32_t)(quad * 32) << 16);
     const float cz = p.cz;
+    const float cb = p.alibi ? p.alibi[bh % p.H] * p.inv_scale : 0.f;   // ALiBi, raw score units
     uint32_t sfull_par = 0, sbuf = 0;
     float m = -INFINITY;
     float top[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
@@ -628,6 +629,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       tc_fence_before();
       warp_arrive(&sh.s_free[bf]);
       DIAG(dtk = clock64(); dgr[1] += dtk - d2);
+      if (cb != 0.f) alibi_apply(s, cb, i, j0);
       if (!pat.block_full(i0, i1, jt * kTile, jt * kTile + kTile)) {
 #pragma unroll
         for (int c = 0; c < kCols; ++c)
@@ -753,6 +755,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           float s[kCols];
           ldc(tl + pa + qp * kCols, s);
           DIAG(const long long d2 = clock64(); dgr[6] += d2 - d1);
+          if (cb != 0.f) alibi_apply(s, cb, i, j0);
           if (!pat.block_full(i0, i1, jt * kTile, jt * kTile + kTile)) {
 #pragma unroll
             for (int cc = 0; cc < kCols; ++cc)
@@ -916,6 +919,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         tc_fence_before();
         warp_arrive(&sh.s_free[bf]);
         DIAG(dtk = clock64(); dgr[4] += dtk - d2);
+        if (cb != 0.f) alibi_apply(s, cb, i, j0);
         if (!pat.block_full(i0, i1, jt * kTile, jt * kTile + kTile)) {
 #pragma unroll
           for (int cc = 0; cc < kCols; ++cc)

@@ -40,6 +40,8 @@ struct FwdParams {
   int H, L, Tr, Tc, Wc, Wr, BH;
   float cz;                 // (alpha - 1) * scale
   float ae, am1;            // 1 / (alpha - 1) and alpha - 1 (the run-time alpha variant)
+  const float* alibi;       // [H] ALiBi slopes (score units per position), or nullptr
+  float inv_scale;          // 1 / scale (ALiBi slopes in raw score units)
   int causal, window, max_sweeps;
   unsigned long long wait_limit_ns;   // bound on every in-kernel wait
   int selftest;             // kSelftestStall: one wait per CTA on a barrier nothing completes
@@ -61,6 +63,7 @@ struct BwdParams {
   float cz;                      // (alpha - 1) * scale
   float scale;
   float ae;                      // 1 / (alpha - 1)
+  const float* alibi;            // [H] ALiBi slopes, or nullptr
   int causal, window;
   unsigned long long wait_limit_ns;
   int selftest;
@@ -82,6 +85,8 @@ struct DeltaParams {
   int H, L, Tr, Wc, BH;
   float cz;
   float ae;                     // 1 / (alpha - 1)
+  const float* alibi;           // [H] ALiBi slopes, or nullptr
+  float scale;
   int causal, window;
 };
 

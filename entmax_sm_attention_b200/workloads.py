@@ -38,6 +38,7 @@ class Workload:
     alphas: tuple = (1.5,)
     sigma_q: float = 1.0
     backward: bool = True
+    alibi: tuple | None = None   # ALiBi slopes per head (score units per position), or None
     note: str = ""
     extra: dict = field(default_factory=dict)
 
@@ -104,10 +105,10 @@ def make_score_rows(rows: int, n: int, seed: int = 0, sigma: float = 1.0) -> tor
 
 
 def small_case(name: str, *, B=1, H=2, L=300, d=64, dtype="bf16", causal=False, window=-1,
-               kv_len=None, sigma_q=1.0, alphas=(1.5, 2.0)) -> Workload:
+               kv_len=None, sigma_q=1.0, alphas=(1.5, 2.0), alibi=None) -> Workload:
     """A reduced workload the oracle finishes in seconds: several tiles plus a ragged tail."""
     return Workload(name, B=B, H=H, L=L, d=d, dtype=dtype, causal=causal, window=window,
-                    kv_len=kv_len, sigma_q=sigma_q, alphas=alphas)
+                    kv_len=kv_len, sigma_q=sigma_q, alphas=alphas, alibi=None if alibi is None else tuple(alibi))
 
 
 def make_planted_inputs(w: Workload, rho: float, seed: int = 0, gamma: float = 3.0) -> dict:

@@ -14,6 +14,7 @@
  *   - Appendix C.4: mask packing, 32 key tiles per uint32.
  *   - "gpt2-adasplash-attention" model card, "Causal Splash Masking with Sink
  *     Preservation": window mask {0} U [max(1, i-W), i].
+ *   - §4.3, NAPE heads: an optional ALiBi distance penalty per head (see alibi_slopes).
  * At alpha = 1.5 this equals the model cards' score-unit form
  * A_ij = max(0, (s_ij - tau'_i)/2)^2 with tau' = tau / (alpha-1).
  *
@@ -95,6 +96,10 @@ typedef struct {
     int max_sweeps;       /* cap on threshold-refinement passes; 0 = library default (12) */
     int wait_limit_us;    /* bound on each in-kernel wait in microseconds; 0 = 2 s.
                              Must be >= 0.                                                 */
+    const float *alibi_slopes; /* device float[H] or NULL. ALiBi ("AdaSplash-2" §4.3: NAPE
+                             heads; Press et al.): the score of key j for query i becomes
+                             scale q_i . k_j - alibi_slopes[h] |i - j| (0 for a head without
+                             it). bf16 inputs only (fp32 -> ENTMAX_EUNSUPPORTED).          */
     int selftest;         /* 0 for normal use. ENTMAX_SELFTEST_STALL makes one thread of
                              every CTA of the fwd/bwd kernels wait on a barrier that
                              nothing completes, so that the wait expires after

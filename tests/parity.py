@@ -31,8 +31,9 @@ MARGIN = 1e-3
 def gpu_run(inp: dict, w: Workload, alpha: float, backward: bool = True, max_sweeps: int = 0):
     dev = {k: v.cuda() for k, v in inp.items()}
     kv = None if w.kv_len is None else torch.tensor(w.kv_len_list(), dtype=torch.int32, device="cuda")
+    ab = None if w.alibi is None else torch.tensor(w.alibi, dtype=torch.float32, device="cuda")
     O, tau, ctx = eb.forward(dev["Q"], dev["K"], dev["V"], alpha=alpha, scale=w.scale, causal=w.causal,
-                             window=w.window, kv_len=kv, max_sweeps=max_sweeps)
+                             window=w.window, kv_len=kv, max_sweeps=max_sweeps, alibi=ab)
     out = {"O": O, "tau": tau}
     if backward:
         out["dQ"], out["dK"], out["dV"] = eb.backward(ctx, dev["Q"], dev["K"], dev["V"], dev["dO"], tau)
@@ -48,7 +49,7 @@ def gpu_run(inp: dict, w: Workload, alpha: float, backward: bool = True, max_swe
 
 def oracle_problem(inp: dict, w: Workload, alpha: float) -> oracle.Problem:
     return oracle.Problem(inp["Q"], inp["K"], inp["V"], inp["dO"], alpha=alpha, scale=w.scale, causal=w.causal,
-                          window=w.window, kv_len=w.kv_len_list())
+                          window=w.window, kv_len=w.kv_len_list(), alibi=w.alibi)
 
 
 def alpha2_exclusions(pr: oracle.Problem, tau_ref: np.ndarray, tau_gpu: np.ndarray):
@@ -82,6 +83,8 @@ def alpha2_exclusions(pr: oracle.Problem, tau_ref: np.ndarray, tau_gpu: np.ndarr
         for h in range(H):
             Q, K = pr.Q[b, h], pr.K[b, h]
             z = c * (Q @ K.T)
+            if pr.alibi is not None:   # ALiBi: the penalty m_h |i - j| on the scores
+                z = z - (pr.alpha - 1) * pr.alibi[h] * np.abs(i - j)
             t = tau_ref[b, h][:, None]
             band = (4 * np.abs(tau_gpu[b, h] - tau_ref[b, h])[:, None]
                     + 2.0 ** -15 * c * (np.abs(Q) @ np.abs(K).T) + 2.0 ** -20)

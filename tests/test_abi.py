@@ -42,11 +42,11 @@ def test_library_exports_every_declared_symbol(lib):
 
 def _desc(**kw):
     base = dict(B=1, H=2, L=300, d=64, alpha=1.5, scale=0.125, causal=0, window=-1, kv_len=None,
-                dtype=eb.ENTMAX_BF16, max_sweeps=0, wait_limit_us=0, selftest=0)
+                dtype=eb.ENTMAX_BF16, max_sweeps=0, wait_limit_us=0, alibi_slopes=None, selftest=0)
     base.update(kw)
     return eb.AttnDesc(base["B"], base["H"], base["L"], base["d"], base["alpha"], base["scale"], base["causal"],
                        base["window"], base["kv_len"], base["dtype"], base["max_sweeps"], base["wait_limit_us"],
-                       base["selftest"])
+                       base["alibi_slopes"], base["selftest"])
 
 
 def test_workspace_bytes_valid_and_invalid(lib):
@@ -66,6 +66,7 @@ def test_workspace_bytes_valid_and_invalid(lib):
     (dict(alpha=1.0), eb.ENTMAX_EINVAL),
     (dict(alpha=0.5), eb.ENTMAX_EINVAL),
     (dict(alpha=1.25, dtype=eb.ENTMAX_FP32), eb.ENTMAX_EUNSUPPORTED),
+    (dict(alibi_slopes=1 << 20, dtype=eb.ENTMAX_FP32), eb.ENTMAX_EUNSUPPORTED),
     (dict(dtype=9), eb.ENTMAX_EINVAL),
     (dict(L=eb.ENTMAX_MAX_L + 128), eb.ENTMAX_EUNSUPPORTED),
     (dict(B=-1), eb.ENTMAX_EINVAL),
@@ -111,3 +112,9 @@ def test_general_alpha_accepted(lib):
     """Any 1 < alpha <= 16 is a valid bf16 attention problem (run-time alpha variant)."""
     for a in (1.01, 1.25, 1.75, 3.0, 16.0):
         assert lib.entmax_attn_workspace_bytes(ctypes.byref(_desc(alpha=a))) > 0, a
+
+
+def test_desc_layout_matches_header():
+    """The ctypes mirror has the header's field order (checked by offsets of the tail)."""
+    assert eb.AttnDesc.alibi_slopes.offset % 8 == 0
+    assert eb.AttnDesc.selftest.offset > eb.AttnDesc.alibi_slopes.offset
