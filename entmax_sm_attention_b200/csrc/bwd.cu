@@ -63,7 +63,7 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 
 int bwd_smem_bytes() { return 1024 + 2 * kTileBytes + kStages * kPairBytes + 6 * kTileBytes + 2 * kTileBytes; }
 
-template <int AK>
+template <int AK, bool kAlibi>
 __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant__ BwdParams p) {
   extern __shared__ uint8_t dsm_raw[];
   __shared__ Shared sh;
@@ -227,7 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     const int row = quad * 32 + lane;
     const uint32_t tl = T + ((uint32_t)(quad * 32) << 16);
     const float cz = p.cz;
-    const float cb = p.alibi ? p.alibi[bh % p.H] / p.scale : 0.f;   // ALiBi, raw score units
+    const float cb = kAlibi ? p.alibi[bh % p.H] / p.scale : 0.f;   // ALiBi, raw score units
     uint32_t seq = 0;
     int prev_it = -1;
     long long cyc_s = 0, cyc_mma = 0, cyc_form = 0, cyc_flush = 0;   // first row-owner warp's breakdown
@@ -290,7 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
         for (int e = 0; e < 4; ++e) {
           const int c = cc * 8 + 2 * e;
           float s0 = __uint_as_float(sr[c]), s1 = __uint_as_float(sr[c + 1]);
-          if (cb != 0.f) {   // ALiBi: -cb |i - j| on the raw scores
+          if constexpr (kAlibi) {   // ALiBi: -cb |i - j| on the raw scores
             const float dj = (float)(i - (j0 + qc * 32 + c));
             s0 = fmaf(-cb, fabsf(dj), s0);
             s1 = fmaf(-cb, fabsf(dj - 1.f), s1);
@@ -397,9 +397,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
 
 cudaError_t launch_bwd(int alpha_kind, const BwdParams& p, int grid, cudaStream_t s) {
   const int smem = bwd_smem_bytes();
-  auto kern = alpha_kind == kAlpha15 ? bwd_kernel<kAlpha15>
-             : alpha_kind == kAlpha2 ? bwd_kernel<kAlpha2>
-                                     : bwd_kernel<kAlphaGen>;
+  const bool ab = p.alibi != nullptr;   // compile-time ALiBi variant, as in the forward
+  auto kern = alpha_kind == kAlpha15 ? (ab ? bwd_kernel<kAlpha15, true> : bwd_kernel<kAlpha15, false>)
+             : alpha_kind == kAlpha2 ? (ab ? bwd_kernel<kAlpha2, true> : bwd_kernel<kAlpha2, false>)
+                                     : (ab ? bwd_kernel<kAlphaGen, true> : bwd_kernel<kAlphaGen, false>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   kern<<<grid, kThreads, smem, s>>>(p);

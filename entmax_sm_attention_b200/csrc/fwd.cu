@@ -340,7 +340,7 @@ __device__ __forceinline__ float solveN(const float (&v)[N], float cz, float e, 
 
 }  // namespace
 
-template <int AK>
+template <int AK, bool kAlibi>
 __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant__ FwdParams p) {
   using OL = OutLayout<AK>;
   constexpr int kOBufs = OL::kBufs;
@@ -606,7 +606,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     const bool valid = i < p.L;
     const uint32_t tl = T + ((uint32_t)(quad * 32) << 16);
     const float cz = p.cz;
-    const float cb = p.alibi ? p.alibi[bh % p.H] * p.inv_scale : 0.f;   // ALiBi, raw score units
+    const float cb = kAlibi ? p.alibi[bh % p.H] * p.inv_scale : 0.f;   // ALiBi, raw score units
     uint32_t sfull_par = 0, sbuf = 0;
     float m = -INFINITY;
     float top[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
@@ -629,7 +629,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       tc_fence_before();
       warp_arrive(&sh.s_free[bf]);
       DIAG(dtk = clock64(); dgr[1] += dtk - d2);
-      if (cb != 0.f) alibi_apply(s, cb, i, j0);
+      if constexpr (kAlibi) alibi_apply(s, cb, i, j0);
       if (!pat.block_full(i0, i1, jt * kTile, jt * kTile + kTile)) {
 #pragma unroll
         for (int c = 0; c < kCols; ++c)
@@ -755,7 +755,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           float s[kCols];
           ldc(tl + pa + qp * kCols, s);
           DIAG(const long long d2 = clock64(); dgr[6] += d2 - d1);
-          if (cb != 0.f) alibi_apply(s, cb, i, j0);
+          if constexpr (kAlibi) alibi_apply(s, cb, i, j0);
           if (!pat.block_full(i0, i1, jt * kTile, jt * kTile + kTile)) {
 #pragma unroll
             for (int cc = 0; cc < kCols; ++cc)
@@ -919,7 +919,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         tc_fence_before();
         warp_arrive(&sh.s_free[bf]);
         DIAG(dtk = clock64(); dgr[4] += dtk - d2);
-        if (cb != 0.f) alibi_apply(s, cb, i, j0);
+        if constexpr (kAlibi) alibi_apply(s, cb, i, j0);
         if (!pat.block_full(i0, i1, jt * kTile, jt * kTile + kTile)) {
 #pragma unroll
           for (int cc = 0; cc < kCols; ++cc)
@@ -1083,9 +1083,11 @@ int fwd_smem_bytes(int Tc) { return 1024 + fwd_off_region() + fwd_region_bytes(T
 
 cudaError_t launch_fwd(int alpha_kind, const FwdParams& p, int grid, cudaStream_t s) {
   const int smem = fwd_smem_bytes(p.Tc);
-  auto kern = alpha_kind == kAlpha15 ? fwd_kernel<kAlpha15>
-             : alpha_kind == kAlpha2 ? fwd_kernel<kAlpha2>
-                                     : fwd_kernel<kAlphaGen>;
+  // ALiBi is a compile-time variant so heads without the bias carry none of its code.
+  const bool ab = p.alibi != nullptr;
+  auto kern = alpha_kind == kAlpha15 ? (ab ? fwd_kernel<kAlpha15, true> : fwd_kernel<kAlpha15, false>)
+             : alpha_kind == kAlpha2 ? (ab ? fwd_kernel<kAlpha2, true> : fwd_kernel<kAlpha2, false>)
+                                     : (ab ? fwd_kernel<kAlphaGen, true> : fwd_kernel<kAlphaGen, false>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   kern<<<grid, kThreads, smem, s>>>(p);
