@@ -86,8 +86,15 @@ constexpr int kMaxVotes = 72;
 #define DIAG(...)
 #endif
 
+// What the decision step publishes to the TMA and MMA warps: a refinement sweep (K tiles,
+// S only), an output pass (K and V tiles, S and O), the fused first pass (an output pass at
+// tau_T whose row owners also collect the candidates; more decisions follow), or nothing
+// more (the fused pass's O is final).
 constexpr int kKindSweep = 0;
 constexpr int kKindOutput = 1;
+constexpr int kKindFused = 2;
+constexpr int kKindDone = 3;
+__device__ __forceinline__ bool last_kind(int kind) { return kind == kKindOutput || kind == kKindDone; }
 
 struct Shared {
   uint64_t full[kSlots], empty[kSlots];
@@ -448,7 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       if (lane == 0) {
         if (kind == kKindSweep) {
           for_each_bit(list, kMaskWords, [&](int jt) { load(&p.tK, jt); });
-        } else {
+        } else if (kind != kKindDone) {
           for_each_bit(list, kMaskWords, [&](int jt) {
             load(&p.tK, jt);
             load(&p.tV, jt);
@@ -456,7 +463,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         }
       }
       __syncwarp();
-      if (kind != kKindSweep) break;
+      if (last_kind(kind)) break;
     }
     DIAG(if (lane == 0) p.stats[((size_t)bh * p.Tr + qt) * kFwdStats + 15] = (int)dg_wait);
     // Make sure no copy is still in flight when the CTA retires.
@@ -471,6 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     uint32_t seq = 0;            // next ring position (sweeps consume in order)
     uint32_t sfree_par = 0;      // per sweep S buffer: parity of its uses so far (bit b)
     uint32_t sbuf = 0;           // next sweep S buffer
+    uint32_t obase = 0;          // output tiles of earlier output-type passes (buffer phases)
     bool live = true;            // false after a failed wait: no further MMA is issued
     // Two S issuers share the max pass and the sweeps: issuer me takes the tiles whose
     // buffer (tile index % 4) has parity me, so each one's barrier probes and commits
@@ -523,42 +531,47 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         if (kind == kKindSweep) {
           sbuf = 0;
           for_each_bit(list, kMaskWords, [&](int) { sweep_tile(); });
-        } else if (me == 0) {
-          // Output pass: this warp issues only the S tiles; tile k uses buffer c = k % 3
-          // at TMEM column 0, 128 or 384, which is free once O and Ot of tile k-3 are done.
-          // K_k is at ring position base + 2k, V_k at base + 2k + 1.
+        } else if (kind != kKindDone) {
           int n = 0;
 #pragma unroll
           for (int w = 0; w < kMaskWords; ++w) n += __popc(list[w]);
-          const uint32_t base = seq;
-          for (int k = 0; k < n; ++k) {
-            const int c = k % kOBufs;
-            const uint32_t pos = base + 2 * k;
-            DIAG(const long long d0 = clock64());
-            if (k >= kOBufs)
-              live = live && mbar_wait2(&sh.pv_done[c], ((k - kOBufs) / kOBufs) & 1, &sh.full[pos % kSlots],
-                                        (pos / kSlots) & 1, wc);
-            else
-              live = live && mbar_wait(&sh.full[pos % kSlots], (pos / kSlots) & 1, wc);
-            DIAG(dg_out += clock64() - d0);
-            if (!live) break;
-            mma_s(pos, OL::sbuf(c));
-            mma_commit(&sh.o_full[c]);
+          if (me == 0) {
+            // Output-type pass: this warp issues only the S tiles. Tile k of the pass is
+            // output tile ko = obase + k overall and uses buffer c = ko % 3 (TMEM column 0,
+            // 128 or 384), free once O of output tile ko - 3 is done. K_k is at ring
+            // position seq + 2k, V_k at seq + 2k + 1.
+            for (int k = 0; k < n; ++k) {
+              const uint32_t ko = obase + k;
+              const int c = ko % kOBufs;
+              const uint32_t pos = seq + 2 * k;
+              DIAG(const long long d0 = clock64());
+              if (ko >= kOBufs)
+                live = live && mbar_wait2(&sh.pv_done[c], ((ko - kOBufs) / kOBufs) & 1, &sh.full[pos % kSlots],
+                                          (pos / kSlots) & 1, wc);
+              else
+                live = live && mbar_wait(&sh.full[pos % kSlots], (pos / kSlots) & 1, wc);
+              DIAG(dg_out += clock64() - d0);
+              if (!live) break;
+              mma_s(pos, OL::sbuf(c));
+              mma_commit(&sh.o_full[c]);
+            }
+            DIAG(p.stats[((size_t)bh * p.Tr + qt) * kFwdStats + 12] = (int)dg_sw);
+            DIAG(p.stats[((size_t)bh * p.Tr + qt) * kFwdStats + 13] = (int)dg_out);
+            DIAG(p.stats[((size_t)bh * p.Tr + qt) * kFwdStats + 25] = (int)(dg_iss - dg_sw));
           }
-          seq = base + 2 * n;
-          DIAG(p.stats[((size_t)bh * p.Tr + qt) * kFwdStats + 12] = (int)dg_sw);
-          DIAG(p.stats[((size_t)bh * p.Tr + qt) * kFwdStats + 13] = (int)dg_out);
-          DIAG(p.stats[((size_t)bh * p.Tr + qt) * kFwdStats + 25] = (int)(dg_iss - dg_sw));
+          seq += 2 * n;
+          obase += n;
         }
       }
       __syncwarp();
-      if (kind != kKindSweep) break;
+      if (last_kind(kind)) break;
     }
   } else if (warp == kOWarp) {
-    // ------------------------------------------------------ O issuer (output pass)
+    // ------------------------------------------------------ O issuer (output passes)
     const uint32_t idO = idesc_f16(128, 64, 0, 1);
     const uint64_t vd0 = sdesc_sw128(smem_u32(ring), 8192, 1024);   // ring slot 0, MN-major
-    uint32_t seq = 0;   // ring positions, tracked exactly like the producer's
+    uint32_t seq = 0;     // ring positions, tracked exactly like the producer's
+    uint32_t obase = 0;   // output tiles of earlier output-type passes
     for_each_bit(act, kMaskWords, [&](int) { ++seq; });
     while (true) {
       named_bar(1, kThreads);
@@ -571,32 +584,36 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       for (int w = 0; w < kMaskWords; ++w) n += __popc(list[w]);
       if (kind == kKindSweep) {
         seq += n;
-      } else if (lane == 0) {
-        DIAG(long long dg_o = 0);
-        const uint32_t base = seq;
-        for (int k = 0; k < n; ++k) {
-          const int c = k % kOBufs;
-          const uint32_t pa = OL::sbuf(c);
-          const uint32_t vpos = base + 2 * k + 1;
-          const int vslot = vpos % kSlots;
-          DIAG(const long long d0 = clock64());
-          if (!mbar_wait2(&sh.full[vslot], (vpos / kSlots) & 1, &sh.o_ready[c], (k / kOBufs) & 1, wc)) break;
-          DIAG(dg_o += clock64() - d0);
-          tc_fence_after();
-          const uint64_t vd = sdesc_add(vd0, vslot * kTileBytes);
+      } else if (kind != kKindDone) {
+        if (lane == 0) {
+          DIAG(long long dg_o = 0);
+          for (int k = 0; k < n; ++k) {
+            const uint32_t ko = obase + k;
+            const int c = ko % kOBufs;
+            const uint32_t pa = OL::sbuf(c);
+            const uint32_t vpos = seq + 2 * k + 1;
+            const int vslot = vpos % kSlots;
+            DIAG(const long long d0 = clock64());
+            if (!mbar_wait2(&sh.full[vslot], (vpos / kSlots) & 1, &sh.o_ready[c], (ko / kOBufs) & 1, wc)) break;
+            DIAG(dg_o += clock64() - d0);
+            tc_fence_after();
+            const uint64_t vd = sdesc_add(vd0, vslot * kTileBytes);
 #pragma unroll
-          for (int t = 0; t < 8; ++t) {
-            // keys 16t..16t+15: part 16t / kCols, pair columns ((16t) % kCols) / 2 of its A block
-            const uint32_t col = pa + (16 * t / kCols) * kCols + ((16 * t) % kCols) / 2;   // A block
-            mma_ts(T + 256, T + col, sdesc_add(vd, t * 2048), idO, (k > 0 || t > 0) ? 1u : 0u);
+            for (int t = 0; t < 8; ++t) {
+              // keys 16t..16t+15: part 16t / kCols, pair columns ((16t) % kCols) / 2 of its A block
+              const uint32_t col = pa + (16 * t / kCols) * kCols + ((16 * t) % kCols) / 2;   // A block
+              mma_ts(T + 256, T + col, sdesc_add(vd, t * 2048), idO, (k > 0 || t > 0) ? 1u : 0u);
+            }
+            mma_commit(&sh.empty[vslot]);   // V_k is read by this issuer only
+            mma_commit(&sh.pv_done[c]);
           }
-          mma_commit(&sh.empty[vslot]);   // V_k is read by this issuer only
-          mma_commit(&sh.pv_done[c]);
+          DIAG(p.stats[((size_t)bh * p.Tr + qt) * kFwdStats + 14] = (int)dg_o);
         }
-        DIAG(p.stats[((size_t)bh * p.Tr + qt) * kFwdStats + 14] = (int)dg_o);
+        seq += 2 * n;
+        obase += n;
       }
       __syncwarp();
-      if (kind != kKindSweep) break;
+      if (last_kind(kind)) break;
     }
   } else {
     // ---------------------------------------------------------------- row owners
@@ -689,15 +706,100 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       DIAG(dgx[0] += clock64() - ds0);
     }
     int sweeps = 0;
-    uint32_t n_s = 0;   // S tiles computed (phase 1, sweeps, output) for the counters
+    int fused_passes = 0;   // the fused first pass counts as a sweep for max_sweeps, not in the counters
+    uint32_t n_s = 0;       // S tiles computed (phase 1, sweeps, output) for the counters
+    uint32_t obase = 0;     // output tiles of earlier output-type passes (barrier phases)
+    float tau_T = tau;      // the threshold at which the fused pass formed A
     for_each_bit(act, kMaskWords, [&](int) { ++n_s; });
+    float* mycand = cand + qp * cap * kTile + row;
+    uint16_t* myidx = cidx + qp * cap * kTile + row;
 
-    // Decision points: publish either one more refinement sweep or the final mask.
+    // Candidate collection on one tile's scores: the maxima of the four 8-key groups
+    // (independent trees), then an element scan of only the groups whose maximum passes
+    // tau. A group is scanned when any lane of the warp has a candidate in it (a
+    // warp-uniform branch); each lane then runs the same branch-free append.
+    auto collect_tile = [&](const float (&sv)[kCols], int j0, bool collect) {
+      float gm[kCols / 8];
+#pragma unroll
+      for (int g = 0; g < kCols / 8; ++g) {
+        const float* x = sv + 8 * g;
+        gm[g] = fmaxf(fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3])), fmaxf(fmaxf(x[4], x[5]), fmaxf(x[6], x[7])));
+      }
+#pragma unroll
+      for (int g = 0; g < kCols / 8; ++g)
+        if (__any_sync(0xffffffffu, collect && fmaf(gm[g], cz, -tau) > 0.f))
+          if (collect) collect8(sv + 8 * g, j0 + 8 * g, cz, tau, cap, mycand, myidx, nc);
+    };
+    // One tile of an output-type pass (output tile ko overall, buffer ko % 3): recompute
+    // S, optionally collect this thread's candidates at tau, and write A = u^{1/(alpha-1)}
+    // at tau in fp16 over the S columns this thread has read (the part's keys qp*kCols..
+    // go into its own columns [qp*kCols, +kCols/2), so the row's other parts never see an
+    // overwritten S value).
+    auto out_tile = [&](int jt, uint32_t ko, bool collect) {
+      const int c = ko % kOBufs;
+      const uint32_t pa = OL::sbuf(c);
+      DIAG(const long long d0 = clock64());
+      warp_wait(&sh.o_full[c], (ko / kOBufs) & 1, wc);
+      DIAG(const long long d1 = clock64(); dg_s3 += d1 - d0);
+      tc_fence_after();
+      const int j0 = jt * kTile + qp * kCols;
+      float s[kCols];
+      ldc(tl + pa + qp * kCols, s);
+      DIAG(const long long d2 = clock64(); dgr[6] += d2 - d1);
+      if constexpr (kAlibi) alibi_apply(s, cb, i, j0);
+      if (!pat.block_full(i0, i1, jt * kTile, jt * kTile + kTile)) {
+#pragma unroll
+        for (int cc = 0; cc < kCols; ++cc)
+          if (!pat.active(i, j0 + cc)) s[cc] = -INFINITY;
+      }
+      if (collect) collect_tile(s, j0, !done);   // collect is warp-uniform
+      uint32_t aw[kCols / 2];
+#pragma unroll
+      for (int cc = 0; cc < kCols / 2; ++cc) {
+        const float2 u = __ffma2_rn(make_float2(s[2 * cc], s[2 * cc + 1]), make_float2(cz, cz),
+                                    make_float2(-tau, -tau));
+        const float v0 = fmaxf(u.x, 0.f), v1 = fmaxf(u.y, 0.f);
+        if constexpr (AK == kAlpha15) {
+          const float2 a = __fmul2_rn(make_float2(v0, v1), make_float2(v0, v1));
+          aw[cc] = pack_f16(a.x, a.y);
+        } else if constexpr (AK == kAlpha2) {
+          aw[cc] = pack_f16(v0, v1);
+        } else {
+          aw[cc] = pack_f16(v0 > 0.f ? pow_pos(v0, p.ae) : 0.f, v1 > 0.f ? pow_pos(v1, p.ae) : 0.f);
+        }
+      }
+      const uint32_t col = pa + qp * kCols;
+      DIAG(const long long d3 = clock64(); dgr[7] += d3 - d2);
+#pragma unroll
+      for (int h = 0; h < kCols / 32; ++h) tmem_st16(tl + col + 16 * h, *reinterpret_cast<uint32_t(*)[16]>(&aw[16 * h]));
+      tmem_wait_st();
+      tc_fence_before();
+      warp_arrive(&sh.o_ready[c]);
+      DIAG(dgr[8] += clock64() - d3);
+      ++n_s;
+    };
+
+    // Decision points: publish one more refinement sweep, the fused first pass, the final
+    // mask with an output pass, or the final mask alone.
+    //
+    // For alpha in {1.5, 2} the first pass after the max pass is fused: an output pass at
+    // tau_T over the tiles where some row has a score above tau_T, whose row owners also
+    // collect the candidates (u_T > 0). A row whose copies fit is then solved exactly on
+    // them, and its O = sum_j A*_j V_j follows from the pass's O_T = sum_j fp16(A_T,j) V_j
+    // (every j with u_T,j > 0 lies in a visited tile) and its copies: the epilogue adds
+    // sum_j (A*_j - fp16(A_T,j)) V_j over the copies in fp32, with A* at the final tau
+    // (zero outside the support). When every row of the tile is solved that way no second
+    // pass over K and V is needed. Otherwise the remaining rows sweep as below, and an
+    // output pass at the final tau recomputes O for the whole tile.
     for (int r = 0;; ++r) {
       DIAG(const long long dd0 = clock64());
       const int buf = r & 1;
       const bool need = !done && sweeps < p.max_sweeps;
       const bool final_mask = !rows_any(need, sh.votes, r, lane, kMathThreads);
+      const bool fuse = AK != kAlphaGen && r == 0 && !final_mask;
+      // The fused pass's O is final when every row was solved on that pass's copies.
+      const bool o_final = AK != kAlphaGen && r == 1 && final_mask &&
+                           !rows_any(valid && !listed, sh.votes, kMaxVotes - 1, lane, kMathThreads);
       if (qp == 0) {
         // Tiles that some row still needs (refinement) or that hold a nonzero (mask): each
         // warp builds a word of 32 tile bits from eight independent loads and votes per
@@ -722,7 +824,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       }
       named_bar(2, kMathThreads);
       if (tid == 0) {
-        sh.ctl_kind = final_mask ? kKindOutput : kKindSweep;
+        sh.ctl_kind = final_mask ? (o_final ? kKindDone : kKindOutput) : (fuse ? kKindFused : kKindSweep);
         sh.ctl_buf = buf;
         for (int w = 0; w < kMaskWords; ++w) sh.lists[buf ^ 1][w] = 0;   // for the next decision
       }
@@ -733,7 +835,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       DIAG(dgx[1] += clock64() - dd0);
 
       if (final_mask) {
-        clk2 = clock64();
+        if (!o_final) clk2 = clock64();
         if (!done && qp == 0) atomicOr(status, kStatusNoConverge);   // cap reached; tau stays bracketed
         // Block mask row of this query tile and the transposed bits (Appendix C.4).
         if (tid < p.Wc) p.M[((size_t)bh * p.Tr + qt) * p.Wc + tid] = list[tid];
@@ -742,60 +844,19 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
             atomicOr(&p.MT[((size_t)bh * p.Tc + jt) * p.Wr + (qt >> 5)], 1u << (qt & 31));
           });
         }
-        // Phase 4: output pass over the flagged tiles, buffers c = k % 3.
-        int k = 0;
-        for_each_bit(list, kMaskWords, [&](int jt) {
-          const int c = k % kOBufs;
-          const uint32_t pa = OL::sbuf(c);
-          DIAG(const long long d0 = clock64());
-          warp_wait(&sh.o_full[c], (k / kOBufs) & 1, wc);
-          DIAG(const long long d1 = clock64(); dg_s3 += d1 - d0);
-          tc_fence_after();
-          const int j0 = jt * kTile + qp * kCols;
-          float s[kCols];
-          ldc(tl + pa + qp * kCols, s);
-          DIAG(const long long d2 = clock64(); dgr[6] += d2 - d1);
-          if constexpr (kAlibi) alibi_apply(s, cb, i, j0);
-          if (!pat.block_full(i0, i1, jt * kTile, jt * kTile + kTile)) {
+        int n_out = 0;
 #pragma unroll
-            for (int cc = 0; cc < kCols; ++cc)
-              if (!pat.active(i, j0 + cc)) s[cc] = -INFINITY;
-          }
-          // A = u^{1/(alpha-1)} in fp16 pairs.
-          uint32_t aw[kCols / 2];
-#pragma unroll
-          for (int cc = 0; cc < kCols / 2; ++cc) {
-            const float2 u = __ffma2_rn(make_float2(s[2 * cc], s[2 * cc + 1]), make_float2(cz, cz),
-                                        make_float2(-tau, -tau));
-            const float v0 = fmaxf(u.x, 0.f), v1 = fmaxf(u.y, 0.f);
-            if constexpr (AK == kAlpha15) {
-              const float2 a = __fmul2_rn(make_float2(v0, v1), make_float2(v0, v1));
-              aw[cc] = pack_f16(a.x, a.y);
-            } else if constexpr (AK == kAlpha2) {
-              aw[cc] = pack_f16(v0, v1);
-            } else {
-              aw[cc] = pack_f16(v0 > 0.f ? pow_pos(v0, p.ae) : 0.f, v1 > 0.f ? pow_pos(v1, p.ae) : 0.f);
-            }
-          }
-          // This part's keys qp*kCols.. go back into its own S columns [qp*kCols, +kCols/2):
-          // writing only into columns this thread has read keeps the row's other parts from
-          // seeing overwritten S values.
-          const uint32_t col = pa + qp * kCols;
-          DIAG(const long long d3 = clock64(); dgr[7] += d3 - d2);
-#pragma unroll
-          for (int h = 0; h < kCols / 32; ++h) tmem_st16(tl + col + 16 * h, *reinterpret_cast<uint32_t(*)[16]>(&aw[16 * h]));
-          tmem_wait_st();
-          tc_fence_before();
-          warp_arrive(&sh.o_ready[c]);
-          DIAG(dgr[8] += clock64() - d3);
-          ++k;
-          ++n_s;
-        });
-        const int n_out = k;
+        for (int w = 0; w < kMaskWords; ++w) n_out += __popc(list[w]);
         DIAG(const long long de0 = clock64());
-        // Epilogue: O from TMEM (each thread of a row writes kOCols of the 64 columns).
-        if (n_out > 0) warp_wait(&sh.pv_done[(n_out - 1) % kOBufs], ((n_out - 1) / kOBufs) & 1, wc);
+        if (!o_final) {
+          // Phase 4: output pass at the final tau over the flagged tiles.
+          int k = 0;
+          for_each_bit(list, kMaskWords, [&](int jt) { out_tile(jt, obase + k++, false); });
+          if (k > 0) warp_wait(&sh.pv_done[(obase + k - 1) % kOBufs], ((obase + k - 1) / kOBufs) & 1, wc);
+          obase += k;
+        }
         DIAG(const long long de1 = clock64(); dgx[4] += de1 - de0);
+        // Epilogue: O from TMEM (each thread of a row writes kOCols of the 64 columns).
         tc_fence_after();
         uint32_t o[kOCols];
         ldw(tl + 256 + qp * kOCols, o);
@@ -818,6 +879,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         if (qp == 0) {
           part[3 * kTile + row] = tau;
           part[7 * kTile + row] = (valid && listed) ? 1.f : 0.f;
+          part[11 * kTile + row] = tau_T;
           if (valid) p.tau[(size_t)bh * p.L + i] = tau;
         }
         named_bar(3, kMathThreads);
@@ -831,7 +893,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
               const size_t rix = (size_t)bh * p.L + ir;
               if (part[7 * kTile + r] != 0.f) {
                 const float tr = part[3 * kTile + r];
+                const float tT = part[11 * kTile + r];
                 float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                float aco[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // O correction (o_final)
                 float sgv = 0.f;
                 int pe[kParts + 1];
                 pe[0] = 0;
@@ -839,7 +903,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
                 for (int q = 0; q < kParts; ++q) pe[q + 1] = pe[q] + (int)part[(q * 4 + 2) * kTile + r];
                 const int ntot = pe[kParts];
                 for (int k0 = 0; k0 < ntot; k0 += 4) {   // four V rows in flight
-                  float gk[4];
+                  float gk[4], ck[4];
                   uint4 vw[4];
 #pragma unroll
                   for (int t = 0; t < 4; ++t) {
@@ -849,6 +913,15 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
                     const float u = fmaf(cand[e], cz, -tr);
                     const float gu = AK == kAlpha15 ? u : (AK == kAlpha2 ? 1.f : pow_pos(fmaxf(u, 1e-30f), p.ae - 1.f));
                     gk[t] = (k0 + t < ntot && u > 0.f) ? gu : 0.f;
+                    if constexpr (AK != kAlphaGen) {
+                      // A* at the final tau minus the fp16 A_T the fused pass multiplied.
+                      const float uT = fmaf(cand[e], cz, -tT);
+                      const float aT = round_f16(AK == kAlpha15 ? uT * uT : uT);
+                      const float as = u > 0.f ? (AK == kAlpha15 ? u * u : u) : 0.f;
+                      ck[t] = (o_final && k0 + t < ntot) ? as - aT : 0.f;
+                    } else {
+                      ck[t] = 0.f;
+                    }
                     vw[t] = vbase[(size_t)cidx[e] * (kD / 8)];
                   }
 #pragma unroll
@@ -857,8 +930,11 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
                     const uint32_t w4[4] = {vw[t].x, vw[t].y, vw[t].z, vw[t].w};
 #pragma unroll
                     for (int c2 = 0; c2 < 4; ++c2) {   // bf16 pair -> two floats: shifts, exact
-                      acc[2 * c2] = fmaf(gk[t], __uint_as_float(w4[c2] << 16), acc[2 * c2]);
-                      acc[2 * c2 + 1] = fmaf(gk[t], __uint_as_float(w4[c2] & 0xffff0000u), acc[2 * c2 + 1]);
+                      const float va = __uint_as_float(w4[c2] << 16), vb = __uint_as_float(w4[c2] & 0xffff0000u);
+                      acc[2 * c2] = fmaf(gk[t], va, acc[2 * c2]);
+                      acc[2 * c2 + 1] = fmaf(gk[t], vb, acc[2 * c2 + 1]);
+                      aco[2 * c2] = fmaf(ck[t], va, aco[2 * c2]);
+                      aco[2 * c2 + 1] = fmaf(ck[t], vb, aco[2 * c2 + 1]);
                     }
                   }
                 }
@@ -866,6 +942,14 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
                 dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
                 dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
                 if (sub == 0) p.sumg[rix] = sgv;
+                if (o_final) {   // O = O_T + the correction (this row's O_T was written above)
+                  float4* po = reinterpret_cast<float4*>(p.O + rix * kD + 8 * sub);
+                  float4 x0 = po[0], x1 = po[1];
+                  x0.x += aco[0]; x0.y += aco[1]; x0.z += aco[2]; x0.w += aco[3];
+                  x1.x += aco[4]; x1.y += aco[5]; x1.z += aco[6]; x1.w += aco[7];
+                  po[0] = x0;
+                  po[1] = x1;
+                }
               } else if (sub == 0) {
                 p.sumg[rix] = -1.f;
               }
@@ -878,7 +962,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           for (int w = 0; w < kMaskWords; ++w) na += __popc(act[w]);
           const long long clk3 = clock64();
           int4* st = reinterpret_cast<int4*>(p.stats + ((size_t)bh * p.Tr + qt) * kFwdStats);
-          st[0] = make_int4(sweeps, (int)n_s, n_out, na);
+          st[0] = make_int4(sweeps - fused_passes, (int)n_s, n_out, na);
           st[1] = make_int4((int)(clk1 - clk0), (int)(clk2 - clk1), (int)(clk3 - clk2), (int)(clk3 - clk0));
           DIAG(st[2] = make_int4((int)dg_s1, (int)dg_s2, (int)dg_s3, (int)dg_sw1));
           DIAG(st[4] = make_int4((int)dgr[0], (int)dgr[1], (int)dgr[2], (int)dgr[3]));
@@ -901,11 +985,19 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       const bool collect = !done;
       float S1 = 0.f, S2 = 0.f;
       if (collect) nc = 0;
-      float* mycand = cand + qp * cap * kTile + row;
-      uint16_t* myidx = cidx + qp * cap * kTile + row;
       sbuf = 0;
       DIAG(const long long dsw0 = clock64());
-      for_each_bit(list, kMaskWords, [&](int jt) {
+      if (fuse) {
+        // The fused first pass: output pass at tau_T with candidate collection.
+        clk2 = clock64();
+        tau_T = tau;
+        int k = 0;
+        for_each_bit(list, kMaskWords, [&](int jt) { out_tile(jt, obase + k++, true); });
+        // O of the last tile done: the epilogue reads O, and a later sweep reuses its columns.
+        if (k > 0) warp_wait(&sh.pv_done[(obase + k - 1) % kOBufs], ((obase + k - 1) / kOBufs) & 1, wc);
+        obase += k;
+        ++fused_passes;
+      } else for_each_bit(list, kMaskWords, [&](int jt) {
         const uint32_t bf = sbuf;
         DIAG(const long long d0 = clock64());
         warp_wait(&sh.s_full[bf], (sfull_par >> bf) & 1, wc);
@@ -926,20 +1018,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
             if (!pat.active(i, j0 + cc)) s[cc] = -INFINITY;
         }
         if (cand_only) {
-          // Maxima of the four 8-key groups (independent trees), then an element scan of
-          // only the groups whose maximum passes tau.
-          float gm[kCols / 8];
-#pragma unroll
-          for (int g = 0; g < kCols / 8; ++g) {
-            const float* x = s + 8 * g;
-            gm[g] = fmaxf(fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3])), fmaxf(fmaxf(x[4], x[5]), fmaxf(x[6], x[7])));
-          }
-          // Groups are scanned when any lane of the warp has a candidate in them (a
-          // warp-uniform branch), each lane then runs the same branch-free append.
-#pragma unroll
-          for (int g = 0; g < kCols / 8; ++g)
-            if (__any_sync(0xffffffffu, collect && fmaf(gm[g], cz, -tau) > 0.f))
-              if (collect) collect8(s + 8 * g, j0 + 8 * g, cz, tau, cap, mycand, myidx, nc);
+          collect_tile(s, j0, collect);
           ++n_s;
           sbuf = (sbuf + 1) & (kSBufs - 1);
           DIAG(dgr[5] += clock64() - dtk);

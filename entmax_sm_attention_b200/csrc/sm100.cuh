@@ -306,6 +306,15 @@ __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
   return r;
 }
 
+// x rounded to fp16 (round to nearest even, as pack_f16 rounds) and widened back to fp32.
+__device__ __forceinline__ float round_f16(float x) {
+  unsigned short h;
+  float r;
+  asm("cvt.rn.f16.f32 %0, %1;" : "=h"(h) : "f"(x));
+  asm("cvt.f32.f16 %0, %1;" : "=f"(r) : "h"(h));
+  return r;
+}
+
 // Two-term bf16 split of a pair of floats: x = hi + lo + O(2^-17 |x|), where
 // hi = bf16(x) and lo = bf16(x - hi). Feeding both terms to the tensor cores gives
 // products accurate to about fp32 level.
