@@ -319,6 +319,58 @@ __device__ bool solve_list(const float* vals, const int (&n)[kParts], int list_s
   return false;
 }
 
+// The same solve with one row's work spread over the four lanes of a quad (lanes 4r..4r+3
+// of a warp): each lane sums its own list (list[k*stride], k < n) and two butterfly
+// shuffles combine the sums, so all four lanes take the same steps. Every lane of the warp
+// runs the loop until all of its rows have finished; a lane whose row needs no solve passes
+// active = false. Returns true (and the root in t_out) for a row solved exactly.
+template <int AK>
+__device__ bool solve_quad(const float* list, int n, int stride, bool active, float cz, float e, float t, float lo,
+                           float hi, float& t_out) {
+  constexpr int kIters = AK == kAlphaGen ? 96 : 48;
+  bool fin = !active, ok = false;
+  t_out = t;
+  for (int it = 0; it < kIters && !__all_sync(0xffffffffu, fin); ++it) {
+    float S1 = 0.f, S2 = 0.f, C = 0.f, umin = INFINITY;
+    sum_list<AK>(list, n, stride, cz, t, e, S1, S2, C, umin);
+#pragma unroll
+    for (int m = 1; m <= 2; m <<= 1) {
+      S1 += __shfl_xor_sync(0xffffffffu, S1, m);
+      S2 += __shfl_xor_sync(0xffffffffu, S2, m);
+      C += __shfl_xor_sync(0xffffffffu, C, m);
+      umin = fminf(umin, __shfl_xor_sync(0xffffffffu, umin, m));
+    }
+    if (fin) continue;
+    float f, fp;   // f(t) and |f'(t)|
+    root_terms<AK>(S1, S2, C, e, f, fp);
+    if (C > 0.f) {
+      const float d = piece_root<AK>(S1, S2, C);
+      if (d >= 0.f && d < umin) {   // no candidate leaves the support at t + d: exact
+        t_out = t + d;
+        ok = fin = true;
+        continue;
+      }
+    }
+    const float tol = AK == kAlphaGen ? fmaxf(4e-6f, C * 0x1p-19f) : 1e-7f;
+    if (fabsf(f) <= tol && fp > 0.f) {
+      t_out = t + f / fp;
+      ok = fin = true;
+      continue;
+    }
+    if (f > 0.f) lo = t; else hi = t;
+    if (AK == kAlphaGen && hi - lo <= fmaxf(fabsf(lo), 1.f) * 0x1p-22f) {
+      t_out = 0.5f * (lo + hi);
+      ok = fin = true;
+      continue;
+    }
+    float tn = t + f / fp;
+    if (!(tn > lo && tn <= hi && tn != t)) tn = 0.5f * (lo + hi);
+    if (AK == kAlphaGen && (it & 3) == 3) tn = 0.5f * (lo + hi);
+    t = tn;
+  }
+  return ok;
+}
+
 // Threshold of Eq. 4 restricted to N raw scores v (some may be -inf), in registers:
 // safeguarded Newton from lo inside [lo, hi], finished by the exact root of the current
 // support's piece once no value leaves the support. A subset of the row's scores has a
@@ -630,6 +682,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     DIAG(long long dg_s1 = 0; long long dg_s2 = 0; long long dg_s3 = 0; long long dg_sw1 = 0);
     DIAG(long long dgr[9] = {0, 0, 0, 0, 0, 0, 0, 0, 0}; long long dtk = 0);
     DIAG(long long dgx[6] = {0, 0, 0, 0, 0, 0});   // [26] tau_T solve, [27] decisions, [28] post-sweep solves, [29] epilogue
+    DIAG(long long dg_solve = 0);                  // [11] the exact solves alone
 
     // Phase 1: per-key-tile row maxima over this thread's column part (combined in smem).
     for_each_bit(act, kMaskWords, [&](int jt) {
@@ -964,7 +1017,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           int4* st = reinterpret_cast<int4*>(p.stats + ((size_t)bh * p.Tr + qt) * kFwdStats);
           st[0] = make_int4(sweeps - fused_passes, (int)n_s, n_out, na);
           st[1] = make_int4((int)(clk1 - clk0), (int)(clk2 - clk1), (int)(clk3 - clk2), (int)(clk3 - clk0));
-          DIAG(st[2] = make_int4((int)dg_s1, (int)dg_s2, (int)dg_s3, (int)dg_sw1));
+          DIAG(st[2] = make_int4((int)dg_s1, (int)dg_s2, (int)dg_s3, (int)dg_solve));
           DIAG(st[4] = make_int4((int)dgr[0], (int)dgr[1], (int)dgr[2], (int)dgr[3]));
           DIAG(st[5] = make_int4((int)dgr[4], (int)dgr[5], (int)dgr[6], (int)dgr[7]));
           DIAG(st[6].x = (int)dgr[8]);
@@ -1091,15 +1144,39 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       const float C = (float)ntot;   // support size at tau (alpha = 2: |f'(tau)|)
       named_bar(3, kMathThreads);   // partials consumed before anyone rewrites them
       ++sweeps;
-      if (!done && cand_only) {
+      DIAG(const long long dsv0 = clock64());
+      if (cand_only) {
         // tau = tau_T <= tau*: if the copies fit they hold the support; solve on them.
-        // Otherwise tau stays and the next sweep measures f(tau) and f'(tau).
-        float t;
-        if (fits && solve_list<AK>(cand + row, ncs, cap * kTile, kTile, cz, p.ae, tau, lo, hi, t)) {
-          tau = t;
+        // Otherwise tau stays and the next sweep measures f(tau) and f'(tau). The solve
+        // runs with four lanes of one warp per row (solve_quad), eight rows per warp:
+        // the row's tau and bracket go through shared memory and the result comes back.
+        if (qp == 0) {
+          part[3 * kTile + row] = tau;
+          part[7 * kTile + row] = lo;
+          part[11 * kTile + row] = hi;
+          part[15 * kTile + row] = (!done && fits) ? 1.f : 0.f;
+        }
+        named_bar(3, kMathThreads);
+        {
+          const int rq = warp * 8 + (lane >> 2), sub = lane & 3;
+          const bool go = part[15 * kTile + rq] != 0.f;
+          const int nq = (int)part[(sub * 4 + 2) * kTile + rq];
+          float t;
+          const bool ok = solve_quad<AK>(cand + sub * cap * kTile + rq, go ? nq : 0, kTile, go, cz, p.ae,
+                                         part[3 * kTile + rq], part[7 * kTile + rq], part[11 * kTile + rq], t);
+          named_bar(3, kMathThreads);   // every quad has read its row's inputs
+          if (sub == 0) {
+            part[3 * kTile + rq] = t;
+            part[15 * kTile + rq] = ok ? 1.f : 0.f;
+          }
+        }
+        named_bar(3, kMathThreads);
+        if (!done && fits && part[15 * kTile + row] != 0.f) {
+          tau = part[3 * kTile + row];
           done = true;
           listed = true;
         }
+        DIAG(dg_solve += clock64() - dsv0);
       } else if (!done) {
         float f, fp;   // f(tau) and |f'(tau)|
         root_terms<AK>(S1, S2, C, p.ae, f, fp);
