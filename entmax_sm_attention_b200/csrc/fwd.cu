@@ -202,6 +202,27 @@ __device__ __forceinline__ void collect8(const float* s, int j, float cz, float 
   }
 }
 
+// The same append for four scores against a threshold in score units (s > thr).
+__device__ __forceinline__ void collect4(const float* s, int j, float thr, int cap, float* mycand, uint16_t* myidx,
+                                         int& nc) {
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const bool pass = s[e] > thr;
+    const int slot = min(nc, cap - 1);
+    mycand[slot * kTile] = s[e];
+    myidx[slot * kTile] = (uint16_t)(j + e);
+    nc += pass ? 1 : 0;
+  }
+}
+
+// A score threshold below tau / cz (cz > 0): every s with fmaf(s, cz, -tau) > 0, that is
+// s cz > tau exactly, has s > thr. The few extra scores at the boundary (u <= 0) are
+// harmless candidates: every use of the copies tests u > 0.
+__device__ __forceinline__ float cand_threshold(float tau, float cz) {
+  const float q = tau / cz;
+  return q - (fabsf(q) * 0x1p-20f + 1e-30f);
+}
+
 // Adds one candidate at u = z - t to the sums of the current support (u > 0), without
 // a branch: the lanes of a warp follow one path whatever their candidates. S1 and S2 are
 // sum u and sum u^2 (alpha = 1.5, 2); for the run-time variant they are sum g = sum u^{e-1}
@@ -767,28 +788,26 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     float* mycand = cand + qp * cap * kTile + row;
     uint16_t* myidx = cidx + qp * cap * kTile + row;
 
-    // Candidate collection on one tile's scores: the maxima of the four 8-key groups
-    // (independent trees), then an element scan of only the groups whose maximum passes
-    // tau. A group is scanned when any lane of the warp has a candidate in it (a
-    // warp-uniform branch); each lane then runs the same branch-free append.
-    auto collect_tile = [&](const float (&sv)[kCols], int j0, bool collect) {
-      float gm[kCols / 8];
+    // Candidate collection on one tile's scores: the maxima of the eight 4-key groups
+    // (independent pairs), then an append of only the groups whose maximum passes the
+    // threshold thr (cand_threshold). A group is appended when any lane of the warp has a
+    // candidate in it (a warp-uniform branch; 32 rows share the vote, so smaller groups
+    // are scanned less often); each lane then runs the same branch-free append.
+    auto collect_tile = [&](const float (&sv)[kCols], int j0, bool collect, float thr) {
+      float gm[kCols / 4];
 #pragma unroll
-      for (int g = 0; g < kCols / 8; ++g) {
-        const float* x = sv + 8 * g;
-        gm[g] = fmaxf(fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3])), fmaxf(fmaxf(x[4], x[5]), fmaxf(x[6], x[7])));
-      }
+      for (int g = 0; g < kCols / 4; ++g) gm[g] = fmaxf(fmaxf(sv[4 * g], sv[4 * g + 1]), fmaxf(sv[4 * g + 2], sv[4 * g + 3]));
 #pragma unroll
-      for (int g = 0; g < kCols / 8; ++g)
-        if (__any_sync(0xffffffffu, collect && fmaf(gm[g], cz, -tau) > 0.f))
-          if (collect) collect8(sv + 8 * g, j0 + 8 * g, cz, tau, cap, mycand, myidx, nc);
+      for (int g = 0; g < kCols / 4; ++g)
+        if (__any_sync(0xffffffffu, collect && gm[g] > thr))
+          if (collect) collect4(sv + 4 * g, j0 + 4 * g, thr, cap, mycand, myidx, nc);
     };
     // One tile of an output-type pass (output tile ko overall, buffer ko % 3): recompute
     // S, optionally collect this thread's candidates at tau, and write A = u^{1/(alpha-1)}
     // at tau in fp16 over the S columns this thread has read (the part's keys qp*kCols..
     // go into its own columns [qp*kCols, +kCols/2), so the row's other parts never see an
     // overwritten S value).
-    auto out_tile = [&](int jt, uint32_t ko, bool collect) {
+    auto out_tile = [&](int jt, uint32_t ko, bool collect, float thr) {
       const int c = ko % kOBufs;
       const uint32_t pa = OL::sbuf(c);
       DIAG(const long long d0 = clock64());
@@ -805,7 +824,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         for (int cc = 0; cc < kCols; ++cc)
           if (!pat.active(i, j0 + cc)) s[cc] = -INFINITY;
       }
-      if (collect) collect_tile(s, j0, !done);   // collect is warp-uniform
+      if (collect) collect_tile(s, j0, !done, thr);   // collect is warp-uniform
       uint32_t aw[kCols / 2];
 #pragma unroll
       for (int cc = 0; cc < kCols / 2; ++cc) {
@@ -904,7 +923,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         if (!o_final) {
           // Phase 4: output pass at the final tau over the flagged tiles.
           int k = 0;
-          for_each_bit(list, kMaskWords, [&](int jt) { out_tile(jt, obase + k++, false); });
+          for_each_bit(list, kMaskWords, [&](int jt) { out_tile(jt, obase + k++, false, 0.f); });
           if (k > 0) warp_wait(&sh.pv_done[(obase + k - 1) % kOBufs], ((obase + k - 1) / kOBufs) & 1, wc);
           obase += k;
         }
@@ -969,7 +988,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
                     if constexpr (AK != kAlphaGen) {
                       // A* at the final tau minus the fp16 A_T the fused pass multiplied.
                       const float uT = fmaf(cand[e], cz, -tT);
-                      const float aT = round_f16(AK == kAlpha15 ? uT * uT : uT);
+                      const float aT = uT > 0.f ? round_f16(AK == kAlpha15 ? uT * uT : uT) : 0.f;
                       const float as = u > 0.f ? (AK == kAlpha15 ? u * u : u) : 0.f;
                       ck[t] = (o_final && k0 + t < ntot) ? as - aT : 0.f;
                     } else {
@@ -1039,13 +1058,15 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       float S1 = 0.f, S2 = 0.f;
       if (collect) nc = 0;
       sbuf = 0;
+      const float cthr = cand_threshold(tau, cz);   // the candidate-only sweep's threshold
       DIAG(const long long dsw0 = clock64());
       if (fuse) {
         // The fused first pass: output pass at tau_T with candidate collection.
         clk2 = clock64();
         tau_T = tau;
         int k = 0;
-        for_each_bit(list, kMaskWords, [&](int jt) { out_tile(jt, obase + k++, true); });
+        const float thr = cand_threshold(tau, cz);
+        for_each_bit(list, kMaskWords, [&](int jt) { out_tile(jt, obase + k++, true, thr); });
         // O of the last tile done: the epilogue reads O, and a later sweep reuses its columns.
         if (k > 0) warp_wait(&sh.pv_done[(obase + k - 1) % kOBufs], ((obase + k - 1) / kOBufs) & 1, wc);
         obase += k;
@@ -1071,7 +1092,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
             if (!pat.active(i, j0 + cc)) s[cc] = -INFINITY;
         }
         if (cand_only) {
-          collect_tile(s, j0, collect);
+          collect_tile(s, j0, collect, cthr);
           ++n_s;
           sbuf = (sbuf + 1) & (kSBufs - 1);
           DIAG(dgr[5] += clock64() - dtk);
