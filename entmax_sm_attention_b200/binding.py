@@ -222,7 +222,8 @@ def block_mask(ctx):
 def bwd_counters(ctx):
     """int32 [B, H, Tc, 8] counters of the last backward per key tile: flagged query tiles
     visited, total cycles, and the first row-owner warp's cycles waiting for S/dA, waiting
-    for the previous tile's MMAs, forming A/dS, staging dQ (then two zeros)."""
+    for the previous tile's MMAs, forming A/dS, staging dQ, and the part of forming spent
+    loading S and dA from tensor memory (then a zero)."""
     desc, ws = ctx
     st = torch.empty(mask_shape(desc)[:3] + (BWD_STATS,), dtype=torch.int32, device=ws.device)
     entmax_attn_block_mask(desc, ws, None, None, st)

@@ -230,7 +230,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     const float cb = kAlibi ? p.alibi[bh % p.H] / p.scale : 0.f;   // ALiBi, raw score units
     uint32_t seq = 0;
     int prev_it = -1;
-    long long cyc_s = 0, cyc_mma = 0, cyc_form = 0, cyc_flush = 0;   // first row-owner warp's breakdown
+    long long cyc_s = 0, cyc_mma = 0, cyc_form = 0, cyc_flush = 0, cyc_ld = 0;   // first row-owner warp's breakdown
     // Adds dQ of the query tile `it` handled at step `s` (TMEM buffer s % 2) to global
     // memory. The caller has already waited for that step's MMAs. Each thread stages its
     // 16 columns (scaled) in the swizzled box that holds them (one box per 32 of dQ's 64
@@ -271,61 +271,74 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       warp_wait(&sh.s_full, seq & 1, wc);
       const long long c1 = clock64();
       tc_fence_after();
-      uint32_t sr[32], ar[32];
-      tmem_ld32(tl + qc * 32, sr);
-      tmem_ld32(tl + 128 + qc * 32, ar);
+      // S and dA are read in two halves of 16 columns, so only 32 of them are live at a
+      // time; the second half's read releases the TMEM columns (sda_free) for the next tile.
+      uint32_t sr[16], ar[16];
+      tmem_ld16(tl + qc * 32, sr);
+      tmem_ld16(tl + 128 + qc * 32, ar);
       tmem_wait_ld();
-      tc_fence_before();
-      warp_arrive(&sh.sda_free);
+      const long long c1b = clock64();
       // The previous tile's dV/dK/dQ MMAs must be done reading sA / sdS.
       const long long c2 = clock64();
       if (seq > 0) warp_wait(&sh.mma2_done, (seq - 1) & 1, wc);
       const long long c3 = clock64();
       // Keys [32 qc, 32 qc + 32) of row `row`: panel qc/2, 16-byte chunks 4(qc%2)..+3.
       const int pan = (qc >> 1) * kTileBytes;
+      auto form_half = [&](int hf) {
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t ah[4], dh[4], dl2[4];
+        for (int ch = 0; ch < 2; ++ch) {
+          const int cc = 2 * hf + ch;
+          uint32_t ah[4], dh[4], dl2[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int c = cc * 8 + 2 * e;
-          float s0 = __uint_as_float(sr[c]), s1 = __uint_as_float(sr[c + 1]);
-          if constexpr (kAlibi) {   // ALiBi: -cb |i - j| on the raw scores
-            const float dj = (float)(i - (j0 + qc * 32 + c));
-            s0 = fmaf(-cb, fabsf(dj), s0);
-            s1 = fmaf(-cb, fabsf(dj - 1.f), s1);
+          for (int e = 0; e < 4; ++e) {
+            const int c = ch * 8 + 2 * e;         // column within the half
+            const int cq = hf * 16 + c;           // column within the thread's 32 keys
+            float s0 = __uint_as_float(sr[c]), s1 = __uint_as_float(sr[c + 1]);
+            if constexpr (kAlibi) {   // ALiBi: -cb |i - j| on the raw scores
+              const float dj = (float)(i - (j0 + qc * 32 + cq));
+              s0 = fmaf(-cb, fabsf(dj), s0);
+              s1 = fmaf(-cb, fabsf(dj - 1.f), s1);
+            }
+            if (!full) {
+              const int jj = j0 + qc * 32 + cq;
+              if (!pat.active(i, jj)) s0 = -INFINITY;
+              if (!pat.active(i, jj + 1)) s1 = -INFINITY;
+            }
+            const float2 u = __ffma2_rn(make_float2(s0, s1), make_float2(cz, cz), make_float2(-tau, -tau));
+            const float v0 = fmaxf(u.x, 0.f), v1 = fmaxf(u.y, 0.f);
+            const float2 d = __fadd2_rn(make_float2(__uint_as_float(ar[c]), __uint_as_float(ar[c + 1])),
+                                        make_float2(-dl, -dl));
+            if constexpr (AK == kAlpha15) {
+              const float2 a = __fmul2_rn(make_float2(v0, v1), make_float2(v0, v1));
+              const float2 ds = __fmul2_rn(make_float2(v0, v1), d);
+              ah[e] = pack_f16(a.x, a.y);
+              split_bf16x2(ds.x, ds.y, dh[e], dl2[e]);
+            } else if constexpr (AK == kAlpha2) {
+              ah[e] = pack_f16(v0, v1);
+              split_bf16x2(u.x > 0.f ? d.x : 0.f, u.y > 0.f ? d.y : 0.f, dh[e], dl2[e]);
+            } else {
+              // A = u^e and g = u^{e-1} from one logarithm each.
+              const float l0 = __log2f(u.x > 0.f ? u.x : 1.f), l1 = __log2f(u.y > 0.f ? u.y : 1.f);
+              const float a0 = u.x > 0.f ? exp2f(p.ae * l0) : 0.f, a1 = u.y > 0.f ? exp2f(p.ae * l1) : 0.f;
+              const float g0 = u.x > 0.f ? exp2f((p.ae - 1.f) * l0) : 0.f;
+              const float g1 = u.y > 0.f ? exp2f((p.ae - 1.f) * l1) : 0.f;
+              ah[e] = pack_f16(a0, a1);
+              split_bf16x2(g0 * d.x, g1 * d.y, dh[e], dl2[e]);
+            }
           }
-          if (!full) {
-            const int jj = j0 + qc * 32 + c;
-            if (!pat.active(i, jj)) s0 = -INFINITY;
-            if (!pat.active(i, jj + 1)) s1 = -INFINITY;
-          }
-          const float2 u = __ffma2_rn(make_float2(s0, s1), make_float2(cz, cz), make_float2(-tau, -tau));
-          const float v0 = fmaxf(u.x, 0.f), v1 = fmaxf(u.y, 0.f);
-          const float d0 = __uint_as_float(ar[c]) - dl, d1 = __uint_as_float(ar[c + 1]) - dl;
-          if constexpr (AK == kAlpha15) {
-            const float2 a = __fmul2_rn(make_float2(v0, v1), make_float2(v0, v1));
-            const float2 ds = __fmul2_rn(make_float2(v0, v1), make_float2(d0, d1));
-            ah[e] = pack_f16(a.x, a.y);
-            split_bf16x2(ds.x, ds.y, dh[e], dl2[e]);
-          } else if constexpr (AK == kAlpha2) {
-            ah[e] = pack_f16(v0, v1);
-            split_bf16x2(u.x > 0.f ? d0 : 0.f, u.y > 0.f ? d1 : 0.f, dh[e], dl2[e]);
-          } else {
-            // A = u^e and g = u^{e-1} from one logarithm each.
-            const float l0 = __log2f(u.x > 0.f ? u.x : 1.f), l1 = __log2f(u.y > 0.f ? u.y : 1.f);
-            const float a0 = u.x > 0.f ? exp2f(p.ae * l0) : 0.f, a1 = u.y > 0.f ? exp2f(p.ae * l1) : 0.f;
-            const float g0 = u.x > 0.f ? exp2f((p.ae - 1.f) * l0) : 0.f;
-            const float g1 = u.y > 0.f ? exp2f((p.ae - 1.f) * l1) : 0.f;
-            ah[e] = pack_f16(a0, a1);
-            split_bf16x2(g0 * d0, g1 * d1, dh[e], dl2[e]);
-          }
+          const uint32_t off = pan + sw128_offset(row, ((qc & 1) * 4 + cc) * 8);
+          *reinterpret_cast<uint4*>(sA + off) = make_uint4(ah[0], ah[1], ah[2], ah[3]);
+          *reinterpret_cast<uint4*>(sdS + off) = make_uint4(dh[0], dh[1], dh[2], dh[3]);
+          *reinterpret_cast<uint4*>(sdSl + off) = make_uint4(dl2[0], dl2[1], dl2[2], dl2[3]);
         }
-        const uint32_t off = pan + sw128_offset(row, ((qc & 1) * 4 + cc) * 8);
-        *reinterpret_cast<uint4*>(sA + off) = make_uint4(ah[0], ah[1], ah[2], ah[3]);
-        *reinterpret_cast<uint4*>(sdS + off) = make_uint4(dh[0], dh[1], dh[2], dh[3]);
-        *reinterpret_cast<uint4*>(sdSl + off) = make_uint4(dl2[0], dl2[1], dl2[2], dl2[3]);
-      }
+      };
+      form_half(0);
+      tmem_ld16(tl + qc * 32 + 16, sr);
+      tmem_ld16(tl + 128 + qc * 32 + 16, ar);
+      tmem_wait_ld();
+      tc_fence_before();
+      warp_arrive(&sh.sda_free);
+      form_half(1);
       fence_proxy_async_smem();
       warp_arrive(&sh.p_ready);
       const long long c4 = clock64();
@@ -334,6 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       cyc_s += c1 - c0;
       cyc_mma += c3 - c2;
       cyc_form += (c2 - c1) + (c4 - c3);
+      cyc_ld += c1b - c1;
       cyc_flush += c5 - c4;
       prev_it = it;
       ++seq;
@@ -378,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     if (tid == 0) {
       int4* st = reinterpret_cast<int4*>(p.stats + ((size_t)bh * p.Tc + kt) * kBwdStats);
       st[0] = make_int4(nq, (int)(clock64() - clk0), (int)cyc_s, (int)cyc_mma);
-      st[1] = make_int4((int)cyc_form, (int)cyc_flush, 0, 0);
+      st[1] = make_int4((int)cyc_form, (int)cyc_flush, (int)cyc_ld, 0);
     }
     __syncwarp();
   }

@@ -19,7 +19,8 @@ constexpr int kFwdStats = 8;
 #endif
 // Per-key-tile counters of the backward kernel: 0 flagged query tiles visited, then cycles
 // of 1 the whole CTA, and, for the first row-owner warp, 2 waiting for S and dA, 3 waiting
-// for the previous tile's gradient MMAs, 4 forming A and dS, 5 staging dQ (reduce-add).
+// for the previous tile's gradient MMAs, 4 forming A and dS, 5 staging dQ (reduce-add),
+// 6 the part of 4 spent loading S and dA from tensor memory.
 constexpr int kBwdStats = 8;
 // Self-test switch: every CTA makes one bounded wait on an mbarrier that nothing
 // completes, so the wait expires and the abort path runs.

@@ -321,7 +321,8 @@ __device__ __forceinline__ float round_f16(float x) {
 __device__ __forceinline__ void split_bf16x2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
   hi = pack_bf16(x0, x1);
   const float h0 = __uint_as_float(hi << 16), h1 = __uint_as_float(hi & 0xffff0000u);
-  lo = pack_bf16(x0 - h0, x1 - h1);
+  const float2 r = __fadd2_rn(make_float2(x0, x1), make_float2(-h0, -h1));
+  lo = pack_bf16(r.x, r.y);
 }
 
 // Byte offset of element (row, col) in a [rows][64] bf16 tile stored with the 128-byte
