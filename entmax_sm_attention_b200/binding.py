@@ -23,7 +23,8 @@ ENTMAX_BF16, ENTMAX_FP32 = 0, 1
 ENTMAX_MAX_L = 16384
 ENTMAX_TILE = 128
 EXPORTS = ("entmax_attn_workspace_bytes", "entmax_attn_fwd", "entmax_attn_bwd", "entmax_rows",
-           "entmax_last_device_status", "entmax_attn_block_mask", "entmax_attn_fwd_noalloc")
+           "entmax_last_device_status", "entmax_attn_block_mask", "entmax_attn_block_mask64",
+           "entmax_attn_fwd_noalloc")
 ENTMAX_NOALLOC_SCRATCH_BYTES = 16 << 20
 ENTMAX_SELFTEST_STALL = 1
 FWD_STATS = 8     # int32 counters per query tile (forward)
@@ -44,6 +45,7 @@ class AttnDesc(ctypes.Structure):
         ("causal", ctypes.c_int), ("window", ctypes.c_int),
         ("kv_len", ctypes.c_void_p), ("dtype", ctypes.c_int), ("max_sweeps", ctypes.c_int),
         ("wait_limit_us", ctypes.c_int), ("alibi_slopes", ctypes.c_void_p), ("selftest", ctypes.c_int),
+        ("mask64", ctypes.c_int),
     ]
 
 
@@ -72,6 +74,8 @@ def load_library(path: str = LIB_PATH):
     lib.entmax_last_device_status.restype = i
     lib.entmax_attn_block_mask.argtypes = [dp, vp, vp, vp, vp, vp]
     lib.entmax_attn_block_mask.restype = i
+    lib.entmax_attn_block_mask64.argtypes = [dp, vp, vp, vp]
+    lib.entmax_attn_block_mask64.restype = i
     lib.entmax_attn_fwd_noalloc.argtypes = [dp, vp, vp, vp, vp, vp, vp]
     lib.entmax_attn_fwd_noalloc.restype = i
     _lib = lib
@@ -116,7 +120,7 @@ class Options:
 def make_desc(B: int, H: int, L: int, d: int = 64, *, alpha: float = 1.5, scale: float | None = None,
               causal: bool = False, window: int = -1, kv_len: torch.Tensor | None = None,
               dtype: int = ENTMAX_BF16, max_sweeps: int = 0, wait_limit_us: int = 0,
-              alibi: torch.Tensor | None = None, selftest: int = 0) -> AttnDesc:
+              alibi: torch.Tensor | None = None, selftest: int = 0, mask64: bool = False) -> AttnDesc:
     """Fill an entmax_attn_desc. kv_len, if given, is a device int32 tensor [B]; alibi, if
     given, a device float32 tensor [H] of ALiBi slopes."""
     if kv_len is not None and (kv_len.dtype != torch.int32 or not kv_len.is_cuda):
@@ -125,7 +129,7 @@ def make_desc(B: int, H: int, L: int, d: int = 64, *, alpha: float = 1.5, scale:
         raise ValueError("alibi must be a CUDA float32 tensor of H slopes")
     return AttnDesc(B, H, L, d, float(alpha), float(scale if scale is not None else d ** -0.5),
                     int(bool(causal) or window >= 0), int(window), _ptr(kv_len), int(dtype), int(max_sweeps),
-                    int(wait_limit_us), _ptr(alibi), int(selftest))
+                    int(wait_limit_us), _ptr(alibi), int(selftest), int(bool(mask64)))
 
 
 def entmax_attn_workspace_bytes(desc: AttnDesc) -> int:
@@ -163,6 +167,11 @@ def entmax_attn_block_mask(desc: AttnDesc, workspace, M=None, stats=None, bwd_st
         ctypes.byref(desc), _ptr(workspace), _ptr(M), _ptr(stats), _ptr(bwd_stats), _stream(stream)))
 
 
+def entmax_attn_block_mask64(desc: AttnDesc, workspace, M64, stream=None) -> int:
+    return _check("entmax_attn_block_mask64", load_library().entmax_attn_block_mask64(
+        ctypes.byref(desc), _ptr(workspace), _ptr(M64), _stream(stream)))
+
+
 def entmax_attn_fwd_noalloc(desc: AttnDesc, Q, K, V, O, tau, stream=None) -> int:
     """Forward for callers that cannot allocate: the library's fixed per-GPU scratch
     replaces the workspace (see include/entmax_attn.h for the size limit and the rule
@@ -184,15 +193,20 @@ def mask_shape(desc: AttnDesc) -> tuple:
     return (desc.B, desc.H, T, -(-T // 32))
 
 
+def mask64_shape(desc: AttnDesc) -> tuple:
+    T = -(-desc.L // ENTMAX_TILE)
+    return (desc.B, desc.H, 2 * T, -(-2 * T // 32))
+
+
 def forward(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, *, alpha: float = 1.5, scale=None,
             causal: bool = False, window: int = -1, kv_len=None, max_sweeps: int = 0, wait_limit_us: int = 0,
-            alibi=None, selftest: int = 0):
+            alibi=None, selftest: int = 0, mask64: bool = False):
     """O, tau and the (desc, workspace) context of one forward call on [B, H, L, 64] tensors."""
     B, H, L, d = Q.shape
     dtype = ENTMAX_BF16 if Q.dtype == torch.bfloat16 else ENTMAX_FP32
     desc = make_desc(B, H, L, d, alpha=alpha, scale=scale, causal=causal, window=window, kv_len=kv_len,
                      dtype=dtype, max_sweeps=max_sweeps, wait_limit_us=wait_limit_us, alibi=alibi,
-                     selftest=selftest)
+                     selftest=selftest, mask64=mask64)
     ws = alloc_workspace(desc, Q.device)
     O = torch.empty((B, H, L, d), dtype=torch.float32, device=Q.device)
     tau = torch.empty((B, H, L), dtype=torch.float32, device=Q.device)
@@ -217,6 +231,14 @@ def block_mask(ctx):
     st = torch.empty(mask_shape(desc)[:3] + (FWD_STATS,), dtype=torch.int32, device=ws.device)
     entmax_attn_block_mask(desc, ws, Mv, st)
     return Mv, st
+
+
+def block_mask64(ctx):
+    """The forward's mask at 64 x 64 blocks as int32 bit patterns [B, H, 2 Tr, ceil(2 Tc/32)]."""
+    desc, ws = ctx
+    M64 = torch.empty(mask64_shape(desc), dtype=torch.int32, device=ws.device)
+    entmax_attn_block_mask64(desc, ws, M64)
+    return M64
 
 
 def bwd_counters(ctx):

@@ -24,10 +24,10 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 // Workspace layout. Everything the forward writes comes first (up to fwd_total); the
 // backward-only parts follow.
 struct Layout {
-  int BH, Tr, Tc, Wc, Wr;
-  size_t off_status, off_M, off_MT, off_sumg, off_Ot, off_stats, off_v16, fwd_total;
+  int BH, Tr, Tc, Wc, Wr, W64c, W64r;
+  size_t off_status, off_M, off_MT, off_M64T, off_M64, off_sumg, off_Ot, off_stats, off_v16, fwd_total;
   size_t off_delta, off_bstats, off_do16, total;
-  size_t bytes_M, bytes_MT, bytes_stats, bytes_bstats;
+  size_t bytes_M, bytes_MT, bytes_M64T, bytes_M64, bytes_stats, bytes_bstats;
 };
 
 bool layout_of(const entmax_attn_desc* d, Layout* l) {
@@ -36,6 +36,8 @@ bool layout_of(const entmax_attn_desc* d, Layout* l) {
   l->Tc = l->Tr;
   l->Wc = (l->Tc + 31) / 32;
   l->Wr = (l->Tr + 31) / 32;
+  l->W64c = (2 * l->Tc + 31) / 32;
+  l->W64r = (2 * l->Tr + 31) / 32;
   const size_t rows = (size_t)l->BH * d->L;
   size_t off = 0;
   l->off_status = off;
@@ -55,6 +57,12 @@ bool layout_of(const entmax_attn_desc* d, Layout* l) {
   off += align256(l->bytes_stats);
   l->off_v16 = off;
   off += align256(rows * kD * 2);
+  l->off_M64T = off;
+  l->bytes_M64T = (size_t)l->BH * 2 * l->Tc * l->W64r * 4;
+  off += align256(l->bytes_M64T);
+  l->off_M64 = off;
+  l->bytes_M64 = (size_t)l->BH * 2 * l->Tr * l->W64c * 4;
+  off += align256(l->bytes_M64);
   l->fwd_total = off;
   l->off_delta = off;
   off += align256(rows * 4);
@@ -77,6 +85,7 @@ entmax_status check_desc(const entmax_attn_desc* d) {
   if (d->dtype != ENTMAX_BF16 && d->dtype != ENTMAX_FP32) return ENTMAX_EINVAL;
   if (d->wait_limit_us < 0) return ENTMAX_EINVAL;
   if (d->selftest != 0 && d->selftest != ENTMAX_SELFTEST_STALL) return ENTMAX_EINVAL;
+  if (d->mask64 != 0 && d->mask64 != 1) return ENTMAX_EINVAL;
   if (d->d != kD) return ENTMAX_EUNSUPPORTED;
   if (d->L > ENTMAX_MAX_L) return ENTMAX_EUNSUPPORTED;
   if (!(d->alpha > 1.0f) || !std::isfinite(d->alpha)) return ENTMAX_EINVAL;
@@ -166,6 +175,7 @@ extern "C" entmax_status entmax_attn_fwd(const entmax_attn_desc* d, const void* 
   uint8_t* w = static_cast<uint8_t*>(ws);
   if (cudaMemsetAsync(w + l.off_status, 0, 256, s) != cudaSuccess) return ENTMAX_ECUDA;
   if (cudaMemsetAsync(w + l.off_MT, 0, l.bytes_MT, s) != cudaSuccess) return ENTMAX_ECUDA;
+  if (d->mask64 && cudaMemsetAsync(w + l.off_M64T, 0, l.bytes_M64T, s) != cudaSuccess) return ENTMAX_ECUDA;
   if (d->dtype == ENTMAX_FP32) {
     FwdF32Params q;
     std::memset(&q, 0, sizeof(q));
@@ -176,6 +186,10 @@ extern "C" entmax_status entmax_attn_fwd(const entmax_attn_desc* d, const void* 
     q.tau = tau;
     q.M = reinterpret_cast<uint32_t*>(w + l.off_M);
     q.MT = reinterpret_cast<uint32_t*>(w + l.off_MT);
+    q.M64 = d->mask64 ? reinterpret_cast<uint32_t*>(w + l.off_M64) : nullptr;
+    q.M64T = d->mask64 ? reinterpret_cast<uint32_t*>(w + l.off_M64T) : nullptr;
+    q.W64c = l.W64c;
+    q.W64r = l.W64r;
     q.stats = reinterpret_cast<int*>(w + l.off_stats);
     q.status = reinterpret_cast<int*>(w + l.off_status);
     q.kv_len = d->kv_len;
@@ -206,6 +220,10 @@ extern "C" entmax_status entmax_attn_fwd(const entmax_attn_desc* d, const void* 
   p.Vb = static_cast<const uint16_t*>(V);
   p.M = reinterpret_cast<uint32_t*>(w + l.off_M);
   p.MT = reinterpret_cast<uint32_t*>(w + l.off_MT);
+  p.M64 = d->mask64 ? reinterpret_cast<uint32_t*>(w + l.off_M64) : nullptr;   // the 64 x 64 variant
+  p.M64T = d->mask64 ? reinterpret_cast<uint32_t*>(w + l.off_M64T) : nullptr;
+  p.W64c = l.W64c;
+  p.W64r = l.W64r;
   p.stats = reinterpret_cast<int*>(w + l.off_stats);
   p.status = reinterpret_cast<int*>(w + l.off_status);
   p.kv_len = d->kv_len;
@@ -254,6 +272,8 @@ extern "C" entmax_status entmax_attn_bwd(const entmax_attn_desc* d, const void* 
   p.tau = tau;
   p.delta = delta;
   p.MT = reinterpret_cast<const uint32_t*>(w + l.off_MT);
+  p.M64T = d->mask64 ? reinterpret_cast<const uint32_t*>(w + l.off_M64T) : nullptr;
+  p.W64r = l.W64r;
   p.dQ = dQ;
   p.dK = dK;
   p.dV = dV;
@@ -333,6 +353,18 @@ extern "C" entmax_status entmax_last_device_status(const entmax_attn_desc* d, co
   if (word & kStatusTimeout) return ENTMAX_ETIMEOUT;
   if (word & kStatusRange) return ENTMAX_ERANGE;
   if (word & kStatusNoConverge) return ENTMAX_ENOCONVERGE;
+  return ENTMAX_OK;
+}
+
+extern "C" entmax_status entmax_attn_block_mask64(const entmax_attn_desc* d, const void* ws, uint32_t* M64,
+                                                  void* stream) {
+  if (check_desc(d) != ENTMAX_OK || !aligned(ws, 256) || !M64 || !d->mask64) return ENTMAX_EINVAL;
+  Layout l;
+  layout_of(d, &l);
+  const uint8_t* w = static_cast<const uint8_t*>(ws);
+  if (cudaMemcpyAsync(M64, w + l.off_M64, l.bytes_M64, cudaMemcpyDeviceToDevice, static_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return ENTMAX_ECUDA;
   return ENTMAX_OK;
 }
 

@@ -52,6 +52,8 @@ struct Shared {
   uint32_t tmem_base;
   int abort_flag;
   uint32_t qlist[kMaskWords];
+  uint32_t k64[2][2 * kMaskWords];   // rows 2 kt and 2 kt + 1 of the transposed 64 x 64 mask
+  uint8_t quarters[32 * kMaskWords];   // per visited query tile: bit 2 qh + kh = quarter (qh, kh) nonzero
 };
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -61,9 +63,38 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 
 }  // namespace
 
+// dQ_s = dS K_j over key steps T0..T0+NT-1 (16 keys each; panel t/4): straight-line issue.
+template <int T0, int NT>
+__device__ __forceinline__ void dq_steps(uint32_t dq, uint64_t dHd, uint64_t dLd, uint64_t kM, uint32_t idQ) {
+#pragma unroll
+  for (int t = 0; t < NT; ++t) {
+    constexpr int kTb = kTileBytes;
+    const int tk = T0 + t;
+    const uint32_t koff = (tk >> 2) * kTb + (tk & 3) * 32;
+    const uint64_t bK = sdesc_add(kM, tk * 2048);
+    mma_ss(dq, sdesc_add(dHd, koff), bK, idQ, t > 0 ? 1u : 0u);
+    mma_ss(dq, sdesc_add(dLd, koff), bK, idQ, 1u);
+  }
+}
+
+// dV += A^T dO_s and dK += dS^T Q_s over query steps T0..T0+NT-1 (16 queries each).
+template <int T0, int NT>
+__device__ __forceinline__ void dvk_steps(uint32_t T, uint64_t aM, uint64_t dHM, uint64_t dLM, uint64_t oM,
+                                          uint64_t qM, uint32_t idV, uint32_t idK, bool started) {
+#pragma unroll
+  for (int tq = 0; tq < NT; ++tq) {
+    const int t = T0 + tq;
+    const uint32_t acc = (started || tq > 0) ? 1u : 0u;
+    const uint64_t bO = sdesc_add(oM, t * 2048), bQ = sdesc_add(qM, t * 2048);
+    mma_ss(T + 256, sdesc_add(aM, t * 2048), bO, idV, acc);
+    mma_ss(T + 320, sdesc_add(dHM, t * 2048), bQ, idK, acc);
+    mma_ss(T + 320, sdesc_add(dLM, t * 2048), bQ, idK, 1u);
+  }
+}
+
 int bwd_smem_bytes() { return 1024 + 2 * kTileBytes + kStages * kPairBytes + 6 * kTileBytes + 2 * kTileBytes; }
 
-template <int AK, bool kAlibi>
+template <int AK, bool kAlibi, bool kM64>
 __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant__ BwdParams p) {
   extern __shared__ uint8_t dsm_raw[];
   __shared__ Shared sh;
@@ -104,9 +135,32 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     fence_mbar_init();
   }
   if (tid < kMaskWords) sh.qlist[tid] = (tid < p.Wr) ? p.MT[((size_t)bh * p.Tc + kt) * p.Wr + tid] : 0u;
+  if (kM64 && tid >= 32 && tid < 32 + 4 * kMaskWords) {
+    const int h = (tid - 32) / (2 * kMaskWords), w = (tid - 32) % (2 * kMaskWords);
+    sh.k64[h][w] = w < p.W64r ? p.M64T[((size_t)bh * 2 * p.Tc + 2 * kt + h) * p.W64r + w] : 0u;
+  }
   if (warp == kMmaWarp) {
     tmem_alloc(&sh.tmem_base, 512);
     tmem_relinquish();
+  }
+  __syncthreads();
+  // The 64 x 64 quarters of each visited query tile (query half qh, key half kh): the
+  // thread of query tile it writes entry rank(it) = number of visited tiles before it.
+  for (int it = tid; kM64 && it < p.Tr; it += kThreads) {
+    const uint32_t wbits = sh.qlist[it >> 5];
+    if ((wbits >> (it & 31)) & 1u) {
+      int rank = __popc(wbits & ((1u << (it & 31)) - 1u));
+      for (int w = 0; w < (it >> 5); ++w) rank += __popc(sh.qlist[w]);
+      uint32_t q = 0;
+#pragma unroll
+      for (int qh = 0; qh < 2; ++qh)
+#pragma unroll
+        for (int kh = 0; kh < 2; ++kh) {
+          const int qb = 2 * it + qh;
+          q |= ((sh.k64[kh][qb >> 5] >> (qb & 31)) & 1u) << (2 * qh + kh);
+        }
+      sh.quarters[rank] = (uint8_t)q;
+    }
   }
   __syncthreads();
   tc_fence_after();
@@ -180,14 +234,15 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
         if (!live) break;
         tc_fence_after();
         const uint32_t dq = T + 384 + (s & 1) * 64;
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          // dQ_s = dS K_j: K = keys (16 per step; panel t/4), M = queries.
-          const uint32_t koff = (t >> 2) * kTileBytes + (t & 3) * 32;
-          const uint64_t bK = sdesc_add(kM, t * 2048);
-          mma_ss(dq, sdesc_add(dHd, koff), bK, idQ, t > 0 ? 1u : 0u);
-          mma_ss(dq, sdesc_add(dLd, koff), bK, idQ, 1u);
-        }
+        // dQ_s = dS K_j: K = keys, M = queries. A key half with no nonzero weight in either
+        // query half (64 x 64 mask) contributes nothing, so its four steps are left out; the
+        // choice is made once per tile between straight-line sequences (a branch around each
+        // MMA would slow the issue).
+        const uint32_t qu = kM64 ? sh.quarters[s] : 15u;
+        const uint32_t kl = (qu | (qu >> 2)) & 3u;   // bit kh: key half kh has a nonzero weight
+        if (!kM64 || kl == 3u) dq_steps<0, 8>(dq, dHd, dLd, kM, idQ);
+        else if (kl == 1u) dq_steps<0, 4>(dq, dHd, dLd, kM, idQ);
+        else dq_steps<4, 4>(dq, dHd, dLd, kM, idQ);
         mma_commit(&sh.empty[s % kStages]);   // S and dA of tile s were this warp's last reads
         mma_commit(&sh.mma2_done);
       }
@@ -201,21 +256,21 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       const uint64_t aM = sdesc_sw128(smem_u32(sA), 16384, 1024);      // A, MN-major (dV)
       const uint64_t dHM = sdesc_sw128(smem_u32(sdS), 16384, 1024), dLM = sdesc_sw128(smem_u32(sdSl), 16384, 1024);
       const uint64_t rM = sdesc_sw128(smem_u32(ring), 8192, 1024);     // ring stage 0, MN-major
+      bool started = false;   // the dV and dK accumulators hold a first product
       for (int s = 0; s < nq; ++s) {
         const int st = s % kStages;
         const uint64_t qM = sdesc_add(rM, st * kPairBytes), oM = sdesc_add(qM, kTileBytes);
         if (!mbar_wait(&sh.full[st], (s / kStages) & 1, wc)) break;   // Q_s and dO_s landed
         if (!mbar_wait(&sh.p_ready, s & 1, wc)) break;                // A and dS of tile s written
         tc_fence_after();
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          // dV += A^T dO_s and dK += dS^T Q_s: K = queries (16 per step), M = keys.
-          const uint32_t acc = (s > 0 || t > 0) ? 1u : 0u;
-          const uint64_t bO = sdesc_add(oM, t * 2048), bQ = sdesc_add(qM, t * 2048);
-          mma_ss(T + 256, sdesc_add(aM, t * 2048), bO, idV, acc);
-          mma_ss(T + 320, sdesc_add(dHM, t * 2048), bQ, idK, acc);
-          mma_ss(T + 320, sdesc_add(dLM, t * 2048), bQ, idK, 1u);
-        }
+        // dV += A^T dO_s and dK += dS^T Q_s: K = queries, M = keys. A query half with no
+        // nonzero weight in either key half contributes nothing (chosen once per tile).
+        const uint32_t qu = kM64 ? sh.quarters[s] : 15u;
+        const uint32_t ql = ((qu & 3u) ? 1u : 0u) | ((qu & 12u) ? 2u : 0u);   // bit qh: query half qh live
+        if (!kM64 || ql == 3u) dvk_steps<0, 8>(T, aM, dHM, dLM, oM, qM, idV, idK, started);
+        else if (ql == 1u) dvk_steps<0, 4>(T, aM, dHM, dLM, oM, qM, idV, idK, started);
+        else dvk_steps<4, 4>(T, aM, dHM, dLM, oM, qM, idV, idK, started);
+        started = true;
         mma_commit(&sh.empty[st]);
         mma_commit(&sh.mma2_done);
       }
@@ -271,19 +326,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       warp_wait(&sh.s_full, seq & 1, wc);
       const long long c1 = clock64();
       tc_fence_after();
+      // Keys [32 qc, 32 qc + 32) of row `row`: panel qc/2, 16-byte chunks 4(qc%2)..+3.
+      const int pan = (qc >> 1) * kTileBytes;
       // S and dA are read in two halves of 16 columns, so only 32 of them are live at a
       // time; the second half's read releases the TMEM columns (sda_free) for the next tile.
       uint32_t sr[16], ar[16];
-      tmem_ld16(tl + qc * 32, sr);
-      tmem_ld16(tl + 128 + qc * 32, ar);
-      tmem_wait_ld();
-      const long long c1b = clock64();
-      // The previous tile's dV/dK/dQ MMAs must be done reading sA / sdS.
-      const long long c2 = clock64();
-      if (seq > 0) warp_wait(&sh.mma2_done, (seq - 1) & 1, wc);
-      const long long c3 = clock64();
-      // Keys [32 qc, 32 qc + 32) of row `row`: panel qc/2, 16-byte chunks 4(qc%2)..+3.
-      const int pan = (qc >> 1) * kTileBytes;
       auto form_half = [&](int hf) {
 #pragma unroll
         for (int ch = 0; ch < 2; ++ch) {
@@ -332,6 +379,16 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
           *reinterpret_cast<uint4*>(sdSl + off) = make_uint4(dl2[0], dl2[1], dl2[2], dl2[3]);
         }
       };
+      tmem_ld16(tl + qc * 32, sr);
+      tmem_ld16(tl + 128 + qc * 32, ar);
+      tmem_wait_ld();
+      const long long c1b = clock64();
+      // The previous tile's dV/dK/dQ MMAs must be done reading sA / sdS.
+      const long long c2 = clock64();
+      if (seq > 0) warp_wait(&sh.mma2_done, (seq - 1) & 1, wc);
+      const long long c3 = clock64();
+      // In a 64 x 64 quarter without a nonzero weight every u <= 0, so A and dS come out
+      // zero there; the MMA issuers leave out the steps of empty halves.
       form_half(0);
       tmem_ld16(tl + qc * 32 + 16, sr);
       tmem_ld16(tl + 128 + qc * 32 + 16, ar);
@@ -411,10 +468,16 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
 
 cudaError_t launch_bwd(int alpha_kind, const BwdParams& p, int grid, cudaStream_t s) {
   const int smem = bwd_smem_bytes();
-  const bool ab = p.alibi != nullptr;   // compile-time ALiBi variant, as in the forward
-  auto kern = alpha_kind == kAlpha15 ? (ab ? bwd_kernel<kAlpha15, true> : bwd_kernel<kAlpha15, false>)
-             : alpha_kind == kAlpha2 ? (ab ? bwd_kernel<kAlpha2, true> : bwd_kernel<kAlpha2, false>)
-                                     : (ab ? bwd_kernel<kAlphaGen, true> : bwd_kernel<kAlphaGen, false>);
+  // ALiBi and the 64 x 64 skipping are compile-time variants, as in the forward.
+  const bool ab = p.alibi != nullptr, m64 = p.M64T != nullptr;
+  using K = void (*)(BwdParams);
+  auto pick = [&](K a00, K a01, K a10, K a11) { return ab ? (m64 ? a11 : a10) : (m64 ? a01 : a00); };
+  const K kern = alpha_kind == kAlpha15 ? pick(bwd_kernel<kAlpha15, false, false>, bwd_kernel<kAlpha15, false, true>,
+                                               bwd_kernel<kAlpha15, true, false>, bwd_kernel<kAlpha15, true, true>)
+                 : alpha_kind == kAlpha2 ? pick(bwd_kernel<kAlpha2, false, false>, bwd_kernel<kAlpha2, false, true>,
+                                                bwd_kernel<kAlpha2, true, false>, bwd_kernel<kAlpha2, true, true>)
+                                         : pick(bwd_kernel<kAlphaGen, false, false>, bwd_kernel<kAlphaGen, false, true>,
+                                                bwd_kernel<kAlphaGen, true, false>, bwd_kernel<kAlphaGen, true, true>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   kern<<<grid, kThreads, smem, s>>>(p);

@@ -47,6 +47,8 @@
 //     [32q, 32q+32) writes their A (fp16 pairs) into columns [32q, 32q+16): only over S
 //     columns it has read itself;
 //   - O at [256,320).
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -108,6 +110,7 @@ struct Shared {
   int ctl_kind, ctl_buf;
   uint32_t act[kMaskWords];          // structurally active key tiles
   uint32_t lists[2][kMaskWords];     // key tiles of the next sweep / the final mask
+  uint32_t m64[2][2 * kMaskWords];   // the mask at 64 x 64 blocks: [row half][key block bits]
   int votes[kMaxVotes];
 };
 
@@ -420,7 +423,55 @@ __device__ __forceinline__ float solveN(const float (&v)[N], float cz, float e, 
 
 }  // namespace
 
-template <int AK, bool kAlibi>
+// The 64 x 64 mask from the support lists (row owners, once per CTA; kept out of line so
+// that it does not change the register allocation of the kernel's loops). A thread's keys
+// lie in its column part qp of each tile, so a support key of tile jt is in 64-key block
+// 2 jt + qp/2: the thread marks tiles, the warp (32 rows of one row half, one part) ORs the
+// marks, and lane 0 spreads them to blocks and adds them to the shared mask m64 [2][8].
+__device__ __noinline__ void m64_mark(uint32_t* m64, const float* mycand, const uint16_t* myidx, int nc, bool use,
+                                      float cz, float tau, int quad, int qp, int lane) {
+  uint32_t tm[kMaskWords];
+#pragma unroll
+  for (int w = 0; w < kMaskWords; ++w) tm[w] = 0u;
+  if (use)
+    for (int k = 0; k < nc; ++k)
+      if (fmaf(mycand[k * kTile], cz, -tau) > 0.f) {
+        const int jt = myidx[k * kTile] >> 7;
+#pragma unroll
+        for (int w = 0; w < kMaskWords; ++w) tm[w] |= (jt >> 5) == w ? 1u << (jt & 31) : 0u;
+      }
+#pragma unroll
+  for (int w = 0; w < kMaskWords; ++w) {
+    const uint32_t x = __reduce_or_sync(0xffffffffu, tm[w]);
+    if (lane == 0 && x != 0u) {
+      // tile bit b of word w -> block bit 2 b + qp/2, in words 2w and 2w + 1
+#pragma unroll
+      for (int hw = 0; hw < 2; ++hw) {
+        uint32_t v = (x >> (16 * hw)) & 0xffffu;   // spread 16 bits to the even positions
+        v = (v | (v << 8)) & 0x00ff00ffu;
+        v = (v | (v << 4)) & 0x0f0f0f0fu;
+        v = (v | (v << 2)) & 0x33333333u;
+        v = (v | (v << 1)) & 0x55555555u;
+        if (v) atomicOr(&m64[(quad >> 1) * 2 * kMaskWords + 2 * w + hw], v << (qp >> 1));
+      }
+    }
+  }
+}
+
+// Rows 2 qt and 2 qt + 1 of the 64 x 64 mask and their bits of the transpose (threads
+// tid < 2 W64c, after every mark is in m64).
+__device__ __noinline__ void m64_write(const uint32_t* m64, const FwdParams& p, int tid, int bh, int qt) {
+  const int h = tid / p.W64c, w = tid % p.W64c;
+  const uint32_t bits = m64[h * 2 * kMaskWords + w];
+  const int qb = 2 * qt + h;
+  p.M64[((size_t)bh * 2 * p.Tr + qb) * p.W64c + w] = bits;
+  for (uint32_t b = bits; b; b &= b - 1) {
+    const int kb = w * 32 + __ffs(b) - 1;
+    atomicOr(&p.M64T[((size_t)bh * 2 * p.Tc + kb) * p.W64r + (qb >> 5)], 1u << (qb & 31));
+  }
+}
+
+template <int AK, bool kAlibi, bool kM64>
 __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant__ FwdParams p) {
   using OL = OutLayout<AK>;
   constexpr int kOBufs = OL::kBufs;
@@ -471,6 +522,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     sh.lists[1][tid] = 0;
   }
   for (int v = tid; v < kMaxVotes; v += kThreads) sh.votes[v] = 0;
+  if (tid < 4 * kMaskWords) (&sh.m64[0][0])[tid] = 0;
   for (int e = tid; e < p.Tc * kTile; e += kThreads) tmax[e] = f2ord(-INFINITY);
   if (warp == kMmaWarp) {
     tmem_alloc(&sh.tmem_base, 512);
@@ -807,7 +859,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     // at tau in fp16 over the S columns this thread has read (the part's keys qp*kCols..
     // go into its own columns [qp*kCols, +kCols/2), so the row's other parts never see an
     // overwritten S value).
-    auto out_tile = [&](int jt, uint32_t ko, bool collect, float thr) {
+    auto out_tile = [&](int jt, uint32_t ko, float thr, auto collect_tag, auto mark_tag) {
+      constexpr bool collect = decltype(collect_tag)::value, mark = decltype(mark_tag)::value;
       const int c = ko % kOBufs;
       const uint32_t pa = OL::sbuf(c);
       DIAG(const long long d0 = clock64());
@@ -824,7 +877,15 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         for (int cc = 0; cc < kCols; ++cc)
           if (!pat.active(i, j0 + cc)) s[cc] = -INFINITY;
       }
-      if (collect) collect_tile(s, j0, !done, thr);   // collect is warp-uniform
+      if constexpr (collect) collect_tile(s, j0, !done, thr);
+      if constexpr (mark) {   // the 64 x 64 mask at the final tau: a score of this part above tau
+        float mx = s[0];
+#pragma unroll
+        for (int cc = 1; cc < kCols; ++cc) mx = fmaxf(mx, s[cc]);
+        const int kb = 2 * jt + (qp >> 1);
+        if (__any_sync(0xffffffffu, fmaf(mx, cz, -tau) > 0.f) && lane == 0)
+          atomicOr(&sh.m64[quad >> 1][kb >> 5], 1u << (kb & 31));
+      }
       uint32_t aw[kCols / 2];
 #pragma unroll
       for (int cc = 0; cc < kCols / 2; ++cc) {
@@ -923,7 +984,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         if (!o_final) {
           // Phase 4: output pass at the final tau over the flagged tiles.
           int k = 0;
-          for_each_bit(list, kMaskWords, [&](int jt) { out_tile(jt, obase + k++, false, 0.f); });
+          for_each_bit(list, kMaskWords,
+                       [&](int jt) { out_tile(jt, obase + k++, 0.f, std::false_type{}, std::integral_constant<bool, kM64>{}); });
           if (k > 0) warp_wait(&sh.pv_done[(obase + k - 1) % kOBufs], ((obase + k - 1) / kOBufs) & 1, wc);
           obase += k;
         }
@@ -948,6 +1010,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         // copies (refinement cap, or a Newton finish) gets sum g = -1, and the backward
         // recomputes its support.
         DIAG(const long long de2 = clock64(); dgx[5] += de2 - de1);
+        if constexpr (kM64)
+          if (o_final)   // the 64 x 64 mask from the support lists
+            m64_mark(&sh.m64[0][0], mycand, myidx, nc, valid && listed, cz, tau, quad, qp, lane);
         if (qp == 0) {
           part[3 * kTile + row] = tau;
           part[7 * kTile + row] = (valid && listed) ? 1.f : 0.f;
@@ -955,6 +1020,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           if (valid) p.tau[(size_t)bh * p.L + i] = tau;
         }
         named_bar(3, kMathThreads);
+        if constexpr (kM64)
+          if (tid < 2 * p.W64c) m64_write(&sh.m64[0][0], p, tid, bh, qt);
         {
           const int sub = lane & 7;                      // columns 8 sub .. 8 sub + 7
           const uint4* vbase = reinterpret_cast<const uint4*>(p.Vb + (size_t)bh * p.L * kD) + sub;
@@ -1066,7 +1133,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         tau_T = tau;
         int k = 0;
         const float thr = cand_threshold(tau, cz);
-        for_each_bit(list, kMaskWords, [&](int jt) { out_tile(jt, obase + k++, true, thr); });
+        for_each_bit(list, kMaskWords, [&](int jt) { out_tile(jt, obase + k++, thr, std::true_type{}, std::false_type{}); });
         // O of the last tile done: the epilogue reads O, and a later sweep reuses its columns.
         if (k > 0) warp_wait(&sh.pv_done[(obase + k - 1) % kOBufs], ((obase + k - 1) / kOBufs) & 1, wc);
         obase += k;
@@ -1260,11 +1327,17 @@ int fwd_smem_bytes(int Tc) { return 1024 + fwd_off_region() + fwd_region_bytes(T
 
 cudaError_t launch_fwd(int alpha_kind, const FwdParams& p, int grid, cudaStream_t s) {
   const int smem = fwd_smem_bytes(p.Tc);
-  // ALiBi is a compile-time variant so heads without the bias carry none of its code.
-  const bool ab = p.alibi != nullptr;
-  auto kern = alpha_kind == kAlpha15 ? (ab ? fwd_kernel<kAlpha15, true> : fwd_kernel<kAlpha15, false>)
-             : alpha_kind == kAlpha2 ? (ab ? fwd_kernel<kAlpha2, true> : fwd_kernel<kAlpha2, false>)
-                                     : (ab ? fwd_kernel<kAlphaGen, true> : fwd_kernel<kAlphaGen, false>);
+  // ALiBi and the 64 x 64 mask are compile-time variants, so calls without them carry none of
+  // their code.
+  const bool ab = p.alibi != nullptr, m64 = p.M64 != nullptr;
+  using K = void (*)(FwdParams);
+  auto pick = [&](K a00, K a01, K a10, K a11) { return ab ? (m64 ? a11 : a10) : (m64 ? a01 : a00); };
+  const K kern = alpha_kind == kAlpha15 ? pick(fwd_kernel<kAlpha15, false, false>, fwd_kernel<kAlpha15, false, true>,
+                                               fwd_kernel<kAlpha15, true, false>, fwd_kernel<kAlpha15, true, true>)
+                 : alpha_kind == kAlpha2 ? pick(fwd_kernel<kAlpha2, false, false>, fwd_kernel<kAlpha2, false, true>,
+                                                fwd_kernel<kAlpha2, true, false>, fwd_kernel<kAlpha2, true, true>)
+                                         : pick(fwd_kernel<kAlphaGen, false, false>, fwd_kernel<kAlphaGen, false, true>,
+                                                fwd_kernel<kAlphaGen, true, false>, fwd_kernel<kAlphaGen, true, true>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   kern<<<grid, kThreads, smem, s>>>(p);

@@ -104,6 +104,7 @@ __global__ void __launch_bounds__(kThreads32) fwd_f32_kernel(const FwdF32Params 
   float* tmax = sV + kTile * kD;           // [Tc][128]
   float* cand = tmax + p.Tc * kTile;       // [64][128]
   __shared__ uint32_t act[kMaskWords], flag[kMaskWords];
+  __shared__ uint32_t m64[2][2 * kMaskWords];   // the mask at 64 x 64 blocks: [row half][key block bits]
   __shared__ int any_need;
 
   const int r = threadIdx.x;
@@ -118,6 +119,7 @@ __global__ void __launch_bounds__(kThreads32) fwd_f32_kernel(const FwdF32Params 
   const float cz = p.cz;
 
   if (r < kMaskWords) act[r] = flag[r] = 0;
+  if (r < 4 * kMaskWords) (&m64[0][0])[r] = 0;
   __syncthreads();
   for (int jt = r; jt < p.Tc; jt += kThreads32)
     if (pat.block_active(i0, i1, jt * kTile, min(p.L, jt * kTile + kTile))) atomicOr(&act[jt >> 5], 1u << (jt & 31));
@@ -233,10 +235,12 @@ __global__ void __launch_bounds__(kThreads32) fwd_f32_kernel(const FwdF32Params 
     stage_tile(sV, p.V + head, jt * kTile, p.L);
     __syncthreads();
     ++n_out;
+    bool nz[2] = {false, false};   // a nonzero weight in key half 0 / 1 of the tile
     for (int c = 0; c < kTile; ++c) {
       if (!pat.active(i, jt * kTile + c)) continue;
       const float u = fmaf(dot64(q, sK + c * kD), cz, -tau);
       if (!(u > 0.f)) continue;
+      nz[c >> 6] = true;
       const float w = (AK == kAlpha15) ? u * u : u;
       const float4* v4 = reinterpret_cast<const float4*>(sV + c * kD);
 #pragma unroll
@@ -248,7 +252,21 @@ __global__ void __launch_bounds__(kThreads32) fwd_f32_kernel(const FwdF32Params 
         o[4 * cc + 3] = fmaf(w, v.w, o[4 * cc + 3]);
       }
     }
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+      if (nz[h]) atomicOr(&m64[r >> 6][(2 * jt + h) >> 5], 1u << ((2 * jt + h) & 31));
   });
+  __syncthreads();
+  if (p.M64 && r < 2 * p.W64c) {   // rows 2 qt and 2 qt + 1 of the 64 x 64 mask, and its transpose
+    const int h = r / p.W64c, w = r % p.W64c;
+    const uint32_t bits = m64[h][w];
+    const int qb = 2 * qt + h;
+    p.M64[((size_t)bh * 2 * p.Tr + qb) * p.W64c + w] = bits;
+    for (uint32_t b = bits; b; b &= b - 1) {
+      const int kb = w * 32 + __ffs(b) - 1;
+      atomicOr(&p.M64T[((size_t)bh * 2 * p.Tc + kb) * p.W64r + (qb >> 5)], 1u << (qb & 31));
+    }
+  }
   if (valid) {
     float4* dst = reinterpret_cast<float4*>(p.O + head + (size_t)i * kD);
 #pragma unroll

@@ -35,10 +35,13 @@ struct FwdParams {
   const uint16_t* Vb;       // [B*H][L][64]  V as given (bf16)
   uint32_t* M;              // [B*H][Tr][Wc]
   uint32_t* MT;             // [B*H][Tc][Wr] (zeroed before the launch)
+  uint32_t* M64;            // [B*H][2 Tr][W64c]: the mask at 64 x 64 blocks, or nullptr (not built)
+  uint32_t* M64T;           // [B*H][2 Tc][W64r] (zeroed before the launch), or nullptr
   int* stats;               // [B*H][Tr][kFwdStats] (layout above)
   int* status;
   const int* kv_len;        // [B] or nullptr
   int H, L, Tr, Tc, Wc, Wr, BH;
+  int W64c, W64r;           // words per row of M64 and of M64T
   float cz;                 // (alpha - 1) * scale
   float ae, am1;            // 1 / (alpha - 1) and alpha - 1 (the run-time alpha variant)
   const float* alibi;       // [H] ALiBi slopes (score units per position), or nullptr
@@ -54,6 +57,7 @@ struct BwdParams {
   const float* tau;              // [B*H][L]
   const float* delta;            // [B*H][L]
   const uint32_t* MT;            // [B*H][Tc][Wr]
+  const uint32_t* M64T;          // [B*H][2 Tc][W64r]: the transposed mask at 64 x 64 blocks, or nullptr
   float* dQ;                     // [B*H][L][64] (zeroed, accumulated with atomics)
   float* dK;
   float* dV;
@@ -61,6 +65,7 @@ struct BwdParams {
   int* stats;                    // [B*H][Tc][kBwdStats] (layout above)
   const int* kv_len;
   int H, L, Tr, Tc, Wr, BH;
+  int W64r;
   float cz;                      // (alpha - 1) * scale
   float scale;
   float ae;                      // 1 / (alpha - 1)
@@ -99,10 +104,13 @@ struct FwdF32Params {
   float* tau;
   uint32_t* M;
   uint32_t* MT;
+  uint32_t* M64;            // as in FwdParams
+  uint32_t* M64T;
   int* stats;               // [B*H][Tr][kFwdStats]
   int* status;
   const int* kv_len;
   int H, L, Tr, Tc, Wc, Wr, BH;
+  int W64c, W64r;
   float cz;
   int causal, window, max_sweeps;
 };

@@ -105,6 +105,12 @@ typedef struct {
                              nothing completes, so that the wait expires after
                              wait_limit_us and the call reports ENTMAX_ETIMEOUT: a test of
                              the failure path that faults and hangs nothing.              */
+    int mask64;           /* 0 (default) or 1. With 1 the forward also builds the block mask at
+                             64 x 64 blocks (entmax_attn_block_mask64) and the backward
+                             leaves out the MMA steps of 64-row and 64-key halves of a
+                             flagged tile that hold no nonzero weight. Both passes of a call
+                             pair must use the same value. Separate kernel builds, so the
+                             default path carries none of it.                              */
 } entmax_attn_desc;
 
 #define ENTMAX_SELFTEST_STALL 1
@@ -172,10 +178,22 @@ entmax_status entmax_last_device_status(const entmax_attn_desc *desc, const void
  *   - bwd_stats is int32 [B, H, Tc, 8]. Per key tile of the last backward: the flagged
  *     query tiles visited, the CTA's cycles in total, then the first row-owner warp's
  *     cycles waiting for S and dA, waiting for the previous tile's gradient MMAs,
- *     forming A and dS, and staging dQ for its reduce-add; two zero words.
+ *     forming A and dS, staging dQ for its reduce-add, and the part of forming spent
+ *     loading S and dA from tensor memory; one zero word.
  * Any output may be NULL. */
 entmax_status entmax_attn_block_mask(const entmax_attn_desc *desc, const void *workspace,
                                      uint32_t *M, int *stats, int *bwd_stats, void *stream);
+
+/* Copies the forward's block mask at 64 x 64 blocks ("AdaSplash-2", §4.2 and Fig. 7 measure
+ * block sparsity at this unit) out of the workspace, device to device, on `stream`.
+ * M64 is uint32 [B, H, 2*Tr, ceil(2*Tc/32)] (Tr = Tc = ceil(L/128)): bit (kb % 32) of word
+ * kb/32 of row qb is set when some query row in [64 qb, 64 qb + 64) has a nonzero weight on
+ * a key in [64 kb, 64 kb + 64). Blocks past L are 0. Like the 128 x 128 mask it is exact for
+ * the fp32 scores at the final tau. Only a forward run with desc->mask64 = 1 builds it
+ * (otherwise ENTMAX_EINVAL). The backward of such a call pair reads its transpose from the
+ * workspace and leaves out the empty halves of flagged 128 x 128 tiles. */
+entmax_status entmax_attn_block_mask64(const entmax_attn_desc *desc, const void *workspace, uint32_t *M64,
+                                       void *stream);
 
 /* Forward for callers that cannot allocate device memory. Some callers are handed
  * only their input and output buffers: a plugin inside a host framework that owns

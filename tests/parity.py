@@ -28,20 +28,24 @@ MARGIN = 1e-3
 # are reported, not compared. A = [z - tau]_+ is continuous, so dV is always compared.
 
 
-def gpu_run(inp: dict, w: Workload, alpha: float, backward: bool = True, max_sweeps: int = 0):
+def gpu_run(inp: dict, w: Workload, alpha: float, backward: bool = True, max_sweeps: int = 0,
+            mask64: bool = False):
     dev = {k: v.cuda() for k, v in inp.items()}
     kv = None if w.kv_len is None else torch.tensor(w.kv_len_list(), dtype=torch.int32, device="cuda")
     ab = None if w.alibi is None else torch.tensor(w.alibi, dtype=torch.float32, device="cuda")
     O, tau, ctx = eb.forward(dev["Q"], dev["K"], dev["V"], alpha=alpha, scale=w.scale, causal=w.causal,
-                             window=w.window, kv_len=kv, max_sweeps=max_sweeps, alibi=ab)
+                             window=w.window, kv_len=kv, max_sweeps=max_sweeps, alibi=ab, mask64=mask64)
     out = {"O": O, "tau": tau}
     if backward:
         out["dQ"], out["dK"], out["dV"] = eb.backward(ctx, dev["Q"], dev["K"], dev["V"], dev["dO"], tau)
     M, stats = eb.block_mask(ctx)
+    M64 = eb.block_mask64(ctx) if mask64 else None
     code, word = eb.entmax_last_device_status(ctx[0], ctx[1])
     torch.cuda.synchronize()
     res = {k: v.cpu().double().numpy() for k, v in out.items()}
     res["M"] = M.cpu().numpy().view(np.uint32)
+    if M64 is not None:
+        res["M64"] = M64.cpu().numpy().view(np.uint32)
     res["stats"] = stats.cpu().numpy()
     res["status"] = (code, word)
     return res
@@ -106,23 +110,39 @@ def alpha2_exclusions(pr: oracle.Problem, tau_ref: np.ndarray, tau_gpu: np.ndarr
     return rows, keys
 
 
-def check_mask(pr: oracle.Problem, tau_ref: np.ndarray, M_gpu: np.ndarray):
-    M, Mlo, Mhi = pr.block_mask(tau_ref, 128, 128, margin=MARGIN)
+def check_mask(pr: oracle.Problem, tau_ref: np.ndarray, M_gpu: np.ndarray, block: int = 128):
+    """Bits of the GPU block mask that disagree with the oracle's, away from the ambiguity
+    margin, and the number of ambiguous bits. block = 64: the 64 x 64 mask, whose GPU copy
+    has 2 ceil(L/128) rows per head (a last row past L must be empty)."""
+    M, Mlo, Mhi = pr.block_mask(tau_ref, block, block, margin=MARGIN)
+    G = M_gpu
+    if G.shape != M.shape:
+        extra = G[..., M.shape[2]:, :]
+        assert not extra.any(), "64 x 64 mask rows past L must be empty"
+        G = G[..., : M.shape[2], : M.shape[3]]
     decided = ~(Mlo ^ Mhi)
-    bad = (M_gpu ^ M) & decided
+    bad = (G ^ M) & decided
     n_amb = int(sum(bin(int(x)).count("1") for x in (Mlo ^ Mhi).ravel()))
     return int(np.count_nonzero(bad)), n_amb
 
 
-def compare(w: Workload, alpha: float, backward: bool = True, seed: int = 0, report: dict | None = None):
+def compare(w: Workload, alpha: float, backward: bool = True, seed: int = 0, report: dict | None = None,
+            mask64: bool = True):
+    """GPU against the oracle on one small case. mask64 (default on here) also builds the
+    64 x 64 mask, checks it bit for bit, and runs the backward variant that skips empty
+    64-wide halves."""
     inp = make_inputs(w, seed)
-    g = gpu_run(inp, w, alpha, backward)
+    g = gpu_run(inp, w, alpha, backward, mask64=mask64)
     pr = oracle_problem(inp, w, alpha)
     ref = pr.backward() if backward else pr.forward()
     err = {"tau": np.abs(g["tau"] - ref["tau"]).max(), "O": np.abs(g["O"] - ref["O"]).max()}
     assert g["status"][0] == eb.ENTMAX_OK, g["status"]
     nbad, namb = check_mask(pr, ref["tau"], g["M"])
     err["mask_bad"], err["mask_ambiguous"] = nbad, namb
+    nbad64 = 0
+    if mask64:
+        nbad64, namb64 = check_mask(pr, ref["tau"], g["M64"], 64)
+        err["mask64_bad"], err["mask64_ambiguous"] = nbad64, namb64
     if backward:
         if alpha == 2.0:
             xr, xk = alpha2_exclusions(pr, ref["tau"], g["tau"])
@@ -139,6 +159,7 @@ def compare(w: Workload, alpha: float, backward: bool = True, seed: int = 0, rep
     assert err["tau"] <= TOL_TAU, err
     assert err["O"] <= TOL_O, err
     assert nbad == 0, err
+    assert nbad64 == 0, err
     if backward:
         assert max(err["dQ"], err["dK"], err["dV"]) <= TOL_GRAD, err
     return err, g, ref

@@ -42,11 +42,11 @@ def test_library_exports_every_declared_symbol(lib):
 
 def _desc(**kw):
     base = dict(B=1, H=2, L=300, d=64, alpha=1.5, scale=0.125, causal=0, window=-1, kv_len=None,
-                dtype=eb.ENTMAX_BF16, max_sweeps=0, wait_limit_us=0, alibi_slopes=None, selftest=0)
+                dtype=eb.ENTMAX_BF16, max_sweeps=0, wait_limit_us=0, alibi_slopes=None, selftest=0, mask64=0)
     base.update(kw)
     return eb.AttnDesc(base["B"], base["H"], base["L"], base["d"], base["alpha"], base["scale"], base["causal"],
                        base["window"], base["kv_len"], base["dtype"], base["max_sweeps"], base["wait_limit_us"],
-                       base["alibi_slopes"], base["selftest"])
+                       base["alibi_slopes"], base["selftest"], base["mask64"])
 
 
 def test_workspace_bytes_valid_and_invalid(lib):
@@ -56,7 +56,7 @@ def test_workspace_bytes_valid_and_invalid(lib):
     assert lib.entmax_attn_workspace_bytes(ctypes.byref(_desc(L=4096))) > n
     for bad in (dict(B=0), dict(L=0), dict(d=32), dict(alpha=1.0), dict(alpha=17.0), dict(scale=0.0), dict(causal=2),
                 dict(max_sweeps=-1), dict(max_sweeps=65), dict(L=eb.ENTMAX_MAX_L + 1), dict(dtype=7),
-                dict(wait_limit_us=-1), dict(selftest=2)):
+                dict(wait_limit_us=-1), dict(selftest=2), dict(mask64=2)):
         assert lib.entmax_attn_workspace_bytes(ctypes.byref(_desc(**bad))) == 0, bad
 
 
@@ -74,6 +74,7 @@ def test_workspace_bytes_valid_and_invalid(lib):
     (dict(max_sweeps=100), eb.ENTMAX_EINVAL),
     (dict(wait_limit_us=-5), eb.ENTMAX_EINVAL),
     (dict(selftest=3), eb.ENTMAX_EINVAL),
+    (dict(mask64=-1), eb.ENTMAX_EINVAL),
 ])
 def test_forward_rejects_on_host(lib, bad, code):
     d = _desc(**bad)
@@ -118,3 +119,10 @@ def test_desc_layout_matches_header():
     """The ctypes mirror has the header's field order (checked by offsets of the tail)."""
     assert eb.AttnDesc.alibi_slopes.offset % 8 == 0
     assert eb.AttnDesc.selftest.offset > eb.AttnDesc.alibi_slopes.offset
+
+
+def test_block_mask64_needs_a_mask64_forward(lib):
+    """entmax_attn_block_mask64 rejects a descriptor without mask64 before touching memory."""
+    good = ctypes.c_void_p(1 << 20)
+    assert lib.entmax_attn_block_mask64(ctypes.byref(_desc()), good, good, None) == eb.ENTMAX_EINVAL
+    assert lib.entmax_attn_block_mask64(ctypes.byref(_desc(mask64=1)), good, None, None) == eb.ENTMAX_EINVAL

@@ -7,8 +7,9 @@ the headline inputs:
   - planted block structure with rho in {1, 1/2, 1/4, 1/8, 1/16} of the key tiles
     holding each query tile's support (a stand-in for trained models' block sparsity).
 Here one whole head of each extreme (sigma_Q = 24; rho = 1 and 1/16), at both alphas, runs
-at L = 8192 in the bench's launch configuration and is compared element by element:
-every row's tau and O, every row's dQ, every key's dK and dV, and the block mask. A
+at L = 8192 in the bench's launch configuration, with the 64 x 64 mask built and used by the
+backward, and is compared element by element: every row's tau and O, every row's dQ, every
+key's dK and dV, and the block masks at 128 x 128 and 64 x 64. A
 smaller sigma_Q = 24 case with several heads and a ragged tail covers the same family at
 a size where the oracle also checks a second head.
 """
@@ -26,7 +27,7 @@ HEAD = WORKLOADS["long_causal_L8192"].with_(B=1, H=1)
 
 
 def _check_head(inp, w, alpha, label):
-    g = gpu_run(inp, w, alpha, backward=True)
+    g = gpu_run(inp, w, alpha, backward=True, mask64=True)
     assert g["status"][0] == eb.ENTMAX_OK, g["status"]
     pr = oracle_problem(inp, w, alpha)
     ref = pr.backward()
@@ -41,6 +42,7 @@ def _check_head(inp, w, alpha, label):
     err["dK"] = np.abs(np.where(keys_ok, g["dK"] - ref["dK"], 0)).max()
     err["dV"] = np.abs(g["dV"] - ref["dV"]).max()
     nbad, namb = check_mask(pr, ref["tau"], g["M"])
+    err["mask64_bad"] = check_mask(pr, ref["tau"], g["M64"], 64)[0]
     st = g["stats"].reshape(-1, eb.FWD_STATS)
     err["block_sparsity"] = 1.0 - st[:, 2].sum() / st[:, 3].sum()
     err["mask_bad"], err["mask_ambiguous"] = nbad, namb
@@ -49,6 +51,7 @@ def _check_head(inp, w, alpha, label):
     assert err["O"] <= TOL_O, err
     assert max(err["dQ"], err["dK"], err["dV"]) <= TOL_GRAD, err
     assert nbad == 0, err
+    assert err["mask64_bad"] == 0, err
     return err
 
 

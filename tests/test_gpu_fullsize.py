@@ -66,3 +66,4 @@ def test_full_size(name, alpha, heads):
         M, Mlo, Mhi = pr.block_mask(ref["tau"], 128, 128, margin=MARGIN)
         decided = ~(Mlo ^ Mhi)
         assert np.count_nonzero((g["M"][b, h] ^ M[0, 0]) & decided[0, 0]) == 0
+

@@ -41,9 +41,21 @@ CASES = [
 @pytest.mark.parametrize("alpha", [1.5, 2.0])
 @pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
 def test_fwd_bwd_small(w, alpha):
+    """Every case with the 64 x 64 mask built (checked bit for bit) and the backward variant
+    that leaves out empty 64-wide halves."""
     rep = {}
     compare(w, alpha, backward=True, report=rep)
     print(w.name, alpha, {k: (float(v) if not isinstance(v, int) else v) for k, v in rep.items()})
+
+
+@pytest.mark.parametrize("alpha", [1.5, 2.0])
+@pytest.mark.parametrize("w", [c for c in CASES if c.name in ("causal_L300", "window_L300", "padded_L300",
+                                                                  "peaked_causal_L520", "tile_plus_one_L129")],
+                         ids=lambda w: w.name)
+def test_fwd_bwd_small_without_mask64(w, alpha):
+    """The default kernels (no 64 x 64 mask) on the cases whose structure leaves 64-wide
+    halves empty."""
+    compare(w, alpha, backward=True, mask64=False)
 
 
 @pytest.mark.parametrize("alpha", [1.5, 2.0])
@@ -119,6 +131,8 @@ def test_single_head_fp32_workload():
     assert np.abs(g["tau"] - ref["tau"]).max() <= TOL_TAU
     assert np.abs(g["O"] - ref["O"]).max() <= 1e-2
     assert check_mask(pr, ref["tau"], g["M"])[0] == 0
+    if "M64" in g:
+        assert check_mask(pr, ref["tau"], g["M64"], 64)[0] == 0
     # entmax_rows on the explicit scores (computed in fp32 on the GPU by torch: plumbing)
     S = (inp["Q"][0, 0].cuda() @ inp["K"][0, 0].cuda().T) * w.scale
     P, tau = eb.rows(S.contiguous(), 1.5)
@@ -188,6 +202,8 @@ def test_planted_block_structure(alpha):
     for k in ("dQ", "dK", "dV"):
         assert np.abs(g[k] - ref[k]).max() <= 2e-2, k
     assert check_mask(pr, ref["tau"], g["M"])[0] == 0
+    if "M64" in g:
+        assert check_mask(pr, ref["tau"], g["M64"], 64)[0] == 0
     st = g["stats"].reshape(-1, eb.FWD_STATS)
     sparsity = 1.0 - st[:, 2].sum() / st[:, 3].sum()
     assert sparsity > 0.5, sparsity
