@@ -479,29 +479,47 @@ def sparsity_sweeps(w, alpha, dev, steps: int = 10):
     stream = torch.cuda.current_stream(dev)
     desc = eb.make_desc(w.B, w.H, w.L, w.d, alpha=alpha, scale=w.scale, causal=w.causal, window=w.window)
     ws = eb.alloc_workspace(desc, dev)
+    desc64 = eb.make_desc(w.B, w.H, w.L, w.d, alpha=alpha, scale=w.scale, causal=w.causal, window=w.window,
+                          mask64=True)
+    ws64 = eb.alloc_workspace(desc64, dev)
+    active64 = int(block_pair_counts(w, 64).astype(bool).sum()) * w.H   # structurally active 64 x 64 blocks
     shp = (w.B, w.H, w.L, w.d)
     O = torch.empty(shp, dtype=torch.float32, device=dev)
     tau = torch.empty(shp[:3], dtype=torch.float32, device=dev)
     dQ, dK, dV = (torch.empty(shp, dtype=torch.float32, device=dev) for _ in range(3))
 
-    def point(inp):
-        d = {k: v.to(dev) for k, v in inp.items()}
+    def timed(d, dsc, wsp):
         fwd, bwd = [], []
         for k in range(2 + steps):
             flush.zero_()
             e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
             e[0].record(stream)
-            eb.entmax_attn_fwd(desc, d["Q"], d["K"], d["V"], O, tau, ws, stream)
+            eb.entmax_attn_fwd(dsc, d["Q"], d["K"], d["V"], O, tau, wsp, stream)
             e[1].record(stream)
-            eb.entmax_attn_bwd(desc, d["Q"], d["K"], d["V"], d["dO"], tau, ws, dQ, dK, dV, stream)
+            eb.entmax_attn_bwd(dsc, d["Q"], d["K"], d["V"], d["dO"], tau, wsp, dQ, dK, dV, stream)
             e[2].record(stream)
             torch.cuda.synchronize(dev)
             if k >= 2:
                 fwd.append(e[0].elapsed_time(e[1]))
                 bwd.append(e[1].elapsed_time(e[2]))
+        return fwd, bwd
+
+    def point(inp, with64=False):
+        d = {k: v.to(dev) for k, v in inp.items()}
+        fwd, bwd = timed(d, desc, ws)
         _, st = eb.block_mask((desc, ws))
         st = st.cpu().long()
-        return {"block_sparsity_128": 1.0 - float(st[..., 2].sum()) / max(1, int(st[..., 3].sum())),
+        extra = {}
+        if with64:
+            # The same inputs with the 64 x 64 mask built by the kernel (mask64): its block
+            # sparsity over the structurally active 64 x 64 blocks, and the times of that
+            # variant (the backward then leaves out empty 64-wide halves).
+            f64, b64 = timed(d, desc64, ws64)
+            M64 = eb.block_mask64((desc64, ws64)).cpu().numpy().view("uint32")
+            nset = int(sum(bin(int(x)).count("1") for x in M64.ravel()))
+            extra = {"block_sparsity_64": 1.0 - nset / max(1, active64),
+                     "mask64_fwd_ms": statistics.mean(f64), "mask64_bwd_ms": statistics.mean(b64)}
+        return {**extra, "block_sparsity_128": 1.0 - float(st[..., 2].sum()) / max(1, int(st[..., 3].sum())),
                 "refine_sweeps_mean": float(st[..., 0].float().mean()),
                 "s_tiles_per_active": float(st[..., 1].sum()) / max(1, int(st[..., 3].sum())),
                 "s_tiles": int(st[..., 1].sum()), "flagged_tiles": int(st[..., 2].sum()),
@@ -515,7 +533,7 @@ def sparsity_sweeps(w, alpha, dev, steps: int = 10):
         planted.append(r)
     sigma = []
     for sq in (1.0, 3.0, 8.0, 24.0):
-        r = point(make_inputs(w.with_(sigma_q=sq), seed=7))
+        r = point(make_inputs(w.with_(sigma_q=sq), seed=7), with64=True)
         r["sigma_q"] = sq
         sigma.append(r)
     return {"planted_rho": planted, "iid_sigma_q": sigma, "marginal": marginal_throughput(planted),
@@ -543,12 +561,13 @@ def marginal_throughput(points) -> dict:
     return out
 
 
-def block_pair_counts(w):
-    """Structurally active (query, key) pairs in every 128 x 128 block, per batch entry:
-    int64 [B, T, T] (the same for every head)."""
+def block_pair_counts(w, tile: int = TILE):
+    """Structurally active (query, key) pairs in every tile x tile block, per batch entry:
+    int64 [B, T, T] with T = ceil(L / tile) (the same for every head)."""
     import numpy as np
 
-    L, T = w.L, -(-w.L // TILE)
+    TILE_ = tile
+    L, T = w.L, -(-w.L // TILE_)
     out = np.zeros((w.B, T, T), np.int64)
     i = np.arange(L)[:, None]
     j = np.arange(L)[None, :]
@@ -559,9 +578,9 @@ def block_pair_counts(w):
             act = act & (j <= i) & ((j == 0) | (i - j <= w.window))
         elif w.causal:
             act = act & (j <= i)
-        pad = np.zeros((T * TILE, T * TILE), np.int64)
+        pad = np.zeros((T * TILE_, T * TILE_), np.int64)
         pad[:L, :L] = act
-        out[b] = pad.reshape(T, TILE, T, TILE).sum((1, 3))
+        out[b] = pad.reshape(T, TILE_, T, TILE_).sum((1, 3))
     return out
 
 
