@@ -54,6 +54,8 @@ def _load():
         lib.orc_tau_sort.restype = d_
         lib.orc_tau_bisect.argtypes = [dp, i, d_, i]
         lib.orc_tau_bisect.restype = d_
+        lib.orc_tau_hist.argtypes = [dp, i, d_, i]
+        lib.orc_tau_hist.restype = d_
         lib.orc_entmax_rows.argtypes = [dp, ctypes.c_long, i, ctypes.c_long, d_, i, dp, dp]
         lib.orc_entmax_rows.restype = None
         shape = [i, i, i, i, d_, d_, i, i, ip, dp]   # ..., kv_len, alibi slopes
@@ -110,6 +112,14 @@ def tau_bisect(z, alpha: float, iters: int = 200) -> float:
     """Bisection on Eq. 4 over the §2.4 bracket (any alpha > 1)."""
     z = _f64(z).ravel()
     return float(_load().orc_tau_bisect(_p(z), z.size, float(alpha), int(iters)))
+
+
+def tau_hist(z, alpha: float, bins: int) -> float:
+    """Histogram initialisation of tau (AdaSplash-2 §3.1, Appendix C.3) on z = (alpha-1) s:
+    the root of Eq. 4 with every score replaced by the left edge of its bin (B bins over the
+    shifted range [0, 1]); Proposition 3.1 bounds it by tau* - 1/B < tau_h <= tau*."""
+    z = _f64(z).ravel()
+    return float(_load().orc_tau_hist(_p(z), z.size, float(alpha), int(bins)))
 
 
 def entmax_rows(S, alpha: float, method: int = METHOD_AUTO):

@@ -19,6 +19,8 @@
  *   - same page, Appendix C.4: bit-packed block mask, 32 column blocks per uint32.
  *   - "Hooshaai/gpt2-adasplash-attention" model card, "Causal Splash Masking with
  *     Sink Preservation": active set {0} U {j <= i : i - j <= W}.
+ *   - "AdaSplash-2", §3.1 and Appendix C.3: the histogram initialisation of tau
+ *     (orc_tau_hist), with Proposition 3.1's bound tau* - 1/B < tau_h <= tau*.
  *   - "AdaSplash-2", §4.3: NAPE gives half of the heads no positional encoding and half
  *     ALiBi (Press et al.), a per-head linear penalty on the scores by query-key distance:
  *     s_ij = scale q_i . k_j - m_h |i - j| (m_h = 0 for a head without it).
@@ -121,6 +123,65 @@ double orc_tau_bisect(const double *z, int n, double alpha, int iters) {
         if (orc_f(z, n, alpha, mid) > 0) lo = mid; else hi = mid;
     }
     return 0.5 * (lo + hi);
+}
+
+/* Histogram initialisation of tau ("AdaSplash-2", §3.1 and Appendix C.3), for any alpha > 1.
+ * z = (alpha-1) s for the n active entries (Eq. 3 units). The scores are shifted so that
+ * the largest is 1 (z~ = z - (m - 1), m = max z), and each z~ in [0, 1] goes to bin
+ * b = min(floor(B z~), B - 1), whose left edge k/B stands in for it: the histogram
+ * objective is f_h(t) = -1 + sum_k H_k [k/B - t]_+^{1/(alpha-1)}. Entries with z~ < 0 are
+ * left out: their edges lie at or below -1/B, and the root tau_h of f_h lies above -1/B
+ * (Proposition 3.1: tau* - 1/B < tau_h <= tau*, with tau* >= 0 in shifted units).
+ * tau_h is found on the bins: for alpha in {1.5, 2} the exact solve of §2.4 with each bin
+ * counted H_k times (the support is a run of top bins), otherwise bisection of f_h over
+ * [-1/B, 1] (200 halvings). Returns tau_h in Eq. 3 units, or NAN if B < 1 or n < 1. */
+double orc_tau_hist(const double *z, int n, double alpha, int B) {
+    if (n < 1 || B < 1) return NAN;
+    double m = -INFINITY;
+    for (int j = 0; j < n; ++j) m = z[j] > m ? z[j] : m;
+    double *H = (double *)calloc((size_t)B, sizeof(double));
+    for (int j = 0; j < n; ++j) {
+        const double zt = z[j] - (m - 1.0);
+        if (zt < 0) continue;
+        int b = (int)floor(B * zt);
+        if (b > B - 1) b = B - 1;
+        H[b] += 1.0;
+    }
+    double t = NAN;
+    if (alpha == 2.0 || alpha == 1.5) {
+        double S0 = 0, S1 = 0, S2 = 0;
+        for (int k = B - 1; k >= 0; --k) {   /* top bins first */
+            if (H[k] == 0) continue;
+            const double e = (double)k / B;
+            S0 += H[k];
+            S1 += H[k] * e;
+            S2 += H[k] * e * e;
+            double tk;
+            if (alpha == 2.0) {
+                tk = (S1 - 1.0) / S0;
+            } else {
+                const double disc = S1 * S1 - S0 * (S2 - 1.0);
+                if (disc < 0) continue;
+                tk = (S1 - sqrt(disc)) / S0;
+            }
+            if (tk < e) t = tk;   /* every bin of this run lies above tk */
+        }
+    } else {
+        const double ex = 1.0 / (alpha - 1.0);
+        double lo = -1.0 / B, hi = 1.0;
+        for (int it = 0; it < 200; ++it) {
+            const double mid = 0.5 * (lo + hi);
+            double f = -1.0;
+            for (int k = 0; k < B; ++k) {
+                const double u = (double)k / B - mid;
+                if (u > 0 && H[k] > 0) f += H[k] * pow(u, ex);
+            }
+            if (f > 0) lo = mid; else hi = mid;
+        }
+        t = 0.5 * (lo + hi);
+    }
+    free(H);
+    return t + (m - 1.0);
 }
 
 /* One row of alpha-entmax on raw scores s (entries equal to -inf are inactive).

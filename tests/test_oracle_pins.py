@@ -406,3 +406,63 @@ def test_alibi_block_mask_brute_force():
             for jt in range(-(-L // Bc)):
                 want = (P[it * Br:(it + 1) * Br, jt * Bc:(jt + 1) * Bc] > 0).any()
                 assert bool((M[0, h, it, jt // 32] >> (jt % 32)) & 1) == want
+
+
+# ---------------------------------------------------------------- histogram initialisation
+def _hist_root_brute(z, alpha, B):
+    """The root of the histogram objective of AdaSplash-2 §3.1, written out directly: shift
+    so that max z = 1, replace each score in [0, 1] by the left edge of its bin
+    min(floor(B z), B - 1) / B, and bisect f_h(t) = -1 + sum [edge - t]_+^{1/(alpha-1)}."""
+    z = np.asarray(z, dtype=np.float64)
+    m = z.max()
+    zt = z - (m - 1.0)
+    zt = zt[zt >= 0]
+    edges = np.minimum(np.floor(B * zt), B - 1) / B
+    e = 1.0 / (alpha - 1.0)
+    lo, hi = -1.0 / B, 1.0
+    for _ in range(200):
+        mid = 0.5 * (lo + hi)
+        f = -1.0 + np.sum(np.clip(edges - mid, 0.0, None) ** e)
+        lo, hi = (mid, hi) if f > 0 else (lo, mid)
+    return 0.5 * (lo + hi) + (m - 1.0)
+
+
+@pytest.mark.parametrize("alpha", [1.25, 1.5, 2.0, 3.0])
+@pytest.mark.parametrize("B", [4, 8, 16, 64])
+def test_histogram_bound_proposition(alpha, B):
+    """Proposition 3.1 (AdaSplash-2 §3.2): tau* - 1/B <= tau_h <= tau*, on rows of several
+    sizes and spreads, with tau* from the exact solvers of §2.4 (a different algorithm).
+    The page states the left inequality strictly, but its proof needs z < edge + 1/B for
+    every score, which fails for the row maximum: the clamp min(floor(B z), B - 1) puts
+    z = 1 exactly 1/B above its edge. When the support is that maximum alone (a dominant
+    key), tau_h = tau* - 1/B; otherwise the inequality is strict."""
+    rng = np.random.default_rng(11)
+    for n in (1, 2, 7, 64, 4096):
+        for spread in (0.05, 0.5, 3.0):
+            z = (alpha - 1.0) * rng.normal(size=n) * spread
+            ts = oracle.tau_sort(z, alpha) if alpha in (1.5, 2.0) else oracle.tau_bisect(z, alpha)
+            th = oracle.tau_hist(z, alpha, B)
+            assert ts - 1.0 / B - 1e-12 <= th <= ts + 1e-12, (n, spread, ts, th)
+            single = np.sum(z > ts + 1e-12) <= 1   # support = the maximum alone
+            if not single:
+                assert ts - 1.0 / B < th, (n, spread, ts, th)
+
+
+@pytest.mark.parametrize("alpha", [1.25, 1.5, 2.0, 3.0])
+def test_histogram_solve_matches_brute_force(alpha):
+    """The oracle's exact solve on bin counts (α in {1.5, 2}) or bisection on bins gives the
+    root of the histogram objective computed directly from the binned scores."""
+    rng = np.random.default_rng(5)
+    for n, B in ((3, 4), (50, 8), (1000, 16), (4096, 8)):
+        z = rng.normal(size=n) * 0.7
+        assert abs(oracle.tau_hist(z, alpha, B) - _hist_root_brute(z, alpha, B)) < 1e-9
+
+
+def test_histogram_converges_with_bins():
+    """tau_h -> tau* as B grows (error below 1/B for B up to 2^14)."""
+    rng = np.random.default_rng(3)
+    z = 0.5 * rng.normal(size=2000)
+    ts = oracle.tau_sort(z, 1.5)
+    for k in range(2, 15):
+        B = 2 ** k
+        assert 0.0 <= ts - oracle.tau_hist(z, 1.5, B) < 1.0 / B
