@@ -14,9 +14,10 @@
 // tensor cores compute S = Q_i K_j^T and dA = dO_i V_j^T into TMEM (M = queries).
 // Warps 0-15 are row owners: warp w reads TMEM lanes 32(w%4)..+31 (one query row per
 // lane) and the columns of keys [32(w/4), 32(w/4)+32), so four threads share a row and
-// four warps share each SM sub-partition, which hides the latency of forming A and dS. Once a warp holds its S and dA
-// values in registers it releases them, so the MMA warp computes S and dA of the next
-// query tile while the row owners form A and dS. Both go to swizzled shared-memory
+// four warps share each SM sub-partition, which hides the latency of forming A and dS.
+// A warp reads its S and dA in two halves of 16 columns (fewer live registers) and
+// releases them after the second, so the MMA warp computes S and dA of the next query
+// tile while the row owners finish forming A and dS. Both go to swizzled shared-memory
 // buffers: A in fp16 (with the fp16 copy of dO; 2^-11 rounding), dS as a two-term
 // bf16 split (hi + lo, about fp32 accuracy in its products). A single 16-bit dS costs
 // too much in dK at large query variance. Those buffers then feed dV += A^T dO_i and
@@ -29,6 +30,8 @@
 // warp 18 the dV and dK chains: one thread issues an N=64 MMA only every ~54 cycles, so
 // the 40 MMAs of a tile's gradient products are split between two issuers.
 // TMEM: [0,128) S, [128,256) dA, [256,320) dV, [320,384) dK, [384,512) dQ x2.
+// With the 64 x 64 mask (kM64) the MMA warps leave out the dQ steps of a 64-key half and
+// the dV/dK steps of a 64-query half that hold no nonzero weight.
 #include "common.cuh"
 #include "kernels.h"
 

@@ -11,27 +11,33 @@
 //     tau_T <= tau* (entmax on a subset of the scores has fewer nonnegative terms in
 //     Eq. 4). It plays the role the paper gives its on-chip histogram (Phase 2), without
 //     an extra pass over K.
-//   Phase 3 (refinement): a sweep at tau copies every score with u = z - tau > 0 into
-//     shared memory (32 per row and column part, 128 per row). While tau <= tau*
-//     (f(tau) >= 0, true at tau_T) those copies hold the whole support, so a row whose
-//     copies fit is solved exactly on chip: safeguarded Newton on Eq. 4 (§3.2), finished
-//     by the exact root of the current support's piece (alpha = 2: (S1-1)/C; alpha =
-//     1.5: the smaller root of C d^2 - 2 S1 d + S2 - 1 = 0) once no candidate leaves the
-//     support. The first sweep runs at tau_T and only collects; a row whose copies
-//     overflow sweeps again, now also accumulating S1 = sum u, S2 = sum u^2 and the count
-//     for a Newton step bracketed by §2.4. Eq. 4's f is convex and decreasing in tau, so a
-//     Newton step from tau <= tau* stays <= tau*, and the next sweep's copies (fewer,
-//     above a higher tau) again qualify.
+//   Phase 3 and 4 fused (alpha 1.5 and 2): one output pass at tau_T over the key tiles
+//     where some row has a score above tau_T. Per tile the row owners copy every score
+//     with u_T = z - tau_T > 0 (score and key index) into shared memory (32 per row and
+//     column part, 128 per row), and write A_T = u_T^{1/(alpha-1)} in fp16 (2^-11
+//     rounding; bf16 would give 2^-8) into TMEM over the S columns they have read; the
+//     tensor cores accumulate O_T = sum A_T V with the A operand read from TMEM and B an
+//     fp16 copy of V. Since tau_T <= tau*, the copies hold the whole support, so a row
+//     whose copies fit is solved exactly on chip (four lanes of one warp per row):
+//     safeguarded Newton on Eq. 4 (§3.2), finished by the exact root of the current
+//     support's piece (alpha = 2: (S1-1)/C; alpha = 1.5: the smaller root of
+//     C d^2 - 2 S1 d + S2 - 1 = 0) once no candidate leaves the support. Every key with
+//     u_T > 0 lies in a visited tile, so the epilogue turns O_T into O at the final tau by
+//     adding sum_j (A*_j - fp16(A_T,j)) V_j over the copies in fp32 (A* = 0 outside the
+//     support): the result is the support sum with A* in fp32.
+//   Fallback: a row whose copies overflow sweeps again (S only), accumulating S1 = sum u,
+//     S2 = sum u^2 and the count for a Newton step bracketed by §2.4. Eq. 4's f is convex
+//     and decreasing in tau, so a Newton step from tau <= tau* stays <= tau*, and the
+//     next sweep's copies (fewer, above a higher tau) again qualify. The query tile then
+//     takes an output pass at the final tau over its flagged tiles, which recomputes O.
+//     The run-time alpha variant always takes a collecting sweep and then this output
+//     pass.
 //   Block mask: bit (query tile, key tile) = some row has a key-tile max above its
 //     final tau. Packed 32 key tiles per uint32 (Appendix C.4), plus the transpose for
-//     the backward.
-//   Phase 4 (output): only the flagged key tiles. Recompute S, form A = u^{1/(alpha-1)}
-//     in fp16 (2^-11 rounding; bf16 would give 2^-8) over the S columns it replaces, and
-//     compute O += A V on the tensor cores with the A operand read from TMEM and B an fp16
-//     copy of V. The backward's delta = sum_j g_ij dO_i . V_j / sum_j g_ij needs the
-//     support of each row, not a g V product: the row owners list every key with u > 0
-//     (index and u) per row and column part, and a small kernel of the backward sums over
-//     those lists in fp32.
+//     the backward; with the 64 x 64 variant also the mask at 64 x 64 blocks.
+//   Epilogue: the backward's delta = sum_j g_ij dO_i . V_j / sum_j g_ij needs sum g V and
+//     sum g over each row's support; a row solved on its copies has its support listed,
+//     and the epilogue sums over it in fp32, gathering the bf16 V rows.
 //
 // Roles (640 threads): warps 0-15 are row owners. Warp w reads TMEM lanes 32(w%4)..+31
 // (one query row per lane) and columns [32(w/4), 32(w/4)+32) of every S tile, so four
@@ -40,9 +46,11 @@
 // 4-slot ring of 16 KB K/V tiles. Warps 17 and 18 issue the S = Q K^T MMAs of the max pass
 // and the sweeps, alternating tiles (one thread blocks while its MMAs enter the tensor
 // pipe, so two issuers keep the pipe fed while each probes barriers and commits); warp 17
-// owns TMEM and issues the output pass's S tiles, and warp 19 the O = A V chain.
-// TMEM (512 columns): during the sweeps, four S buffers at 0/128/256/384, so the issuers
-// run up to three tiles ahead. During the output pass (OutLayout):
+// owns TMEM and issues the S tiles of the output-type passes (fused or final), and warp
+// 19 the O = A V chain.
+// TMEM (512 columns): during the max pass and the sweeps, four S buffers at
+// 0/128/256/384, so the issuers run up to three tiles ahead. During an output-type pass
+// (OutLayout):
 //   - three S buffers at 0, 128 and 384, tile k in buffer k % 3. The row owner of keys
 //     [32q, 32q+32) writes their A (fp16 pairs) into columns [32q, 32q+16): only over S
 //     columns it has read itself;
