@@ -30,10 +30,13 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("mask64", [True, False], ids=["mask64", "default"])
 @pytest.mark.parametrize("w,alpha", CASES, ids=[f"{w.name}-a{a}" for w, a in CASES])
-def test_alibi(w, alpha):
+def test_alibi(w, alpha, mask64):
+    """Each case in both kernel variants: with the 64 x 64 mask (checked bit for bit) and
+    the default kernels."""
     rep = {}
-    compare(w, alpha, backward=True, report=rep)
+    compare(w, alpha, backward=True, report=rep, mask64=mask64)
     print(w.name, alpha, {k: (float(v) if not isinstance(v, int) else v) for k, v in rep.items()})
 
 

@@ -33,8 +33,10 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("mask64", [True, False], ids=["mask64", "default"])
 @pytest.mark.parametrize("w,alpha,backward", CASES, ids=[f"{w.name}-a{a}" for w, a, _ in CASES])
-def test_general_alpha(w, alpha, backward):
+def test_general_alpha(w, alpha, backward, mask64):
+    """Each case in both kernel variants (with and without the 64 x 64 mask)."""
     rep = {}
-    compare(w, alpha, backward=backward, report=rep)
+    compare(w, alpha, backward=backward, report=rep, mask64=mask64)
     print(w.name, alpha, {k: (float(v) if not isinstance(v, int) else v) for k, v in rep.items()})

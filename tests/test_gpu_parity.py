@@ -284,3 +284,18 @@ def test_backward_counters():
     assert (bst[:, 2:6].sum(1) <= bst[:, 1]).all()
     fst = st.cpu().numpy().reshape(-1, eb.FWD_STATS).astype(np.int64)
     assert (fst[:, 4:7].sum(1) <= fst[:, 7]).all() and (fst[:, 7] > 0).all()
+
+
+@pytest.mark.parametrize("alpha", [1.5, 2.0])
+def test_mask64_variant_matches_default(alpha):
+    """The 64 x 64 variant only adds the finer mask and leaves out MMA steps whose products
+    are exactly zero, so O, tau, dK and dV are bit-identical to the default kernels' (dQ is
+    a sum of reduce-adds in no fixed order, so it is compared to fp32 rounding)."""
+    w = small_case("peaked_causal_L520", L=520, causal=True, sigma_q=3.0)
+    inp = make_inputs(w, seed=4)
+    a = gpu_run(inp, w, alpha, backward=True, mask64=False)
+    b = gpu_run(inp, w, alpha, backward=True, mask64=True)
+    for k in ("O", "tau", "dK", "dV"):
+        assert np.array_equal(a[k], b[k]), k
+    assert np.abs(a["dQ"] - b["dQ"]).max() <= 1e-5
+    assert np.array_equal(a["M"], b["M"])
