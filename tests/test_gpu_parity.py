@@ -10,9 +10,9 @@ import torch
 
 import oracle
 from entmax_sm_attention_b200 import binding as eb
-from entmax_sm_attention_b200.workloads import make_score_rows, small_case
+from entmax_sm_attention_b200.workloads import make_inputs, make_score_rows, small_case
 
-from parity import TOL_TAU, compare
+from parity import TOL_TAU, compare, gpu_run
 
 pytestmark = pytest.mark.gpu
 
