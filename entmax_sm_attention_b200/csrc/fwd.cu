@@ -941,15 +941,16 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       // The fused pass's O is final when every row was solved on that pass's copies.
       const bool o_final = AK != kAlphaGen && r == 1 && final_mask &&
                            !rows_any(valid && !listed, sh.votes, kMaxVotes - 1, lane, kMathThreads);
-      if (qp == 0) {
-        // Tiles that some row still needs (refinement) or that hold a nonzero (mask): each
-        // warp builds a word of 32 tile bits from eight independent loads and votes per
-        // step, and ORs it into the list once.
+      {
+        // Tiles that some row still needs (refinement) or that hold a nonzero (mask): the
+        // warps of column part qp take the groups of eight tiles 8 g with g % 4 == qp (the
+        // four warps of a part cover all 128 rows); each builds its bits from eight
+        // independent loads and votes per group and ORs them into the list once per word.
         const bool take = final_mask ? valid : !done;
         for (int w = 0; w < kMaskWords; ++w) {
           if (act[w] == 0) continue;
           uint32_t word = 0;
-          for (int b0 = 0; b0 < 32 && w * 32 + b0 < p.Tc; b0 += 8) {
+          for (int b0 = 8 * qp; b0 < 32 && w * 32 + b0 < p.Tc; b0 += 8 * kParts) {
             const int jb = w * 32 + b0;
             float v[8];
 #pragma unroll
