@@ -453,6 +453,7 @@ def run_ours(args):
     }
     if rank == 0 and world == 1 and not args.no_sweeps:
         result["detail"]["sparsity_sweeps"] = sparsity_sweeps(w, alpha, dev)
+        result["detail"]["variants"] = variant_points(w, dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, cores, sample, osp, _ = cpu_oracle_sample(w, alpha, args.seed, args.cpu_seconds, inp=host)
         result["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
@@ -538,6 +539,58 @@ def sparsity_sweeps(w, alpha, dev, steps: int = 10):
         sigma.append(r)
     return {"planted_rho": planted, "iid_sigma_q": sigma, "marginal": marginal_throughput(planted),
             "note": "same shape as the timed workload; planted inputs are a builder-added family"}
+
+
+def variant_points(w, dev, steps: int = 10) -> list:
+    """The timed workload's shape and inputs through the other kernel variants: the run-time
+    alpha kernels (alpha 1.25 and 1.75; alpha 2 has its own closed forms) and ALiBi on every
+    head (AdaSplash-2 §4.3's NAPE heads) with the geometric slopes 2^(-8 h / H) of Press et
+    al., h = 1..H, at alpha 1.5. Per point: 2 warm-up and `steps` timed forward+backward
+    steps, L2 flushed before each; times, block sparsity and algorithmic TFLOP/s."""
+    import torch
+
+    from entmax_sm_attention_b200 import binding as eb
+    from entmax_sm_attention_b200.workloads import make_inputs
+
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    d = {k: v.to(dev) for k, v in make_inputs(w, seed=0).items()}
+    shp = (w.B, w.H, w.L, w.d)
+    O = torch.empty(shp, dtype=torch.float32, device=dev)
+    tau = torch.empty(shp[:3], dtype=torch.float32, device=dev)
+    dQ, dK, dV = (torch.empty(shp, dtype=torch.float32, device=dev) for _ in range(3))
+    slopes = torch.tensor([2.0 ** (-8.0 * (h + 1) / w.H) for h in range(w.H)], dtype=torch.float32, device=dev)
+    out = []
+    for name, alpha, alibi in (("alpha_1.25", 1.25, None), ("alpha_1.75", 1.75, None), ("alpha_2", 2.0, None),
+                               ("alibi_geometric_alpha_1.5", 1.5, slopes)):
+        desc = eb.make_desc(w.B, w.H, w.L, w.d, alpha=alpha, scale=w.scale, causal=w.causal, window=w.window,
+                            alibi=alibi)
+        ws = eb.alloc_workspace(desc, dev)
+        fwd, bwd = [], []
+        for k in range(2 + steps):
+            flush.zero_()
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            e[0].record(stream)
+            eb.entmax_attn_fwd(desc, d["Q"], d["K"], d["V"], O, tau, ws, stream)
+            e[1].record(stream)
+            eb.entmax_attn_bwd(desc, d["Q"], d["K"], d["V"], d["dO"], tau, ws, dQ, dK, dV, stream)
+            e[2].record(stream)
+            torch.cuda.synchronize(dev)
+            if k >= 2:
+                fwd.append(e[0].elapsed_time(e[1]))
+                bwd.append(e[1].elapsed_time(e[2]))
+        code, _ = eb.entmax_last_device_status(desc, ws, stream)
+        M, st = eb.block_mask((desc, ws))
+        work = pair_work(w, M.cpu(), st.cpu())
+        st = st.cpu().long()
+        f_ms, b_ms = statistics.mean(fwd), statistics.mean(bwd)
+        out.append({"variant": name, "alpha": alpha, "status": eb.STATUS_NAMES[code],
+                    "block_sparsity_128": 1.0 - float(st[..., 2].sum()) / max(1, int(st[..., 3].sum())),
+                    "refine_sweeps_mean": float(st[..., 0].float().mean()),
+                    "fwd_ms": f_ms, "bwd_ms": b_ms, "ms": f_ms + b_ms,
+                    "tflops_fwd_algorithmic": work["fwd_flops"] / (f_ms * 1e-3) / 1e12,
+                    "tflops_bwd_algorithmic": work["bwd_flops"] / (b_ms * 1e-3) / 1e12})
+    return out
 
 
 def marginal_throughput(points) -> dict:

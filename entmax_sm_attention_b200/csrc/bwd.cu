@@ -367,11 +367,12 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
               ah[e] = pack_f16(v0, v1);
               split_bf16x2(u.x > 0.f ? d.x : 0.f, u.y > 0.f ? d.y : 0.f, dh[e], dl2[e]);
             } else {
-              // A = u^e and g = u^{e-1} from one logarithm each.
+              // g = u^{e-1} from one logarithm and one power, and A = u^e = g u (two
+              // special-function operations per score instead of three).
               const float l0 = __log2f(u.x > 0.f ? u.x : 1.f), l1 = __log2f(u.y > 0.f ? u.y : 1.f);
-              const float a0 = u.x > 0.f ? exp2f(p.ae * l0) : 0.f, a1 = u.y > 0.f ? exp2f(p.ae * l1) : 0.f;
               const float g0 = u.x > 0.f ? exp2f((p.ae - 1.f) * l0) : 0.f;
               const float g1 = u.y > 0.f ? exp2f((p.ae - 1.f) * l1) : 0.f;
+              const float a0 = g0 * v0, a1 = g1 * v1;
               ah[e] = pack_f16(a0, a1);
               split_bf16x2(g0 * d.x, g1 * d.y, dh[e], dl2[e]);
             }
